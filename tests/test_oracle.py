@@ -1,0 +1,266 @@
+"""Pins for the fp64 oracle: properties the mathematics fixes, checked on the CPU.
+
+Each test checks the oracle against something other than itself: a library
+matmul on the merged weight, closed forms, invariants, exact finite
+differences, or a hand-derived example.  A dropped term, a wrong sign, a wrong
+index or a transposed operand anywhere in ``oracle.c`` fails at least one.
+"""
+import dataclasses
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import plora_workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def small(seed, dtype="fp32", d_in=24, d_out=20, ranks=(1, 3, 8, 5), counts=(7, 0, 12, 5)):
+    r = np.asarray(ranks)
+    return wl.make_problem("small", dtype, d_in, d_out, r, counts, 2.0 * r + 1.0,
+                           wl.init_small(d_in), seed)
+
+
+def f64(p, a):
+    return wl.to_f64(a, p.dtype)
+
+
+def merged_reference(p):
+    """Y and dX through the merged weight W_eff = W + s_i A_i B_i, one library matmul per segment.
+    Merging the low-rank patch into the base weight gives the full weight ('LLM+LoRA微调加速技术原理解析',
+    深入理解LoRA：基本原理与PEFT实现: the released LoRA weight is a patch merged into the original)."""
+    Wt = f64(p, p.W).T                      # W[j][c]
+    Y = np.zeros((p.T, p.d_out))
+    dX = np.zeros((p.T, p.d_in))
+    X, dY = f64(p, p.X), f64(p, p.dY)
+    for i in range(p.n_adapters):
+        a, b = p.off[i], p.off[i + 1]
+        A = f64(p, p.A[i]).T                # A_i[j][k]
+        B = f64(p, p.B[i]).T                # B_i[k][c]
+        Weff = Wt + float(p.scales[i]) * (A @ B)
+        Y[a:b] = X[a:b] @ Weff
+        dX[a:b] = dY[a:b] @ Weff.T
+    return Y, dX
+
+
+def rel(a, b):
+    den = np.max(np.abs(b)) if np.size(b) else 0.0
+    return float(np.max(np.abs(a - b)) / den) if den > 0 else float(np.max(np.abs(a - b), initial=0.0))
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_forward_and_input_grad_match_merged_weight(seed, dtype):
+    p = small(seed, dtype)
+    Y, dX = merged_reference(p)
+    o = oracle.forward(p)
+    g = oracle.input_grad(p)
+    assert rel(o["Y"], Y) < 1e-12
+    assert rel(g["dX"], dX) < 1e-12
+
+
+def test_config1_matches_merged_weight():
+    p = wl.config1()
+    Y, dX = merged_reference(p)
+    assert rel(oracle.forward(p)["Y"], Y) < 1e-12
+    assert rel(oracle.input_grad(p)["dX"], dX) < 1e-12
+
+
+def test_hand_derived_integer_example():
+    g = json.load(open(os.path.join(GOLDEN, "tiny_integer_example.json")))
+    r = np.asarray(g["ranks"], dtype=np.int32)
+    al = np.asarray(g["alphas"], dtype=np.float64)
+    p = wl.Problem("golden", "fp32", g["d_in"], g["d_out"], np.asarray(g["off"], dtype=np.int64), r, al,
+                   (al / r).astype(np.float32), np.asarray(g["X"], np.float32),
+                   np.asarray(g["W_store"], np.float32), [np.asarray(a, np.float32) for a in g["A_store"]],
+                   [np.asarray(b, np.float32) for b in g["B_store"]], np.asarray(g["dY"], np.float32))
+    o = oracle.full(p)
+    e = g["expect"]
+    assert np.array_equal(o["Y"], np.asarray(e["Y"], float))
+    assert np.array_equal(o["dX"], np.asarray(e["dX"], float))
+    for i in range(2):
+        assert np.array_equal(o["dA"][i], np.asarray(e["dA_store"][i], float))
+        assert np.array_equal(o["dB"][i], np.asarray(e["dB_store"][i], float))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_B_zero_gives_base_exactly_and_zero_dA(dtype):
+    """B = 0 (the LoRA init of B): Y = X W exactly, dA = 0 exactly, dB = s H^T dY."""
+    p = wl.with_zero_B(small(11, dtype))
+    q = dataclasses.replace(p, A=[np.zeros_like(a) for a in p.A])     # branch removed another way
+    o, oq = oracle.full(p), oracle.full(q)
+    assert np.array_equal(o["Y"], oq["Y"])
+    assert np.array_equal(o["dX"], oq["dX"])
+    base = f64(p, p.X) @ f64(p, p.W).T
+    assert rel(o["Y"], base) < 1e-12
+    assert rel(o["dX"], f64(p, p.dY) @ f64(p, p.W)) < 1e-12
+    X, dY = f64(p, p.X), f64(p, p.dY)
+    for i in range(p.n_adapters):
+        assert not np.any(o["dA"][i])
+        a, b = p.off[i], p.off[i + 1]
+        H = X[a:b] @ f64(p, p.A[i]).T
+        dB = float(p.scales[i]) * (dY[a:b].T @ H)
+        assert rel(o["dB"][i], dB) < 1e-12 or (b == a and not np.any(o["dB"][i]))
+
+
+def test_rank1_outer_product_closed_forms():
+    """Rank 1: A = a, B = b^T.  Y - XW = s (X a) b^T; dB = s dY^T (X a); dA = s X^T (dY b)."""
+    p = small(21, "fp32", ranks=(1, 1, 1), counts=(9, 4, 6))
+    o = oracle.full(p)
+    pb = wl.with_zero_B(p)
+    base = oracle.forward(pb)["Y"]
+    base_dx = oracle.input_grad(pb)["dX"]
+    X, dY = f64(p, p.X), f64(p, p.dY)
+    for i in range(3):
+        a, b = p.off[i], p.off[i + 1]
+        av = f64(p, p.A[i])[0]              # a[j]
+        bv = f64(p, p.B[i])[:, 0]           # b[c]
+        s = float(p.scales[i])
+        assert rel(o["Y"][a:b] - base[a:b], s * np.outer(X[a:b] @ av, bv)) < 1e-12
+        assert rel(o["dX"][a:b] - base_dx[a:b], s * np.outer(dY[a:b] @ bv, av)) < 1e-12
+        assert rel(o["dB"][i][:, 0], s * (dY[a:b].T @ (X[a:b] @ av))) < 1e-12
+        assert rel(o["dA"][i][0], s * (X[a:b].T @ (dY[a:b] @ bv))) < 1e-12
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_packed_equals_each_adapter_alone(dtype):
+    """Packing does not change any adapter's result: bit-exact in the oracle."""
+    p = small(31, dtype)
+    o = oracle.full(p)
+    for i in range(p.n_adapters):
+        a, b = int(p.off[i]), int(p.off[i + 1])
+        q = dataclasses.replace(p, off=np.array([0, b - a], np.int64), ranks=p.ranks[i:i + 1],
+                                alphas=p.alphas[i:i + 1], scales=p.scales[i:i + 1], X=p.X[a:b],
+                                A=[p.A[i]], B=[p.B[i]], dY=p.dY[a:b])
+        oq = oracle.full(q)
+        assert np.array_equal(oq["Y"], o["Y"][a:b])
+        assert np.array_equal(oq["dX"], o["dX"][a:b])
+        assert np.array_equal(oq["dA"][0], o["dA"][i])
+        assert np.array_equal(oq["dB"][0], o["dB"][i])
+
+
+def test_linear_in_scale():
+    """dA and dB scale exactly by 2 with s -> 2s; Y - XW and dX - dY W^T scale by 2 up to roundoff."""
+    p = small(41, "fp32")
+    q = dataclasses.replace(p, scales=(2 * p.scales).astype(np.float32))
+    o, oq = oracle.full(p), oracle.full(q)
+    for i in range(p.n_adapters):
+        assert np.array_equal(oq["dA"][i], 2 * o["dA"][i])
+        assert np.array_equal(oq["dB"][i], 2 * o["dB"][i])
+    pb = oracle.full(wl.with_zero_B(p))
+    assert rel(oq["Y"] - pb["Y"], 2 * (o["Y"] - pb["Y"])) < 1e-12
+    assert rel(oq["dX"] - pb["dX"], 2 * (o["dX"] - pb["dX"])) < 1e-12
+
+
+def _loss(p):
+    """L = <dY, Y>: its gradients are exactly dX, dA, dB."""
+    return float(np.sum(f64(p, p.dY) * oracle.forward(p)["Y"]))
+
+
+def test_gradients_match_central_finite_differences():
+    """L is linear in X, in A and in B separately, so the central difference with the
+    actually representable perturbation is exact up to fp64 roundoff."""
+    r = np.asarray([1, 2, 3])
+    p = wl.make_problem("fd", "fp32", 8, 6, r, [2, 0, 3], 2.0 * r + 1.0, wl.init_small(8), 51)
+    o = oracle.full(p)
+    h = np.float32(0.0625)
+
+    def fd(get, put, idx):
+        base = get()
+        up, dn = base.copy(), base.copy()
+        up[idx] = base[idx] + h
+        dn[idx] = base[idx] - h
+        put(up)
+        lp = _loss(p)
+        put(dn)
+        lm = _loss(p)
+        put(base)
+        return (lp - lm) / (float(up[idx]) - float(dn[idx]))
+
+    scale = max(np.max(np.abs(o["dX"])), 1.0)
+    for t in range(p.T):
+        for j in range(p.d_in):
+            g = fd(lambda: p.X, lambda v: setattr(p, "X", v), (t, j))
+            assert abs(g - o["dX"][t, j]) <= 1e-10 * scale
+    for i in range(p.n_adapters):
+        for k in range(int(r[i])):
+            for j in range(p.d_in):
+                g = fd(lambda: p.A[i], lambda v: p.A.__setitem__(i, v), (k, j))
+                assert abs(g - o["dA"][i][k, j]) <= 1e-10 * scale
+            for c in range(p.d_out):
+                g = fd(lambda: p.B[i], lambda v: p.B.__setitem__(i, v), (c, k))
+                assert abs(g - o["dB"][i][c, k]) <= 1e-10 * scale
+    assert not np.any(o["dA"][1]) and not np.any(o["dB"][1])      # the empty segment
+
+
+def signature_problem(counts, dtype="fp32", d_in=16, d_out=24, rank=3):
+    """Segment signature: W = 0, X[t][0] = 1, A_store_i[0][0] = 1, B_store_i[c][0] = 1, s_i = i + 1,
+    dY[t][0] = 1.  Then Y[t][c] = s_adapter(t), dB_store_i[0][0] = dA_store_i[0][0] = s_i n_i."""
+    n = len(counts)
+    off = np.zeros(n + 1, np.int64)
+    off[1:] = np.cumsum(counts)
+    T = int(off[-1])
+    one = wl.from_f64(np.ones(1), dtype)[0]
+    zero = wl.from_f64(np.zeros(1), dtype)[0]
+
+    def z(shape):
+        return np.full(shape, zero)
+    X = z((T, d_in)); X[:, 0] = one
+    dY = z((T, d_out)); dY[:, 0] = one
+    A, B = [], []
+    for i in range(n):
+        a = z((rank, d_in)); a[0, 0] = one; A.append(a)
+        b = z((d_out, rank)); b[:, 0] = one; B.append(b)
+    ranks = np.full(n, rank, np.int32)
+    scales = np.arange(1, n + 1, dtype=np.float32)
+    return wl.Problem("signature", dtype, d_in, d_out, off, ranks, scales.astype(np.float64) * rank,
+                      scales, X, z((d_out, d_in)), A, B, dY)
+
+
+def signature_expect(p):
+    seg = np.repeat(np.arange(p.n_adapters), p.counts)
+    Y = np.zeros((p.T, p.d_out))
+    Y[:, :] = (seg + 1)[:, None]
+    return Y
+
+
+def test_segment_signature_exact():
+    p = signature_problem([5, 1, 0, 9, 2])
+    o = oracle.full(p)
+    assert np.array_equal(o["Y"], signature_expect(p))
+    for i in range(p.n_adapters):
+        e = np.zeros_like(o["dB"][i]); e[0, 0] = (i + 1) * p.counts[i]
+        assert np.array_equal(o["dB"][i], e)
+        e = np.zeros_like(o["dA"][i]); e[0, 0] = (i + 1) * p.counts[i]
+        assert np.array_equal(o["dA"][i], e)
+
+
+def test_rows_api_matches_full_rows():
+    p = small(61, "bf16")
+    rows = np.array([0, 3, 6, 7, 18, 23], np.int64)
+    fo, fg = oracle.forward(p), oracle.input_grad(p)
+    so, sg = oracle.forward(p, rows=rows), oracle.input_grad(p, rows=rows)
+    assert np.array_equal(so["Y"], fo["Y"][rows])
+    assert np.array_equal(sg["dX"], fg["dX"][rows])
+    with pytest.raises(ValueError):
+        oracle.forward(p, rows=np.array([p.T], np.int64))
+
+
+def test_threads_do_not_change_results():
+    p = small(71, "bf16")
+    a, b = oracle.full(p, nthreads=1), oracle.full(p, nthreads=4)
+    assert np.array_equal(a["Y"], b["Y"]) and np.array_equal(a["dX"], b["dX"])
+    for i in range(p.n_adapters):
+        assert np.array_equal(a["dA"][i], b["dA"][i]) and np.array_equal(a["dB"][i], b["dB"][i])
+
+
+def test_input_rounding_is_round_to_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 3.0e-3], np.float32)
+    b = wl.f32_to_bf16_bits(x)
+    back = wl.bf16_bits_to_f32(b)
+    assert back[0] == 1.0 and back[1] == 1.0 and back[2] == 1.0 + 2 ** -6
+    assert back[3] == -2.5
+    assert abs(back[4] - 3.0e-3) <= 3.0e-3 * 2 ** -8
