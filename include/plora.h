@@ -1,0 +1,236 @@
+/*
+ * plora.h -- C ABI of the packed LoRA fine-tuning library for NVIDIA B200 (sm_100a).
+ *
+ * One call computes, for N LoRA adapters that share one frozen base projection
+ * W and own contiguous segments of one packed token buffer, the forward and
+ * the backward of the layer
+ *
+ *     Y_i  = X_i W + s_i (X_i A_i) B_i
+ *     dX_i = dY_i W^T + s_i (dY_i B_i^T) A_i^T
+ *     dB_i = s_i (X_i A_i)^T dY_i          (a sum over the tokens of adapter i)
+ *     dA_i = X_i^T (s_i dY_i B_i^T)        (a sum over the tokens of adapter i)
+ *
+ * where X_i are the rows off[i] .. off[i+1]-1 of X and s_i = alpha_i / r_i.
+ * The layer is LoRA's: a frozen W plus a trainable low-rank branch A then B
+ * whose output is scaled by alpha/r and added ("LLM+LoRA微调加速技术原理解析",
+ * m.youleyou.com, 深入理解LoRA：基本原理与PEFT实现); only A and B get gradients
+ * ("LoRA加速集成方案", cloud.baidu.com, 四、工作原理 › 3. 反向传播阶段).  Packing
+ * many adapters over one shared frozen base and batching their operators over
+ * the concatenated LoRA tensors, tiled along the sequence or hidden dimension
+ * rather than the rank, with load balancing across adapters of unequal rank
+ * and token count, is PLoRA's execution engine (PLoRA summary, gist.science,
+ * arXiv 2508.02932, 技术摘要 › 方法论 › 2. LoRA 执行引擎 › 打包 LoRA 算子,
+ * 算子设计).
+ *
+ * Layouts.  Every tensor is dense and row-major, in the PyTorch / PEFT module
+ * layouts, so that module parameters can be passed without copies:
+ *     X       [T][d_in]       packed tokens               (dtype)
+ *     W       [d_out][d_in]   nn.Linear.weight = W^T      (dtype)
+ *     A_i     [r_i][d_in]     lora_A.weight    = A_i^T    (dtype)
+ *     B_i     [d_out][r_i]    lora_B.weight    = B_i^T    (dtype)
+ *     Y, dY   [T][d_out]                                  (dtype)
+ *     dX      [T][d_in]                                   (dtype)
+ *     dA_i    [r_i][d_in],  dB_i [d_out][r_i]             (fp32)
+ * T = off[N].  dtype is bf16 (products accumulated in fp32, outputs rounded
+ * to nearest even) or fp32 (fp32 FMA throughout, no TF32).
+ *
+ * Ownership.  The caller owns every tensor.  A handle owns only its private
+ * workspace (device scratch, pinned host staging, a device error flag).
+ * `off` and the adapter table are HOST arrays, read during the call; every
+ * pointer inside them, and every tensor pointer, is a DEVICE pointer that
+ * must stay valid until the work enqueued on `stream` has run.
+ *
+ * Semantics.  Y, dX, dA_i and dB_i are overwritten, never accumulated into.
+ * An adapter with no tokens (off[i] == off[i+1]) gets dA_i = dB_i = 0.
+ * All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream); calls return once it is enqueued.
+ *
+ * Errors.  Every argument is checked before anything is enqueued; on an
+ * error nothing is written and the call returns a non-zero status, with a
+ * message available from plora_last_error().  No C++ exception crosses this
+ * ABI.  An asynchronous device failure surfaces as PLORA_ERR_CUDA from the
+ * call that observes it or from plora_check(); a device-side wait that ran
+ * out of time surfaces as PLORA_ERR_TIMEOUT from plora_check().
+ *
+ * Threading.  A handle runs one call at a time (its workspace is reused by
+ * the next call on the same stream); distinct handles are independent.
+ */
+#ifndef PLORA_H
+#define PLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PLORA_API __attribute__((visibility("default")))
+#else
+#define PLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PLORA_OK = 0,
+    PLORA_ERR_INVALID_ARG = 1,  /* a null/misaligned pointer, bad offsets, rank or count out of range */
+    PLORA_ERR_UNSUPPORTED = 2,  /* a shape or dtype the library does not handle */
+    PLORA_ERR_OOM = 3,          /* workspace allocation failed in plora_create */
+    PLORA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+    PLORA_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (see plora_check) */
+} plora_status;
+
+typedef enum {
+    PLORA_BF16 = 0,
+    PLORA_FP32 = 1
+} plora_dtype;
+
+/* plora_config.flags */
+enum {
+    PLORA_FLAG_SIMT = 1u  /* bf16 only: run the plain SIMT kernels instead of the tensor-core ones */
+};
+
+/* Limits. */
+#define PLORA_MAX_RANK 256
+#define PLORA_MAX_ADAPTERS 4096
+
+/*
+ * Handle configuration.  d_in, d_out: projection sizes, multiples of 8 in
+ * [8, 65536].  dtype: a plora_dtype.  max_adapters in [1, PLORA_MAX_ADAPTERS],
+ * max_rank in [1, PLORA_MAX_RANK], max_tokens >= 1: upper bounds of every
+ * later call, used to size the workspace.
+ */
+typedef struct {
+    int64_t d_in;
+    int64_t d_out;
+    int32_t dtype;
+    int32_t max_adapters;
+    int32_t max_rank;
+    uint32_t flags;
+    int64_t max_tokens;
+} plora_config;
+
+/*
+ * One adapter.  rank r in [1, max_rank]; scale = alpha / r as the caller
+ * computed it (finite); A: [r][d_in], B: [d_out][r] in the handle's dtype;
+ * dA: [r][d_in], dB: [d_out][r] in fp32 (written by plora_backward, ignored
+ * by plora_forward).  Every pointer 16-byte aligned.
+ */
+typedef struct {
+    int32_t rank;
+    float scale;
+    const void* A;
+    const void* B;
+    float* dA;
+    float* dB;
+} plora_adapter;
+
+typedef struct plora_ctx* plora_handle;
+
+/*
+ * Create a handle on the current CUDA device and allocate its workspace.
+ * Returns PLORA_ERR_INVALID_ARG / PLORA_ERR_UNSUPPORTED for a bad config,
+ * PLORA_ERR_OOM if the workspace cannot be allocated, PLORA_ERR_CUDA if no
+ * usable sm_100 device is current.  *out is NULL on failure.
+ */
+PLORA_API plora_status plora_create(plora_handle* out, const plora_config* cfg);
+
+/* Free the handle and its workspace (synchronises the device first). NULL is accepted. */
+PLORA_API plora_status plora_destroy(plora_handle h);
+
+/*
+ * Size in bytes of the `saved` buffer that plora_forward fills and
+ * plora_backward reads for this segment map and adapter table.  Its layout
+ * is the library's (per-adapter blocks of X_i A_i rows, padded); read it
+ * only through plora_debug_unpack_saved.
+ */
+PLORA_API plora_status plora_saved_bytes(plora_handle h, int32_t n_adapters, const int64_t* off,
+                               const plora_adapter* tab, size_t* bytes);
+
+/*
+ * Forward.  X: [T][d_in], W: [d_out][d_in], Y (out): [T][d_out], all device.
+ * n_adapters in [0, max_adapters]; off: host int64[n_adapters+1] with
+ * off[0] = 0, non-decreasing, off[n] <= max_tokens; tab: host
+ * plora_adapter[n_adapters].  saved (out): device buffer of
+ * plora_saved_bytes() bytes, 256-byte aligned, kept for plora_backward.
+ * When off[n] == 0 (no tokens), X, Y and saved may be NULL and nothing is written.
+ */
+PLORA_API plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y,
+                           int32_t n_adapters, const int64_t* off, const plora_adapter* tab,
+                           void* saved, void* stream);
+
+/*
+ * Backward.  Same X, W, off, tab and saved as the forward; dY: [T][d_out];
+ * dX (out, may be NULL to skip the input gradient): [T][d_in]; writes every
+ * adapter's dA and dB (which must be non-NULL).  When off[n] == 0, X, dY, dX
+ * and saved may be NULL and only the (zero) weight gradients are written.
+ */
+PLORA_API plora_status plora_backward(plora_handle h, const void* X, const void* W, const void* dY,
+                            void* dX, int32_t n_adapters, const int64_t* off,
+                            const plora_adapter* tab, const void* saved, void* stream);
+
+/*
+ * Synchronise `stream` and report the handle's device error flag: PLORA_OK,
+ * PLORA_ERR_TIMEOUT (a bounded device wait ran out; the flag is then
+ * cleared) or PLORA_ERR_CUDA.
+ */
+PLORA_API plora_status plora_check(plora_handle h, void* stream);
+
+/* Static text for a status code. */
+PLORA_API const char* plora_status_string(plora_status s);
+
+/* Detail text of the handle's last failure ("" if none; valid until the next call on h). */
+PLORA_API const char* plora_last_error(plora_handle h);
+
+/*
+ * Debug: copy adapter i's saved H_i = X_i A_i out of `saved` as fp32
+ * [n_i][r_i] into the device buffer H_out (16-byte aligned).
+ */
+PLORA_API plora_status plora_debug_unpack_saved(plora_handle h, int32_t n_adapters, const int64_t* off,
+                                      const plora_adapter* tab, const void* saved, int32_t i,
+                                      float* H_out, void* stream);
+
+/*
+ * Debug / testing: the schedule one call would run for this configuration,
+ * segment map and adapter table -- host logic only, no handle, no device.
+ * Checks the arguments like plora_forward (or plora_backward if grads != 0)
+ * and writes int32 records to out[0 .. capacity):
+ *   which = 0: token tiles, 4 per tile: adapter, rows (1..128), first token
+ *              row, first row in the saved H / workspace G buffers;
+ *   which = 1: weight-gradient splits, 8 per split: adapter, first token row,
+ *              first H/G row, 64-token blocks, split index, split count,
+ *              first partial slot (-1 if unsplit), first counter (-1);
+ *   which = 2: adapters, 5 per adapter: first token row, tokens, first H/G
+ *              row, rank rounded up to 16, rank rounded up to 64;
+ *   which = 3: two values: the padded rank pitch RP and the H/G row count.
+ * *count receives the number of int32 values the full answer needs.
+ */
+PLORA_API plora_status plora_debug_schedule(const plora_config* cfg, int32_t n_adapters, const int64_t* off,
+                                            const plora_adapter* tab, int32_t grads, int32_t which,
+                                            int32_t* out, int64_t capacity, int64_t* count);
+
+/*
+ * Profiling.  The handle always counts its kernel launches per kernel kind.
+ * With profiling enabled, it also brackets every launch with CUDA events on
+ * the launching stream and sums each kernel's device time.
+ */
+PLORA_API plora_status plora_profile_enable(plora_handle h, int32_t enable);
+
+/*
+ * Synchronise on the recorded events, then report, per kernel kind, the
+ * launches and the summed device milliseconds since the last read (and reset
+ * both).  *n_kinds receives the number of kinds; at most `capacity` entries
+ * of names (static strings), launches and total_ms (each may be NULL) are
+ * written.
+ */
+PLORA_API plora_status plora_profile_read(plora_handle h, int32_t capacity, int32_t* n_kinds,
+                                          const char** names, int64_t* launches, double* total_ms);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+PLORA_API int32_t plora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PLORA_H */

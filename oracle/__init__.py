@@ -54,7 +54,7 @@ def _load():
         _lib.oracle_input_grad.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, pp, pp, _P, i64, _P,
                                            _P, _P, i64, ci]
         _lib.oracle_weight_grads.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, pp, pp, _P, pp,
-                                             pp, ci]
+                                             pp, i64, _P, i64, _P, ci]
         for fn in ("oracle_forward", "oracle_input_grad", "oracle_weight_grads"):
             getattr(_lib, fn).restype = ctypes.c_int
         _lib.oracle_num_procs.restype = ctypes.c_int
@@ -136,20 +136,28 @@ def input_grad(p, rows: Optional[np.ndarray] = None, nthreads: int = 1, want_G: 
     return out
 
 
-def weight_grads(p, nthreads: int = 1) -> Dict[str, List[np.ndarray]]:
-    """dA_i ([r_i][d_in]) and dB_i ([d_out][r_i]) in float64 for every adapter."""
+def weight_grads(p, nthreads: int = 1, cols_a: Optional[np.ndarray] = None,
+                 cols_b: Optional[np.ndarray] = None) -> Dict[str, List[np.ndarray]]:
+    """dA_i ([r_i][d_in]) and dB_i ([d_out][r_i]) in float64 for every adapter.
+    With cols_a / cols_b, only those hidden columns of dA / rows of dB are computed
+    (the rest stay zero)."""
     lib = _load()
     off, rank, scale, A, B, Ap, Bp = _common(p)
     X = np.ascontiguousarray(p.X)
     dY = np.ascontiguousarray(p.dY)
     dA = [np.zeros((int(r), p.d_in), dtype=np.float64) for r in rank]
     dB = [np.zeros((p.d_out, int(r)), dtype=np.float64) for r in rank]
+    ca = None if cols_a is None else np.ascontiguousarray(cols_a, dtype=np.int64)
+    cb = None if cols_b is None else np.ascontiguousarray(cols_b, dtype=np.int64)
     dAp = (_P * max(1, len(dA)))(*[a.ctypes.data for a in dA])
     dBp = (_P * max(1, len(dB)))(*[b.ctypes.data for b in dB])
     lib.oracle_weight_grads(_dt(p), ctypes.c_int64(p.d_in), ctypes.c_int64(p.d_out),
                             ctypes.c_int32(p.n_adapters), off.ctypes.data, rank.ctypes.data,
                             scale.ctypes.data, X.ctypes.data, Ap, Bp, dY.ctypes.data,
-                            dAp, dBp, ctypes.c_int(nthreads))
+                            dAp, dBp,
+                            ctypes.c_int64(0 if cols_a is None else len(ca)), None if cols_a is None else ca.ctypes.data,
+                            ctypes.c_int64(0 if cols_b is None else len(cb)), None if cols_b is None else cb.ctypes.data,
+                            ctypes.c_int(nthreads))
     return {"dA": dA, "dB": dB}
 
 

@@ -180,13 +180,19 @@ int oracle_input_grad(int dtype, int64_t d_in, int64_t d_out, int32_t n, const i
  *   dB_i[k][c] = s_i sum_{t in seg i} H[t][k] dY[t][c]   stored dB_store_i[c][k]
  *   dA_i[j][k] =     sum_{t in seg i} X[t][j] G[t][k]    stored dA_store_i[k][j]
  * An adapter with no tokens gets zeros.  dA[i] is [r_i][d_in], dB[i] is
- * [d_out][r_i], both double.
+ * [d_out][r_i], both double.  If n_cols_a > 0, only the hidden columns
+ * j = cols_a[0..n_cols_a) of dA are computed (the others are left as they
+ * are); likewise cols_b for the rows c of dB.
  */
 int oracle_weight_grads(int dtype, int64_t d_in, int64_t d_out, int32_t n, const int64_t* off,
                         const int32_t* rank, const float* scale, const void* X,
                         const void* const* A, const void* const* B, const void* dY,
-                        double* const* dA, double* const* dB, int nthreads) {
+                        double* const* dA, double* const* dB, int64_t n_cols_a,
+                        const int64_t* cols_a, int64_t n_cols_b, const int64_t* cols_b,
+                        int nthreads) {
     set_threads(nthreads);
+    const int64_t na = n_cols_a > 0 ? n_cols_a : d_in;
+    const int64_t nb = n_cols_b > 0 ? n_cols_b : d_out;
     for (int32_t i = 0; i < n; ++i) {
         const int64_t t0 = off[i], nt = off[i + 1] - off[i];
         const int r = rank[i];
@@ -200,19 +206,23 @@ int oracle_weight_grads(int dtype, int64_t d_in, int64_t d_out, int32_t n, const
                 G[u * r + k] = g_elem(dtype, d_out, r, s, dY, B[i], t0 + u, k);
             }
 #pragma omp parallel for schedule(static)
-        for (int64_t c = 0; c < d_out; ++c)
+        for (int64_t q = 0; q < nb; ++q) {
+            const int64_t c = n_cols_b > 0 ? cols_b[q] : q;
             for (int k = 0; k < r; ++k) {
                 double acc = 0.0;
                 for (int64_t u = 0; u < nt; ++u) acc += H[u * r + k] * ld(dY, dtype, (t0 + u) * d_out + c);
                 dB[i][c * r + k] = s * acc;
             }
+        }
 #pragma omp parallel for schedule(static)
-        for (int64_t j = 0; j < d_in; ++j)
+        for (int64_t q = 0; q < na; ++q) {
+            const int64_t j = n_cols_a > 0 ? cols_a[q] : q;
             for (int k = 0; k < r; ++k) {
                 double acc = 0.0;
                 for (int64_t u = 0; u < nt; ++u) acc += ld(X, dtype, (t0 + u) * d_in + j) * G[u * r + k];
                 dA[i][(int64_t)k * d_in + j] = acc;
             }
+        }
         free(H);
         free(G);
     }

@@ -1,0 +1,288 @@
+"""Packed LoRA fine-tuning for NVIDIA B200 (sm_100a): Python binding of the C ABI.
+
+This module only marshals arguments into ``libplora.so`` (built from
+``csrc/`` by ``packed_lora_fine_b200.build``); every step of the computation
+runs in the library's CUDA kernels.  The functions keep the C names of
+``include/plora.h``: ``plora_create``, ``plora_forward``, ``plora_backward``,
+``plora_check``, ``plora_saved_bytes``, ``plora_debug_unpack_saved``,
+``plora_destroy``.  Tensors are passed as device pointers (ints); PyTorch is
+only a convenient owner of device memory and streams.
+
+There is no fallback: if the library is missing, importing the binding
+raises ``ImportError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Iterable, List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libplora.so")
+
+PLORA_OK = 0
+PLORA_ERR_INVALID_ARG = 1
+PLORA_ERR_UNSUPPORTED = 2
+PLORA_ERR_OOM = 3
+PLORA_ERR_CUDA = 4
+PLORA_ERR_TIMEOUT = 5
+PLORA_BF16 = 0
+PLORA_FP32 = 1
+PLORA_FLAG_SIMT = 1
+PLORA_MAX_RANK = 256
+PLORA_MAX_ADAPTERS = 4096
+
+EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
+            "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
+            "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read")
+
+
+class plora_config(ctypes.Structure):
+    _fields_ = [("d_in", ctypes.c_int64), ("d_out", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("max_adapters", ctypes.c_int32), ("max_rank", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("max_tokens", ctypes.c_int64)]
+
+
+class plora_adapter(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32), ("scale", ctypes.c_float), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p)]
+
+
+class PloraError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{status_string(status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libplora.so (raises ImportError if it is absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libplora.so not built at {path}; run packed_lora_fine_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    H = ctypes.c_void_p
+    lib.plora_create.argtypes = [ctypes.POINTER(H), ctypes.POINTER(plora_config)]
+    lib.plora_destroy.argtypes = [H]
+    lib.plora_saved_bytes.argtypes = [H, I32, P, P, ctypes.POINTER(ctypes.c_size_t)]
+    lib.plora_forward.argtypes = [H, P, P, P, I32, P, P, P, P]
+    lib.plora_backward.argtypes = [H, P, P, P, P, I32, P, P, P, P]
+    lib.plora_check.argtypes = [H, P]
+    lib.plora_status_string.argtypes = [ctypes.c_int]
+    lib.plora_status_string.restype = ctypes.c_char_p
+    lib.plora_last_error.argtypes = [H]
+    lib.plora_last_error.restype = ctypes.c_char_p
+    lib.plora_debug_unpack_saved.argtypes = [H, I32, P, P, P, I32, P, P]
+    lib.plora_debug_schedule.argtypes = [ctypes.POINTER(plora_config), I32, P, P, I32, I32, P, I64,
+                                         ctypes.POINTER(ctypes.c_int64)]
+    lib.plora_debug_schedule.restype = ctypes.c_int
+    lib.plora_profile_enable.argtypes = [H, I32]
+    lib.plora_profile_enable.restype = ctypes.c_int
+    lib.plora_profile_read.argtypes = [H, I32, ctypes.POINTER(I32), P, P, P]
+    lib.plora_profile_read.restype = ctypes.c_int
+    lib.plora_version.argtypes = []
+    lib.plora_version.restype = ctypes.c_int32
+    for fn in ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
+               "plora_check", "plora_debug_unpack_saved"):
+        getattr(lib, fn).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load().plora_status_string(int(s)).decode()
+
+
+def _raise(h, s: int):
+    if s != PLORA_OK:
+        msg = load().plora_last_error(h).decode() if h else ""
+        raise PloraError(s, msg)
+
+
+def _offsets(off) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(off, dtype=np.int64))
+
+
+def make_table(ranks: Sequence[int], scales: Sequence[float], A: Sequence[int], B: Sequence[int],
+               dA: Optional[Sequence[int]] = None, dB: Optional[Sequence[int]] = None):
+    """Build a host plora_adapter[] from ranks, scales and device pointers (ints)."""
+    n = len(ranks)
+    tab = (plora_adapter * max(1, n))()
+    for i in range(n):
+        tab[i].rank = int(ranks[i])
+        tab[i].scale = float(scales[i])
+        tab[i].A = int(A[i])
+        tab[i].B = int(B[i])
+        tab[i].dA = int(dA[i]) if dA is not None else None
+        tab[i].dB = int(dB[i]) if dB is not None else None
+    return tab
+
+
+# ---------------------------------------------------------------- C names
+def plora_create(d_in: int, d_out: int, dtype: int, max_adapters: int, max_rank: int, max_tokens: int,
+                 flags: int = 0) -> int:
+    lib = load()
+    cfg = plora_config(d_in, d_out, dtype, max_adapters, max_rank, flags, max_tokens)
+    h = ctypes.c_void_p()
+    s = lib.plora_create(ctypes.byref(h), ctypes.byref(cfg))
+    if s != PLORA_OK:
+        raise PloraError(s, "plora_create")
+    return h.value
+
+
+def plora_create_status(cfg: plora_config):
+    """Raw form: returns (status, handle-or-None)."""
+    h = ctypes.c_void_p()
+    s = load().plora_create(ctypes.byref(h), ctypes.byref(cfg))
+    return s, h.value
+
+
+def plora_destroy(h: int) -> None:
+    _raise(None, load().plora_destroy(h))
+
+
+def plora_saved_bytes(h: int, n: int, off, tab) -> int:
+    off = _offsets(off)
+    out = ctypes.c_size_t(0)
+    _raise(h, load().plora_saved_bytes(h, n, off.ctypes.data, ctypes.addressof(tab), ctypes.byref(out)))
+    return int(out.value)
+
+
+def plora_forward(h: int, X: int, W: int, Y: int, n: int, off, tab, saved: int, stream: int = 0,
+                  check: bool = True) -> int:
+    off = _offsets(off)
+    s = load().plora_forward(h, X, W, Y, n, off.ctypes.data, ctypes.addressof(tab), saved, stream)
+    if check:
+        _raise(h, s)
+    return s
+
+
+def plora_backward(h: int, X: int, W: int, dY: int, dX: Optional[int], n: int, off, tab, saved: int,
+                   stream: int = 0, check: bool = True) -> int:
+    off = _offsets(off)
+    s = load().plora_backward(h, X, W, dY, dX or None, n, off.ctypes.data, ctypes.addressof(tab), saved, stream)
+    if check:
+        _raise(h, s)
+    return s
+
+
+def plora_check(h: int, stream: int = 0) -> int:
+    return load().plora_check(h, stream)
+
+
+def plora_last_error(h: int) -> str:
+    return load().plora_last_error(h).decode()
+
+
+def plora_debug_unpack_saved(h: int, n: int, off, tab, saved: int, i: int, H_out: int, stream: int = 0) -> None:
+    off = _offsets(off)
+    _raise(h, load().plora_debug_unpack_saved(h, n, off.ctypes.data, ctypes.addressof(tab), saved, i, H_out,
+                                              stream))
+
+
+def plora_debug_schedule(cfg: plora_config, n: int, off, tab, grads: bool, which: int):
+    """Returns (status, int32 numpy array) of the host schedule; see include/plora.h."""
+    lib = load()
+    off = _offsets(off)
+    cnt = ctypes.c_int64(0)
+    tptr = ctypes.addressof(tab) if tab is not None else None
+    s = lib.plora_debug_schedule(ctypes.byref(cfg), n, off.ctypes.data, tptr, int(grads), which, None, 0,
+                                 ctypes.byref(cnt))
+    if s != PLORA_OK:
+        return s, None
+    buf = np.zeros(max(1, cnt.value), dtype=np.int32)
+    s = lib.plora_debug_schedule(ctypes.byref(cfg), n, off.ctypes.data, tptr, int(grads), which,
+                                 buf.ctypes.data, cnt.value, ctypes.byref(cnt))
+    return s, buf[:cnt.value]
+
+
+def plora_profile_enable(h: int, enable: bool) -> None:
+    _raise(h, load().plora_profile_enable(h, int(bool(enable))))
+
+
+def plora_profile_read(h: int) -> dict:
+    """{kernel kind: (launches, total device ms)} since the last read."""
+    lib = load()
+    cap = 32
+    n = ctypes.c_int32(0)
+    names = (ctypes.c_char_p * cap)()
+    launches = (ctypes.c_int64 * cap)()
+    ms = (ctypes.c_double * cap)()
+    _raise(h, lib.plora_profile_read(h, cap, ctypes.byref(n), names, launches, ms))
+    return {names[k].decode(): (int(launches[k]), float(ms[k])) for k in range(min(n.value, cap))}
+
+
+def plora_version() -> int:
+    return int(load().plora_version())
+
+
+# ---------------------------------------------------------------- torch convenience
+class PackedLoRA:
+    """Owns a handle; runs the packed forward/backward on torch CUDA tensors.
+
+    ``A[i]`` is ``[r_i][d_in]`` (lora_A.weight), ``B[i]`` is ``[d_out][r_i]``
+    (lora_B.weight), ``W`` is ``[d_out][d_in]`` (nn.Linear.weight), ``X`` is
+    the packed ``[T][d_in]`` token buffer, ``off`` the host segment offsets.
+    """
+
+    def __init__(self, d_in, d_out, dtype="bf16", max_adapters=64, max_rank=PLORA_MAX_RANK,
+                 max_tokens=1 << 16, simt=False):
+        self.d_in, self.d_out = int(d_in), int(d_out)
+        self.dtype = dtype
+        self.h = plora_create(self.d_in, self.d_out, PLORA_BF16 if dtype == "bf16" else PLORA_FP32,
+                              max_adapters, max_rank, max_tokens, PLORA_FLAG_SIMT if simt else 0)
+
+    def close(self):
+        if self.h:
+            plora_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def table(self, scales, A, B, dA=None, dB=None):
+        ranks = [a.shape[0] for a in A]
+        return make_table(ranks, scales, [a.data_ptr() for a in A], [b.data_ptr() for b in B],
+                          None if dA is None else [x.data_ptr() for x in dA],
+                          None if dB is None else [x.data_ptr() for x in dB])
+
+    def saved_bytes(self, off, tab) -> int:
+        return plora_saved_bytes(self.h, len(off) - 1, off, tab)
+
+    def forward(self, X, W, off, scales, A, B, Y=None, saved=None, stream=None):
+        import torch
+        n = len(off) - 1
+        tab = self.table(scales, A, B)
+        if Y is None:
+            Y = torch.empty((X.shape[0], self.d_out), dtype=X.dtype, device=X.device)
+        nbytes = self.saved_bytes(off, tab)
+        if saved is None:
+            saved = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=X.device)
+        st = (stream or torch.cuda.current_stream()).cuda_stream
+        plora_forward(self.h, X.data_ptr(), W.data_ptr(), Y.data_ptr(), n, off, tab, saved.data_ptr(), st)
+        return Y, saved
+
+    def backward(self, X, W, dY, off, scales, A, B, saved, dX=None, dA=None, dB=None, want_dX=True, stream=None):
+        import torch
+        n = len(off) - 1
+        if dA is None:
+            dA = [torch.empty(a.shape, dtype=torch.float32, device=X.device) for a in A]
+        if dB is None:
+            dB = [torch.empty(b.shape, dtype=torch.float32, device=X.device) for b in B]
+        if want_dX and dX is None:
+            dX = torch.empty_like(X)
+        tab = self.table(scales, A, B, dA, dB)
+        st = (stream or torch.cuda.current_stream()).cuda_stream
+        plora_backward(self.h, X.data_ptr(), W.data_ptr(), dY.data_ptr(), dX.data_ptr() if want_dX else None,
+                       n, off, tab, saved.data_ptr(), st)
+        return dX, dA, dB

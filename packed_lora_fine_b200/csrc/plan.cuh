@@ -1,0 +1,72 @@
+// plan.cuh -- per-call schedule structures shared by the host code and the kernels.
+//
+// A call's schedule is built on the host from the segment offsets and the
+// adapter table, copied once to the device (one cudaMemcpyAsync from pinned
+// staging), and read by every kernel of the call.
+#pragma once
+#include <cstdint>
+
+namespace plora {
+
+constexpr int kTileM = 128;     // token rows (or hidden rows) per tensor-core tile
+constexpr int kBlockK = 64;     // K elements per pipeline stage (128 bytes of bf16)
+constexpr int kRankAlign = 64;  // the padded rank width RP of the saved/G buffers is a multiple of this
+constexpr int kSplitTokens = 4096;  // weight-gradient split size along the tokens (fixed: deterministic)
+
+// One adapter, as the kernels see it.
+struct AdapterDev {
+    const void* A;     // A_store [rank][d_in]
+    const void* B;     // B_store [d_out][rank]
+    float* dA;         // [rank][d_in]
+    float* dB;         // [d_out][rank]
+    int32_t x_row;     // first token row in X / Y / dY / dX (= off[i])
+    int32_t n;         // tokens of this adapter
+    int32_t h_row;     // first row of this adapter's block in the saved H / workspace G buffers
+    int32_t rank;
+    float scale;
+    int32_t rp16;      // rank rounded up to 16 (the MMA N or K extent)
+    int32_t rp64;      // rank rounded up to 64 (the MN-major tile width)
+    int32_t pad_;
+};
+static_assert(sizeof(AdapterDev) == 64, "AdapterDev layout");
+
+// A 128-row tile of one adapter's tokens (shrink / expand kernels).
+struct TokTile {
+    int32_t adapter;
+    int32_t rows;      // valid rows in this tile, 1..128
+    int32_t x_row;     // first token row
+    int32_t h_row;     // first row in H / G
+};
+static_assert(sizeof(TokTile) == 16, "TokTile layout");
+
+// One split of one adapter's tokens for the weight gradients (dB, dA).
+struct RedEntry {
+    int32_t adapter;
+    int32_t x_row;     // first token row of the split
+    int32_t h_row;     // first H / G row of the split
+    int32_t kblocks;   // 64-token blocks in the split
+    int32_t split;     // index of the split within the adapter
+    int32_t nsplit;    // number of splits of the adapter
+    int32_t slot;      // first partial slot of the adapter (nsplit > 1), else -1
+    int32_t counter;   // first arrival counter of the adapter (nsplit > 1), else -1
+};
+static_assert(sizeof(RedEntry) == 32, "RedEntry layout");
+
+// A generic strided product for the SIMT path:
+//   C(m, n) = alpha * sum_k A(m, k) B(k, n)  (+ C(m, n) if accumulate)
+// with A(m,k) = A[m*a_sm + k*a_sk], B(k,n) = B[k*b_sk + n*b_sn], C(m,n) = C[m*c_sm + n*c_sn].
+struct SimtOp {
+    const void* A;
+    const void* B;
+    void* C;
+    int64_t a_sm, a_sk, b_sk, b_sn, c_sm, c_sn;
+    int32_t M, N, K;
+    float alpha;
+    int32_t accumulate;
+    int32_t c_fp32;      // 1: C is fp32; 0: C has the input element type
+    int32_t tile_begin;  // first block index of this op in the launch
+    int32_t tiles_n;     // 64-wide tiles along N
+};
+static_assert(sizeof(SimtOp) == 104, "SimtOp layout");
+
+}  // namespace plora

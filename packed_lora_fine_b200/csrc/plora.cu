@@ -1,0 +1,816 @@
+// plora.cu -- host side of the packed LoRA library: argument checking, the
+// per-call schedule (segment tiles, weight-gradient splits, LPT order), the
+// tensor maps, the workspace, and the launches of the sm_100a kernels.
+//
+// The C ABI is declared and documented in include/plora.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/plora.h"
+#include "plan.cuh"
+#include "simt.cuh"
+#include "tc.cuh"
+
+using namespace plora;
+
+namespace {
+
+constexpr int kSlots = 4;                   // host staging / device schedule ring depth
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+struct Region {
+    size_t off = 0, bytes = 0;
+};
+
+}  // namespace
+
+struct plora_ctx {
+    plora_config cfg{};
+    int device = 0;
+    int num_sms = 0;
+    size_t esize = 2;
+    int RPmax = 64;
+    int64_t max_h_rows = 0;
+    int64_t max_slots = 0, max_counters = 0;
+    size_t blob_bytes = 0;
+    bool tc = false;           // tensor-core path (bf16 without PLORA_FLAG_SIMT)
+
+    uint8_t* ws = nullptr;     // one device allocation, carved into regions
+    size_t ws_bytes = 0;
+    Region r_G, r_packA, r_packBT, r_part, r_cnt, r_err, r_blob[kSlots];
+
+    uint8_t* h_blob[kSlots] = {};
+    cudaEvent_t ev[kSlots] = {};
+    int next_slot = 0;
+
+    std::string last_error;
+
+    // Launch accounting and optional per-kernel timing (CUDA events on the launching stream).
+    bool profiling = false;
+    int64_t launches[16] = {};
+    double total_ms[16] = {};
+    struct Rec { int kind; cudaEvent_t a, b; };
+    std::vector<Rec> pending;
+    std::vector<cudaEvent_t> pool;
+
+    template <typename T> T* at(const Region& r) const { return reinterpret_cast<T*>(ws + r.off); }
+};
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+plora_status fail(plora_ctx* h, plora_status s, const char* fmt, ...) {
+    if (h) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        h->last_error = buf;
+    }
+    return s;
+}
+
+plora_status cuda_fail(plora_ctx* h, cudaError_t e, const char* what) {
+    return fail(h, PLORA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool get_encode() {
+    if (g_encode) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return false;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return true;
+}
+
+// Kernel kinds for launch accounting / profiling.
+enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
+            kSimt, kKinds };
+const char* const kKindNames[kKinds] = {"pack_a", "pack_bt", "base_fwd", "shrink_x", "expand_y", "base_dx",
+                                        "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm"};
+
+cudaEvent_t take_event(plora_ctx* h) {
+    if (!h->pool.empty()) {
+        cudaEvent_t e = h->pool.back();
+        h->pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Bracket one launch: record a start event (when profiling), run `launch`, record the end event.
+template <typename F>
+void tracked(plora_ctx* h, int kind, cudaStream_t st, F&& launch) {
+    h->launches[kind] += 1;
+    if (!h->profiling) {
+        launch();
+        return;
+    }
+    plora_ctx::Rec r{kind, take_event(h), take_event(h)};
+    cudaEventRecord(r.a, st);
+    launch();
+    cudaEventRecord(r.b, st);
+    h->pending.push_back(r);
+}
+
+// 2-D bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_elems,
+              uint32_t box_inner, uint32_t box_outer) {
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_elems * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Per-call schedule
+// ---------------------------------------------------------------------------
+struct HostPlan {
+    int32_t n = 0, RP = kRankAlign;
+    int64_t T = 0, h_rows = 0;
+    std::vector<AdapterDev> ad;
+    std::vector<TokTile> tok;
+    std::vector<RedEntry> red;
+    std::vector<int32_t> empty;    // adapters with no tokens
+    int32_t slots = 0, counters = 0;
+};
+
+plora_status check_table(plora_ctx* h, int32_t n, const int64_t* off, const plora_adapter* tab, bool grads) {
+    if (n < 0 || n > h->cfg.max_adapters)
+        return fail(h, PLORA_ERR_INVALID_ARG, "n_adapters=%d outside [0, max_adapters=%d]", n, h->cfg.max_adapters);
+    if (!off) return fail(h, PLORA_ERR_INVALID_ARG, "off is NULL");
+    if (n > 0 && !tab) return fail(h, PLORA_ERR_INVALID_ARG, "adapter table is NULL");
+    if (off[0] != 0) return fail(h, PLORA_ERR_INVALID_ARG, "off[0]=%lld, must be 0", (long long)off[0]);
+    for (int32_t i = 0; i < n; ++i) {
+        if (off[i + 1] < off[i])
+            return fail(h, PLORA_ERR_INVALID_ARG, "offsets decrease at adapter %d (%lld > %lld)", i,
+                        (long long)off[i], (long long)off[i + 1]);
+    }
+    if (off[n] > h->cfg.max_tokens)
+        return fail(h, PLORA_ERR_INVALID_ARG, "off[n]=%lld exceeds max_tokens=%lld", (long long)off[n],
+                    (long long)h->cfg.max_tokens);
+    for (int32_t i = 0; i < n; ++i) {
+        const plora_adapter& a = tab[i];
+        if (a.rank < 1 || a.rank > h->cfg.max_rank)
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: rank %d outside [1, max_rank=%d]", i, a.rank,
+                        h->cfg.max_rank);
+        if (!std::isfinite(a.scale)) return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: scale is not finite", i);
+        if (!a.A || !a.B) return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: A or B is NULL", i);
+        if (!aligned16(a.A) || !aligned16(a.B))
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: A or B not 16-byte aligned", i);
+        if (grads) {
+            if (!a.dA || !a.dB) return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: dA or dB is NULL", i);
+            if (!aligned16(a.dA) || !aligned16(a.dB))
+                return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: dA or dB not 16-byte aligned", i);
+        }
+    }
+    return PLORA_OK;
+}
+
+void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_adapter* tab, HostPlan& P) {
+    P.n = n;
+    P.T = off[n];
+    int maxr = 1;
+    for (int32_t i = 0; i < n; ++i) maxr = std::max(maxr, tab[i].rank);
+    P.RP = (int32_t)round_up(maxr, kRankAlign);
+    P.ad.resize(n);
+    int64_t hrow = 0;
+    const int64_t dtiles = std::max(ceil_div(h->cfg.d_in, kTileM), ceil_div(h->cfg.d_out, kTileM));
+    for (int32_t i = 0; i < n; ++i) {
+        AdapterDev& a = P.ad[i];
+        a.A = tab[i].A;
+        a.B = tab[i].B;
+        a.dA = tab[i].dA;
+        a.dB = tab[i].dB;
+        a.x_row = (int32_t)off[i];
+        a.n = (int32_t)(off[i + 1] - off[i]);
+        a.h_row = (int32_t)hrow;
+        a.rank = tab[i].rank;
+        a.scale = tab[i].scale;
+        a.rp16 = (int32_t)round_up(a.rank, 16);
+        a.rp64 = (int32_t)round_up(a.rank, 64);
+        a.pad_ = 0;
+        hrow += round_up(a.n, kTileM);
+        if (a.n == 0) {
+            P.empty.push_back(i);
+            continue;
+        }
+        for (int32_t t = 0; t < a.n; t += kTileM)
+            P.tok.push_back(TokTile{i, std::min(kTileM, a.n - t), a.x_row + t, a.h_row + t});
+        // Weight-gradient splits: a function of this adapter's token count alone, so an
+        // adapter's dA/dB do not depend on what else is packed with it.
+        const int32_t nsplit = (int32_t)ceil_div(a.n, kSplitTokens);
+        const int32_t slot = nsplit > 1 ? P.slots : -1;
+        const int32_t cnt = nsplit > 1 ? P.counters : -1;
+        if (nsplit > 1) {
+            P.slots += nsplit;
+            P.counters += (int32_t)dtiles;
+        }
+        for (int32_t s = 0; s < nsplit; ++s) {
+            const int32_t t0 = s * kSplitTokens;
+            const int32_t len = std::min(kSplitTokens, a.n - t0);
+            P.red.push_back(RedEntry{i, a.x_row + t0, a.h_row + t0, (int32_t)ceil_div(len, kBlockK), s, nsplit,
+                                     slot, cnt});
+        }
+    }
+    P.h_rows = hrow;
+    // Longest-first order of the weight-gradient work (the static persistent schedule
+    // then deals items round-robin over the SMs).
+    std::stable_sort(P.red.begin(), P.red.end(),
+                     [](const RedEntry& a, const RedEntry& b) { return a.kblocks > b.kblocks; });
+}
+
+size_t saved_bytes_of(const plora_ctx* h, const HostPlan& P) {
+    return (size_t)P.h_rows * (size_t)P.RP * h->esize;
+}
+
+// Copy the plan blob to the device through the staging ring. Returns device pointers.
+struct DevPlan {
+    AdapterDev* ad = nullptr;
+    TokTile* tok = nullptr;
+    RedEntry* red = nullptr;
+    SimtOp* ops = nullptr;
+    int slot = 0;
+};
+
+plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& ops, cudaStream_t st,
+                    DevPlan& D) {
+    const int slot = h->next_slot;
+    h->next_slot = (h->next_slot + 1) % kSlots;
+    cudaError_t e = cudaEventSynchronize(h->ev[slot]);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize(staging slot)");
+    size_t o = 0;
+    auto put = [&](const void* src, size_t bytes) {
+        const size_t at = o;
+        if (bytes) memcpy(h->h_blob[slot] + at, src, bytes);
+        o = round_up((int64_t)(o + bytes), 256);
+        return at;
+    };
+    const size_t o_ad = put(P.ad.data(), P.ad.size() * sizeof(AdapterDev));
+    const size_t o_tok = put(P.tok.data(), P.tok.size() * sizeof(TokTile));
+    const size_t o_red = put(P.red.data(), P.red.size() * sizeof(RedEntry));
+    const size_t o_ops = put(ops.data(), ops.size() * sizeof(SimtOp));
+    if (o > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "schedule exceeds the handle's staging size");
+    uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
+    e = cudaMemcpyAsync(d, h->h_blob[slot], o, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync(schedule)");
+    D.ad = reinterpret_cast<AdapterDev*>(d + o_ad);
+    D.tok = reinterpret_cast<TokTile*>(d + o_tok);
+    D.red = reinterpret_cast<RedEntry*>(d + o_red);
+    D.ops = reinterpret_cast<SimtOp*>(d + o_ops);
+    D.slot = slot;
+    return PLORA_OK;
+}
+
+plora_status finish(plora_ctx* h, const DevPlan& D, cudaStream_t st) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
+    e = cudaEventRecord(h->ev[D.slot], st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    return PLORA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// SIMT ops
+// ---------------------------------------------------------------------------
+void add_op(std::vector<SimtOp>& ops, int32_t& tiles, const void* A, int64_t a_sm, int64_t a_sk, const void* B,
+            int64_t b_sk, int64_t b_sn, void* C, int64_t c_sm, int64_t c_sn, int64_t M, int64_t N, int64_t K,
+            float alpha, bool acc, bool c_fp32) {
+    if (M <= 0 || N <= 0) return;
+    SimtOp o{};
+    o.A = A; o.B = B; o.C = C;
+    o.a_sm = a_sm; o.a_sk = a_sk; o.b_sk = b_sk; o.b_sn = b_sn; o.c_sm = c_sm; o.c_sn = c_sn;
+    o.M = (int32_t)M; o.N = (int32_t)N; o.K = (int32_t)K;
+    o.alpha = alpha;
+    o.accumulate = acc ? 1 : 0;
+    o.c_fp32 = c_fp32 ? 1 : 0;
+    o.tile_begin = tiles;
+    o.tiles_n = (int32_t)ceil_div(N, 64);
+    tiles += (int32_t)(ceil_div(M, 64) * o.tiles_n);
+    ops.push_back(o);
+}
+
+template <typename T>
+void launch_simt(plora_ctx* h, const SimtOp* d_ops, int n_ops, int tiles, cudaStream_t st) {
+    if (tiles > 0)
+        tracked(h, kSimt, st, [&] { simt_gemm_kernel<T><<<tiles, 256, 0, st>>>(d_ops, n_ops); });
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core launches
+// ---------------------------------------------------------------------------
+template <Op OP>
+void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, cudaStream_t st) {
+    if (p.num_tiles <= 0) return;
+    const int grid = std::min(p.num_tiles, h->num_sms);
+    constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : OP == Op::BaseDx ? kBaseDx : OP == Op::ShrinkX ? kShrinkX
+                       : OP == Op::ShrinkDy ? kShrinkDy : OP == Op::ExpandY ? kExpandY : OP == Op::ExpandDx ? kExpandDx
+                       : OP == Op::WgradB ? kWgradB : kWgradA;
+    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, p); });
+}
+
+template <Op OP>
+cudaError_t set_tc_attr() {
+    return cudaFuncSetAttribute(tc_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+}
+
+TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
+    TcParams p{};
+    p.RP = P.RP;
+    p.adapters = D.ad;
+    p.tok = D.tok;
+    p.red = D.red;
+    p.err_flag = h->at<int>(h->r_err);
+    p.timeout_ns = kTimeoutNs;
+    p.partials = h->at<float>(h->r_part);
+    p.counters = h->at<int32_t>(h->r_cnt);
+    p.group_m = 16;
+    return p;
+}
+
+plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, cudaStream_t st) {
+    if (P.n == 0) return PLORA_OK;
+    __nv_bfloat16* pa = h->at<__nv_bfloat16>(h->r_packA);
+    __nv_bfloat16* pb = h->at<__nv_bfloat16>(h->r_packBT);
+    const int64_t vecs = (int64_t)P.n * P.RP * (h->cfg.d_in / 8);
+    const int grid_a = (int)std::min<int64_t>(ceil_div(vecs, 256), (int64_t)h->num_sms * 8);
+    tracked(h, kPackA, st, [&] { pack_a_kernel<<<grid_a, 256, 0, st>>>(D.ad, P.n, P.RP, h->cfg.d_in, pa); });
+    dim3 gb((unsigned)ceil_div(h->cfg.d_out, 64), (unsigned)P.n);
+    tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, 0, st>>>(D.ad, P.RP, h->cfg.d_out, pb); });
+    return PLORA_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* plora_status_string(plora_status s) {
+    switch (s) {
+        case PLORA_OK: return "PLORA_OK";
+        case PLORA_ERR_INVALID_ARG: return "PLORA_ERR_INVALID_ARG";
+        case PLORA_ERR_UNSUPPORTED: return "PLORA_ERR_UNSUPPORTED";
+        case PLORA_ERR_OOM: return "PLORA_ERR_OOM";
+        case PLORA_ERR_CUDA: return "PLORA_ERR_CUDA";
+        case PLORA_ERR_TIMEOUT: return "PLORA_ERR_TIMEOUT";
+    }
+    return "PLORA_ERR_UNKNOWN";
+}
+
+const char* plora_last_error(plora_handle h) { return h ? h->last_error.c_str() : ""; }
+
+int32_t plora_version(void) { return 100; }
+
+plora_status plora_create(plora_handle* out, const plora_config* cfg) {
+    if (!out) return PLORA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!cfg) return PLORA_ERR_INVALID_ARG;
+    if (cfg->dtype != PLORA_BF16 && cfg->dtype != PLORA_FP32) return PLORA_ERR_UNSUPPORTED;
+    if (cfg->d_in < 8 || cfg->d_out < 8 || cfg->d_in > 65536 || cfg->d_out > 65536) return PLORA_ERR_UNSUPPORTED;
+    if (cfg->d_in % 8 || cfg->d_out % 8) return PLORA_ERR_UNSUPPORTED;
+    if (cfg->max_adapters < 1 || cfg->max_adapters > PLORA_MAX_ADAPTERS) return PLORA_ERR_INVALID_ARG;
+    if (cfg->max_rank < 1 || cfg->max_rank > PLORA_MAX_RANK) return PLORA_ERR_INVALID_ARG;
+    if (cfg->max_tokens < 1 || cfg->max_tokens > ((int64_t)1 << 30)) return PLORA_ERR_INVALID_ARG;
+    if (cfg->flags & ~(uint32_t)PLORA_FLAG_SIMT) return PLORA_ERR_INVALID_ARG;
+
+    plora_ctx* h = new (std::nothrow) plora_ctx();
+    if (!h) return PLORA_ERR_OOM;
+    h->cfg = *cfg;
+    h->esize = cfg->dtype == PLORA_BF16 ? 2 : 4;
+    h->tc = cfg->dtype == PLORA_BF16 && !(cfg->flags & PLORA_FLAG_SIMT);
+
+    cudaError_t e = cudaGetDevice(&h->device);
+    cudaDeviceProp prop{};
+    if (e == cudaSuccess) e = cudaGetDeviceProperties(&prop, h->device);
+    if (e != cudaSuccess) { delete h; return PLORA_ERR_CUDA; }
+    if (prop.major != 10) { delete h; return PLORA_ERR_UNSUPPORTED; }
+    h->num_sms = prop.multiProcessorCount;
+    if (h->tc && !get_encode()) { delete h; return PLORA_ERR_CUDA; }
+
+    // Workspace sizing (all bounds follow from the config).
+    const int64_t na = cfg->max_adapters;
+    h->RPmax = (int)round_up(cfg->max_rank, kRankAlign);
+    h->max_h_rows = cfg->max_tokens + (int64_t)(kTileM - 1) * na;
+    const int64_t dtiles = std::max(ceil_div(cfg->d_in, kTileM), ceil_div(cfg->d_out, kTileM));
+    h->max_slots = 2 * (cfg->max_tokens / kSplitTokens) + 1;
+    h->max_counters = (cfg->max_tokens / (kSplitTokens + 1) + 1) * dtiles;
+    const int64_t tok_max = cfg->max_tokens / kTileM + na + 1;
+    const int64_t red_max = h->max_slots + na + 1;
+    const int64_t ops_max = 4 * na + 4;
+    h->blob_bytes = (size_t)round_up(na * (int64_t)sizeof(AdapterDev), 256) +
+                    (size_t)round_up(tok_max * (int64_t)sizeof(TokTile), 256) +
+                    (size_t)round_up(red_max * (int64_t)sizeof(RedEntry), 256) +
+                    (size_t)round_up(ops_max * (int64_t)sizeof(SimtOp), 256) + 1024;
+
+    size_t o = 0;
+    auto carve = [&](Region& r, size_t bytes) {
+        r.off = o;
+        r.bytes = bytes;
+        o = (size_t)round_up((int64_t)(o + bytes), 1024);
+    };
+    carve(h->r_err, 256);
+    carve(h->r_G, (size_t)h->max_h_rows * h->RPmax * h->esize);
+    if (h->tc) {
+        carve(h->r_packA, (size_t)na * h->RPmax * cfg->d_in * 2);
+        carve(h->r_packBT, (size_t)na * h->RPmax * cfg->d_out * 2);
+        carve(h->r_part, (size_t)h->max_slots * dtiles * kTileM * h->RPmax * sizeof(float));
+        carve(h->r_cnt, (size_t)h->max_counters * sizeof(int32_t));
+    }
+    for (int s = 0; s < kSlots; ++s) carve(h->r_blob[s], h->blob_bytes);
+    h->ws_bytes = o;
+    e = cudaMalloc(&h->ws, h->ws_bytes);
+    if (e != cudaSuccess) { cudaGetLastError(); delete h; return PLORA_ERR_OOM; }
+    e = cudaMemset(h->ws, 0, h->ws_bytes);
+    for (int s = 0; s < kSlots && e == cudaSuccess; ++s) {
+        e = cudaMallocHost(&h->h_blob[s], h->blob_bytes);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev[s], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess && h->tc) {
+        e = set_tc_attr<Op::BaseFwd>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::BaseDx>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::ShrinkX>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::ShrinkDy>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::ExpandY>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::ExpandDx>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::WgradB>();
+        if (e == cudaSuccess) e = set_tc_attr<Op::WgradA>();
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        plora_destroy(h);
+        return e == cudaErrorMemoryAllocation ? PLORA_ERR_OOM : PLORA_ERR_CUDA;
+    }
+    *out = h;
+    return PLORA_OK;
+}
+
+plora_status plora_destroy(plora_handle h) {
+    if (!h) return PLORA_OK;
+    cudaDeviceSynchronize();
+    for (int s = 0; s < kSlots; ++s) {
+        if (h->ev[s]) cudaEventDestroy(h->ev[s]);
+        if (h->h_blob[s]) cudaFreeHost(h->h_blob[s]);
+    }
+    for (const plora_ctx::Rec& r : h->pending) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (cudaEvent_t e : h->pool) cudaEventDestroy(e);
+    if (h->ws) cudaFree(h->ws);
+    delete h;
+    return PLORA_OK;
+}
+
+plora_status plora_saved_bytes(plora_handle h, int32_t n, const int64_t* off, const plora_adapter* tab,
+                               size_t* bytes) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    if (!bytes) return fail(h, PLORA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = 0;
+    plora_status s = check_table(h, n, off, tab, false);
+    if (s != PLORA_OK) return s;
+    HostPlan P;
+    build_plan(h, n, off, tab, P);
+    *bytes = saved_bytes_of(h, P);
+    return PLORA_OK;
+}
+
+plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y, int32_t n, const int64_t* off,
+                           const plora_adapter* tab, void* saved, void* stream) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    plora_status s = check_table(h, n, off, tab, false);
+    if (s != PLORA_OK) return s;
+    const bool any_tokens = off[n] > 0;   // with no tokens, X, Y and saved are never touched
+    if (!W || (any_tokens && (!X || !Y || !saved)))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, Y or saved is NULL");
+    if (!aligned16(X) || !aligned16(W) || !aligned16(Y))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W or Y not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0)
+        return fail(h, PLORA_ERR_INVALID_ARG, "saved not 256-byte aligned");
+    cudaError_t ce = cudaSetDevice(h->device);
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    HostPlan P;
+    build_plan(h, n, off, tab, P);
+    if (P.T == 0) return PLORA_OK;
+    const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
+
+    if (!h->tc) {
+        std::vector<SimtOp> ops;
+        int32_t t1 = 0, t2 = 0;
+        const bool f32 = h->cfg.dtype == PLORA_FP32;
+        const size_t es = h->esize;
+        // K1: Y = X W.  K2: H_i = X_i A_i.
+        add_op(ops, t1, X, d_in, 1, W, 1, d_in, Y, d_out, 1, P.T, d_out, d_in, 1.f, false, f32);
+        for (const AdapterDev& a : P.ad) {
+            if (a.n == 0) continue;
+            add_op(ops, t1, (const uint8_t*)X + (size_t)a.x_row * d_in * es, d_in, 1, a.A, 1, d_in,
+                   (uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.n, a.rank, d_in, 1.f, false, f32);
+        }
+        const int n1 = (int)ops.size();
+        // K3: Y_i += s_i H_i B_i.
+        for (const AdapterDev& a : P.ad) {
+            if (a.n == 0) continue;
+            add_op(ops, t2, (const uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.B, 1, a.rank,
+                   (uint8_t*)Y + (size_t)a.x_row * d_out * es, d_out, 1, a.n, d_out, a.rank, a.scale, true, f32);
+        }
+        DevPlan D;
+        s = upload(h, P, ops, st, D);
+        if (s != PLORA_OK) return s;
+        if (f32) {
+            launch_simt<float>(h, D.ops, n1, t1, st);
+            launch_simt<float>(h, D.ops + n1, (int)ops.size() - n1, t2, st);
+        } else {
+            launch_simt<__nv_bfloat16>(h, D.ops, n1, t1, st);
+            launch_simt<__nv_bfloat16>(h, D.ops + n1, (int)ops.size() - n1, t2, st);
+        }
+        return finish(h, D, st);
+    }
+
+    // Tensor-core path.
+    DevPlan D;
+    s = upload(h, P, {}, st, D);
+    if (s != PLORA_OK) return s;
+    pack_factors(h, P, D, st);
+    CUtensorMap mX, mW, mPA, mH, mPB;
+    bool ok = make_map(&mX, X, d_in, P.T, d_in, 64, kTileM) &&
+              make_map(&mW, W, d_in, d_out, d_in, 64, kTileN) &&
+              make_map(&mPA, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, P.RP) &&
+              make_map(&mH, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_map(&mPB, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 64);
+    if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+    TcParams p = base_params(h, P, D);
+    // K1: Y = X W over all packed tokens.
+    p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_out; p.K_total = (int32_t)d_in;
+    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_out, kTileN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.b_box_rows = kTileN;
+    p.out = Y; p.out_ld = d_out;
+    launch_tc<Op::BaseFwd>(h, mX, mW, p, st);
+    // K2: H_i = X_i A_i per 128-token tile.
+    TcParams q = base_params(h, P, D);
+    q.K_total = (int32_t)d_in;
+    q.num_tiles = (int32_t)P.tok.size();
+    q.b_box_rows = P.RP;
+    q.out = saved; q.out_ld = P.RP;
+    launch_tc<Op::ShrinkX>(h, mX, mPA, q, st);
+    // K3: Y_i += s_i H_i B_i.
+    TcParams r = base_params(h, P, D);
+    r.N_total = (int32_t)d_out;
+    r.tiles_n = (int32_t)ceil_div(d_out, kTileN);
+    r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
+    r.out = Y; r.out_ld = d_out;
+    launch_tc<Op::ExpandY>(h, mH, mPB, r, st);
+    return finish(h, D, st);
+}
+
+plora_status plora_backward(plora_handle h, const void* X, const void* W, const void* dY, void* dX, int32_t n,
+                            const int64_t* off, const plora_adapter* tab, const void* saved, void* stream) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    plora_status s = check_table(h, n, off, tab, true);
+    if (s != PLORA_OK) return s;
+    const bool any_tokens = off[n] > 0;   // with no tokens, only dA and dB are written (zeros)
+    if (!W || (any_tokens && (!X || !dY || !saved)))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, dY or saved is NULL");
+    if (!aligned16(X) || !aligned16(W) || !aligned16(dY) || (dX && !aligned16(dX)))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, dY or dX not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0)
+        return fail(h, PLORA_ERR_INVALID_ARG, "saved not 256-byte aligned");
+    cudaError_t ce = cudaSetDevice(h->device);
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    HostPlan P;
+    build_plan(h, n, off, tab, P);
+    const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
+    // Adapters without tokens: their weight gradients are zero.
+    for (int32_t i : P.empty) {
+        ce = cudaMemsetAsync(tab[i].dA, 0, (size_t)tab[i].rank * d_in * sizeof(float), st);
+        if (ce == cudaSuccess) ce = cudaMemsetAsync(tab[i].dB, 0, (size_t)tab[i].rank * d_out * sizeof(float), st);
+        if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaMemsetAsync(dA/dB of an empty adapter)");
+    }
+    if (P.T == 0) return PLORA_OK;
+    void* G = h->at<void>(h->r_G);
+
+    if (!h->tc) {
+        std::vector<SimtOp> ops;
+        int32_t t1 = 0, t2 = 0;
+        const bool f32 = h->cfg.dtype == PLORA_FP32;
+        const size_t es = h->esize;
+        // Phase 1 -- K4: dX = dY W^T; K5: G_i = s_i dY_i B_i^T; K7: dB_i = s_i dY_i^T H_i.
+        if (dX) add_op(ops, t1, dY, d_out, 1, W, d_in, 1, dX, d_in, 1, P.T, d_in, d_out, 1.f, false, f32);
+        for (const AdapterDev& a : P.ad) {
+            if (a.n == 0) continue;
+            add_op(ops, t1, (const uint8_t*)dY + (size_t)a.x_row * d_out * es, d_out, 1, a.B, a.rank, 1,
+                   (uint8_t*)G + (size_t)a.h_row * P.RP * es, P.RP, 1, a.n, a.rank, d_out, a.scale, false, f32);
+            add_op(ops, t1, (const uint8_t*)dY + (size_t)a.x_row * d_out * es, 1, d_out,
+                   (const uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.dB, a.rank, 1, d_out, a.rank,
+                   a.n, a.scale, false, true);
+        }
+        const int n1 = (int)ops.size();
+        // Phase 2 -- K6: dX_i += G_i A_i^T; K8: dA_i = X_i^T G_i.
+        for (const AdapterDev& a : P.ad) {
+            if (a.n == 0) continue;
+            if (dX)
+                add_op(ops, t2, (const uint8_t*)G + (size_t)a.h_row * P.RP * es, P.RP, 1, a.A, d_in, 1,
+                       (uint8_t*)dX + (size_t)a.x_row * d_in * es, d_in, 1, a.n, d_in, a.rank, 1.f, true, f32);
+            add_op(ops, t2, (const uint8_t*)X + (size_t)a.x_row * d_in * es, 1, d_in,
+                   (const uint8_t*)G + (size_t)a.h_row * P.RP * es, P.RP, 1, a.dA, 1, d_in, d_in, a.rank, a.n,
+                   1.f, false, true);
+        }
+        DevPlan D;
+        s = upload(h, P, ops, st, D);
+        if (s != PLORA_OK) return s;
+        if (f32) {
+            launch_simt<float>(h, D.ops, n1, t1, st);
+            launch_simt<float>(h, D.ops + n1, (int)ops.size() - n1, t2, st);
+        } else {
+            launch_simt<__nv_bfloat16>(h, D.ops, n1, t1, st);
+            launch_simt<__nv_bfloat16>(h, D.ops + n1, (int)ops.size() - n1, t2, st);
+        }
+        return finish(h, D, st);
+    }
+
+    DevPlan D;
+    s = upload(h, P, {}, st, D);
+    if (s != PLORA_OK) return s;
+    pack_factors(h, P, D, st);
+    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_k, mG_k, mG_mn, mPA_mn, mH_mn, mX_mn;
+    bool ok = make_map(&mdY_k, dY, d_out, P.T, d_out, 64, kTileM) &&
+              make_map(&mdY_mn, dY, d_out, P.T, d_out, 64, 64) &&
+              make_map(&mW_mn, W, d_in, d_out, d_in, 64, 64) &&
+              make_map(&mPB_k, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, P.RP) &&
+              make_map(&mG_k, G, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_map(&mG_mn, G, P.RP, P.h_rows, P.RP, 64, 64) &&
+              make_map(&mPA_mn, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
+              make_map(&mH_mn, saved, P.RP, P.h_rows, P.RP, 64, 64) &&
+              make_map(&mX_mn, X, d_in, P.T, d_in, 64, 64);
+    if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+    if (dX) {
+        // K4: dX = dY W^T.
+        TcParams p = base_params(h, P, D);
+        p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
+        p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
+        p.num_tiles = p.tiles_m * p.tiles_n;
+        p.out = dX; p.out_ld = d_in;
+        launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, p, st);
+    }
+    // K5: G_i = s_i dY_i B_i^T.
+    TcParams q = base_params(h, P, D);
+    q.K_total = (int32_t)d_out;
+    q.num_tiles = (int32_t)P.tok.size();
+    q.b_box_rows = P.RP;
+    q.out = G; q.out_ld = P.RP;
+    launch_tc<Op::ShrinkDy>(h, mdY_k, mPB_k, q, st);
+    if (dX) {
+        // K6: dX_i += G_i A_i^T.
+        TcParams r = base_params(h, P, D);
+        r.N_total = (int32_t)d_in;
+        r.tiles_n = (int32_t)ceil_div(d_in, kTileN);
+        r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
+        r.out = dX; r.out_ld = d_in;
+        launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, r, st);
+    }
+    // K7: dB_i = s_i dY_i^T H_i; K8: dA_i = X_i^T G_i (sums over each adapter's tokens).
+    TcParams wb = base_params(h, P, D);
+    wb.M_total = (int32_t)d_out;
+    wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
+    wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
+    launch_tc<Op::WgradB>(h, mdY_mn, mH_mn, wb, st);
+    TcParams wa = base_params(h, P, D);
+    wa.M_total = (int32_t)d_in;
+    wa.red_dtiles = (int32_t)ceil_div(d_in, kTileM);
+    wa.num_tiles = (int32_t)P.red.size() * wa.red_dtiles;
+    launch_tc<Op::WgradA>(h, mX_mn, mG_mn, wa, st);
+    return finish(h, D, st);
+}
+
+plora_status plora_check(plora_handle h, void* stream) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamSynchronize");
+    int flag = 0;
+    e = cudaMemcpy(&flag, h->at<int>(h->r_err), sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(h, e, "reading the device error flag");
+    if (flag != 0) {
+        int zero = 0;
+        cudaMemcpy(h->at<int>(h->r_err), &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return fail(h, PLORA_ERR_TIMEOUT, "a device-side wait ran out of time (flag %d)", flag);
+    }
+    return PLORA_OK;
+}
+
+plora_status plora_debug_unpack_saved(plora_handle h, int32_t n, const int64_t* off, const plora_adapter* tab,
+                                      const void* saved, int32_t i, float* H_out, void* stream) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    plora_status s = check_table(h, n, off, tab, false);
+    if (s != PLORA_OK) return s;
+    if (i < 0 || i >= n) return fail(h, PLORA_ERR_INVALID_ARG, "adapter index %d outside [0, %d)", i, n);
+    if (!saved || !H_out || !aligned16(H_out)) return fail(h, PLORA_ERR_INVALID_ARG, "saved or H_out bad");
+    HostPlan P;
+    build_plan(h, n, off, tab, P);
+    const AdapterDev& a = P.ad[i];
+    if (a.n == 0) return PLORA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int grid = (int)std::min<int64_t>(ceil_div((int64_t)a.n * a.rank, 256), 1024);
+    if (h->cfg.dtype == PLORA_FP32)
+        unpack_saved_kernel<float><<<grid, 256, 0, st>>>((const float*)saved, a.h_row, P.RP, a.n, a.rank, H_out);
+    else
+        unpack_saved_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)saved, a.h_row, P.RP, a.n,
+                                                                 a.rank, H_out);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PLORA_OK : cuda_fail(h, e, "unpack launch");
+}
+
+plora_status plora_profile_enable(plora_handle h, int32_t enable) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->profiling = enable != 0;
+    return PLORA_OK;
+}
+
+plora_status plora_profile_read(plora_handle h, int32_t capacity, int32_t* n_kinds, const char** names,
+                                int64_t* launches, double* total_ms) {
+    if (!h || !n_kinds) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    for (const plora_ctx::Rec& r : h->pending) {
+        cudaError_t e = cudaEventSynchronize(r.b);
+        float ms = 0.f;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+        if (e != cudaSuccess) return cuda_fail(h, e, "reading profile events");
+        h->total_ms[r.kind] += ms;
+        h->pool.push_back(r.a);
+        h->pool.push_back(r.b);
+    }
+    h->pending.clear();
+    *n_kinds = kKinds;
+    for (int k = 0; k < kKinds && k < capacity; ++k) {
+        if (names) names[k] = kKindNames[k];
+        if (launches) launches[k] = h->launches[k];
+        if (total_ms) total_ms[k] = h->total_ms[k];
+        h->launches[k] = 0;
+        h->total_ms[k] = 0.0;
+    }
+    return PLORA_OK;
+}
+
+plora_status plora_debug_schedule(const plora_config* cfg, int32_t n, const int64_t* off, const plora_adapter* tab,
+                                  int32_t grads, int32_t which, int32_t* out, int64_t capacity, int64_t* count) {
+    if (!cfg || !count) return PLORA_ERR_INVALID_ARG;
+    *count = 0;
+    plora_ctx tmp;
+    tmp.cfg = *cfg;
+    tmp.esize = cfg->dtype == PLORA_FP32 ? 4 : 2;
+    plora_status s = check_table(&tmp, n, off, tab, grads != 0);
+    if (s != PLORA_OK) return s;
+    HostPlan P;
+    build_plan(&tmp, n, off, tab, P);
+    std::vector<int32_t> v;
+    if (which == 0) {
+        for (const TokTile& t : P.tok) v.insert(v.end(), {t.adapter, t.rows, t.x_row, t.h_row});
+    } else if (which == 1) {
+        for (const RedEntry& r : P.red)
+            v.insert(v.end(), {r.adapter, r.x_row, r.h_row, r.kblocks, r.split, r.nsplit, r.slot, r.counter});
+    } else if (which == 2) {
+        for (const AdapterDev& a : P.ad) v.insert(v.end(), {a.x_row, a.n, a.h_row, a.rp16, a.rp64});
+    } else if (which == 3) {
+        v = {P.RP, (int32_t)P.h_rows};
+    } else {
+        return PLORA_ERR_INVALID_ARG;
+    }
+    *count = (int64_t)v.size();
+    if (out) memcpy(out, v.data(), sizeof(int32_t) * (size_t)std::min<int64_t>(capacity, (int64_t)v.size()));
+    return PLORA_OK;
+}
+
+}  // extern "C"

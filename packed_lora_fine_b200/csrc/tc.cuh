@@ -1,0 +1,519 @@
+// tc.cuh -- the tensor-core (tcgen05 + TMEM + TMA) kernels of the bf16 path.
+//
+// One persistent, warp-specialised kernel template covers every product of
+// the packed LoRA forward and backward (the "four cases" of PLoRA's packed
+// operators -- forward, input gradient, and the two weight gradients that
+// reduce over the sequence -- plus the shared frozen-base GEMMs; PLoRA
+// summary, gist.science, arXiv 2508.02932, 技术摘要 › 方法论 › 2 › 算子设计):
+//
+//   op         computes                                 A operand (smem)        B operand (smem)
+//   BaseFwd    Y  = X W            (all tokens)          X      K-major          W_store    K-major
+//   BaseDx     dX = dY W^T         (all tokens)          dY     K-major          W_store    MN-major
+//   ShrinkX    H_i = X_i A_i       (per 128-token tile)   X      K-major          A pack     K-major
+//   ShrinkDy   G_i = s_i dY_i B_i^T                       dY     K-major          B^T pack   K-major
+//   ExpandY    Y_i += s_i H_i B_i                         H      K-major          B^T pack   MN-major
+//   ExpandDx   dX_i += G_i A_i^T                          G      K-major          A pack     MN-major
+//   WgradB     dB_i = s_i dY_i^T H_i (sum over tokens)    dY     MN-major         H          MN-major
+//   WgradA     dA_i = X_i^T G_i      (sum over tokens)    X      MN-major         G          MN-major
+//
+// Tiles run along the token (sequence) dimension for the shrink/expand
+// products and along the hidden dimension for the weight gradients -- never
+// along the small rank dimension; the rank is only the MMA's N (shrink) or K
+// (expand) extent, padded to 16.  Every tile of every adapter is one work
+// item of a static persistent schedule over all SMs, so adapters of unequal
+// rank and token count share one launch (the load balancing of 算子设计).
+//
+// Warp roles (192 threads): warp 0 issues TMA loads into a 4-stage ring,
+// warp 1 owns TMEM and issues tcgen05.mma into one of two 128x256 fp32
+// accumulators, warps 2-5 drain an accumulator (tcgen05.ld) and run the
+// op's epilogue while the next tile is being multiplied.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "plan.cuh"
+#include "ptx.cuh"
+
+namespace plora {
+
+enum class Op : int { BaseFwd = 0, BaseDx, ShrinkX, ShrinkDy, ExpandY, ExpandDx, WgradB, WgradA };
+
+template <Op OP> struct OpTraits {
+    static constexpr bool kAmn = (OP == Op::WgradB || OP == Op::WgradA);
+    static constexpr bool kBmn = (OP == Op::BaseDx || OP == Op::ExpandY || OP == Op::ExpandDx ||
+                                  OP == Op::WgradB || OP == Op::WgradA);
+    static constexpr bool kBase = (OP == Op::BaseFwd || OP == Op::BaseDx);
+    static constexpr bool kShrink = (OP == Op::ShrinkX || OP == Op::ShrinkDy);
+    static constexpr bool kExpand = (OP == Op::ExpandY || OP == Op::ExpandDx);
+    static constexpr bool kWgrad = (OP == Op::WgradB || OP == Op::WgradA);
+};
+
+constexpr int kStages = 4;
+constexpr int kTileN = 256;                       // N of the base / expand tiles (TMEM columns)
+constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB: 128 rows x 64 bf16
+constexpr int kBBytesMax = kTileN * kBlockK * 2;  // 32 KB: 256 rows x 64 bf16
+constexpr int kStageBytes = kABytes + kBBytesMax;
+constexpr int kTmemCols = 512;                    // two 256-column fp32 accumulators
+constexpr int kTcThreads = 192;
+constexpr int kTcSmemBytes = kStages * kStageBytes + 1024 /* align */ + 256 /* barriers */;
+
+struct TcParams {
+    int32_t M_total;        // Base: T; Wgrad: d (rows of dB_i or columns of dA_i)
+    int32_t N_total;        // Base / Expand: output columns
+    int32_t K_total;        // Base / Shrink: reduction length
+    int32_t tiles_m, tiles_n, num_tiles;
+    int32_t group_m;        // Base: rasterisation group (m tiles sharing an L2 window)
+    int32_t RP;             // padded rank pitch of H / G / packs
+    int32_t b_box_rows;     // K-major B: rows of the B box (Base: 256, Shrink: RP)
+    int32_t red_dtiles;     // Wgrad: 128-row tiles along d
+    const AdapterDev* adapters;
+    const TokTile* tok;
+    const RedEntry* red;
+    void* out;              // bf16 output of Base / Shrink / Expand
+    int64_t out_ld;         // its row pitch in elements
+    float* partials;        // Wgrad split partials, [slot][dtile][128][RP]
+    int32_t* counters;      // Wgrad split arrival counters
+    int* err_flag;
+    uint64_t timeout_ns;
+};
+
+struct TileInfo {
+    int32_t a_x, a_y, b_x, b_y;
+    int32_t kblocks, last_ksteps, mma_n, nb_boxes;
+    int32_t adapter, out_row, rows_valid, n0, cols_valid, red_idx;
+    float scale;
+};
+
+template <Op OP>
+__device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
+    using Tr = OpTraits<OP>;
+    TileInfo ti;
+    ti.last_ksteps = 4;
+    ti.nb_boxes = 1;
+    ti.scale = 1.f;
+    ti.adapter = -1;
+    ti.red_idx = -1;
+    if constexpr (Tr::kBase) {
+        // Grouped rasterisation: group_m m-tiles walk all n-tiles together.
+        const int per_group = p.group_m * p.tiles_n;
+        const int g = t / per_group;
+        const int first_m = g * p.group_m;
+        const int gm = min(p.tiles_m - first_m, p.group_m);
+        const int r = t - g * per_group;
+        const int mb = first_m + r % gm;
+        const int nb = r / gm;
+        ti.a_x = 0;
+        ti.a_y = mb * kTileM;
+        if constexpr (OP == Op::BaseFwd) { ti.b_x = 0; ti.b_y = nb * kTileN; }
+        else { ti.b_x = nb * kTileN; ti.b_y = 0; ti.nb_boxes = kTileN / 64; }
+        ti.kblocks = (p.K_total + kBlockK - 1) / kBlockK;
+        ti.mma_n = kTileN;
+        ti.out_row = mb * kTileM;
+        ti.rows_valid = min(kTileM, p.M_total - ti.out_row);
+        ti.n0 = nb * kTileN;
+        ti.cols_valid = min(kTileN, p.N_total - ti.n0);
+    } else if constexpr (Tr::kShrink) {
+        const TokTile tt = p.tok[t];
+        const AdapterDev ad = p.adapters[tt.adapter];
+        ti.adapter = tt.adapter;
+        ti.a_x = 0;
+        ti.a_y = tt.x_row;
+        ti.b_x = 0;
+        ti.b_y = tt.adapter * p.RP;
+        ti.kblocks = (p.K_total + kBlockK - 1) / kBlockK;
+        ti.mma_n = ad.rp16;
+        ti.out_row = tt.h_row;
+        ti.rows_valid = tt.rows;
+        ti.n0 = 0;
+        ti.cols_valid = p.RP;
+        ti.scale = (OP == Op::ShrinkDy) ? ad.scale : 1.f;
+    } else if constexpr (Tr::kExpand) {
+        const int mt = t / p.tiles_n;
+        const int nb = t - mt * p.tiles_n;
+        const TokTile tt = p.tok[mt];
+        const AdapterDev ad = p.adapters[tt.adapter];
+        ti.adapter = tt.adapter;
+        ti.a_x = 0;
+        ti.a_y = tt.h_row;
+        ti.b_x = nb * kTileN;
+        ti.b_y = tt.adapter * p.RP;
+        ti.nb_boxes = kTileN / 64;
+        const int ksteps = ad.rp16 / 16;
+        ti.kblocks = (ksteps + 3) / 4;
+        ti.last_ksteps = ksteps - (ti.kblocks - 1) * 4;
+        ti.mma_n = kTileN;
+        ti.out_row = tt.x_row;
+        ti.rows_valid = tt.rows;
+        ti.n0 = nb * kTileN;
+        ti.cols_valid = min(kTileN, p.N_total - ti.n0);
+        ti.scale = (OP == Op::ExpandY) ? ad.scale : 1.f;
+    } else {
+        const int e = t / p.red_dtiles;
+        const int db = t - e * p.red_dtiles;
+        const RedEntry re = p.red[e];
+        const AdapterDev ad = p.adapters[re.adapter];
+        ti.adapter = re.adapter;
+        ti.red_idx = e;
+        ti.a_x = db * kTileM;
+        ti.a_y = re.x_row;
+        ti.b_x = 0;
+        ti.b_y = re.h_row;
+        ti.nb_boxes = ad.rp64 / 64;
+        ti.kblocks = re.kblocks;
+        ti.mma_n = ad.rp64;
+        ti.out_row = db * kTileM;
+        ti.rows_valid = min(kTileM, p.M_total - ti.out_row);
+        ti.n0 = db;  // the d-tile index (for partial slots)
+        ti.cols_valid = ad.rank;
+        ti.scale = (OP == Op::WgradB) ? ad.scale : 1.f;
+    }
+    return ti;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+    return __bfloat1622float2(v);
+}
+
+template <Op OP>
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          const TcParams p) {
+    using Tr = OpTraits<OP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* full_bar = bars;                    // [kStages]
+    uint64_t* empty_bar = bars + kStages;         // [kStages]
+    uint64_t* accf_bar = bars + 2 * kStages;      // [2]
+    uint64_t* acce_bar = bars + 2 * kStages + 2;  // [2]
+    uint64_t* drain_bar = bars + 2 * kStages + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* red_flag = reinterpret_cast<int*>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&full_bar[s], 1);
+            ptx::mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&accf_bar[b], 1);
+            ptx::mbar_init(&acce_bar[b], 4);
+        }
+        ptx::mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&tmA);
+        ptx::tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc<kTmemCols>(tmem_slot);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint64_t lim = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+                const TileInfo ti = decode_tile<OP>(p, t);
+                const uint32_t b_bytes = Tr::kBmn ? (uint32_t)ti.nb_boxes * 8192u
+                                                  : (uint32_t)p.b_box_rows * 128u;
+                for (int kb = 0; kb < ti.kblocks; ++kb) {
+                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
+                    uint8_t* sA = smem + stage * kStageBytes;
+                    uint8_t* sB = sA + kABytes;
+                    ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + b_bytes);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    if constexpr (Tr::kAmn) {
+                        ptx::tma_load_2d(sA, &tmA, &full_bar[stage], ti.a_x, ti.a_y + kb * kBlockK);
+                        ptx::tma_load_2d(sA + 8192, &tmA, &full_bar[stage], ti.a_x + 64, ti.a_y + kb * kBlockK);
+                    } else {
+                        ptx::tma_load_2d(sA, &tmA, &full_bar[stage], ti.a_x + kb * kBlockK, ti.a_y);
+                    }
+                    if constexpr (Tr::kBmn) {
+                        for (int h = 0; h < ti.nb_boxes; ++h)
+                            ptx::tma_load_2d(sB + h * 8192, &tmB, &full_bar[stage], ti.b_x + 64 * h,
+                                             ti.b_y + kb * kBlockK);
+                    } else {
+                        ptx::tma_load_2d(sB, &tmB, &full_bar[stage], ti.b_x + kb * kBlockK, ti.b_y);
+                    }
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // Drain: every load this thread issued must have landed before the CTA exits.
+            for (int s = 0; s < kStages; ++s)
+                if (armed & (1u << s)) {
+                    int dummy = 0;
+                    ptx::mbar_wait(&full_bar[s], (armed_par >> s) & 1u, &dummy, lim, p.err_flag);
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int abuf = 0;
+            uint32_t aphase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+                const TileInfo ti = decode_tile<OP>(p, t);
+                const uint32_t idesc = ptx::idesc_bf16_f32(kTileM, ti.mma_n, Tr::kAmn, Tr::kBmn);
+                if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
+                for (int kb = 0; kb < ti.kblocks; ++kb) {
+                    if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, lim, p.err_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t sA = ptx::smem_u32(smem + stage * kStageBytes);
+                    const uint32_t sB = sA + kABytes;
+                    const int steps = (kb == ti.kblocks - 1) ? ti.last_ksteps : 4;
+                    for (int ks = 0; ks < steps; ++ks) {
+                        const uint64_t adesc = Tr::kAmn ? ptx::smem_desc_sw128(sA + ks * 2048, 8192, 1024)
+                                                        : ptx::smem_desc_sw128(sA + ks * 32, 16, 1024);
+                        const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, 8192, 1024)
+                                                        : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
+                        ptx::tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | ks) ? 1u : 0u);
+                    }
+                    ptx::tc_commit(&empty_bar[stage]);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::tc_commit(&accf_bar[abuf]);
+                if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+            }
+            // Drain: all issued MMAs complete before TMEM is released.
+            ptx::tc_commit(drain_bar);
+            int dummy = 0;
+            ptx::mbar_wait(drain_bar, 0, &dummy, lim, p.err_flag);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;          // accumulator row handled by this thread
+        int abuf = 0;
+        uint32_t aphase = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+            const TileInfo ti = decode_tile<OP>(p, t);
+            if (!ptx::mbar_wait(&accf_bar[abuf], aphase, abort_flag, lim, p.err_flag)) break;
+            ptx::tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
+            const bool row_ok = row < ti.rows_valid;
+
+            if constexpr (Tr::kBase) {
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
+                for (int c = 0; c < kTileN; c += 16) {
+                    uint32_t r[16];
+                    ptx::tmem_ld16(t_row + c, r);
+                    ptx::tmem_ld_wait();
+                    if (row_ok) {
+                        uint4 v0, v1;
+                        v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
+                        v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
+                        v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
+                        v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
+                        v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
+                        v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
+                        v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
+                        v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
+                        if (c + 8 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c) = v0;
+                        if (c + 16 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c + 8) = v1;
+                    }
+                }
+            } else if constexpr (Tr::kShrink) {
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld;
+                for (int c = 0; c < ti.cols_valid; c += 16) {
+                    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+                    if (c < ti.mma_n) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(t_row + c, r);
+                        ptx::tmem_ld_wait();
+                        if (row_ok) {
+                            const float s = ti.scale;
+                            v0.x = pack_bf16x2(s * __uint_as_float(r[0]), s * __uint_as_float(r[1]));
+                            v0.y = pack_bf16x2(s * __uint_as_float(r[2]), s * __uint_as_float(r[3]));
+                            v0.z = pack_bf16x2(s * __uint_as_float(r[4]), s * __uint_as_float(r[5]));
+                            v0.w = pack_bf16x2(s * __uint_as_float(r[6]), s * __uint_as_float(r[7]));
+                            v1.x = pack_bf16x2(s * __uint_as_float(r[8]), s * __uint_as_float(r[9]));
+                            v1.y = pack_bf16x2(s * __uint_as_float(r[10]), s * __uint_as_float(r[11]));
+                            v1.z = pack_bf16x2(s * __uint_as_float(r[12]), s * __uint_as_float(r[13]));
+                            v1.w = pack_bf16x2(s * __uint_as_float(r[14]), s * __uint_as_float(r[15]));
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(out + c) = v0;
+                    *reinterpret_cast<uint4*>(out + c + 8) = v1;
+                }
+            } else if constexpr (Tr::kExpand) {
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
+                const float s = ti.scale;
+                for (int h = 0; h < kTileN; h += 128) {
+                    uint4 y[16];
+                    if (row_ok) {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u)
+                            if (h + 8 * u + 8 <= ti.cols_valid) y[u] = *reinterpret_cast<const uint4*>(out + h + 8 * u);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; u += 2) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(t_row + h + 8 * u, r);
+                        ptx::tmem_ld_wait();
+                        if (row_ok) {
+#pragma unroll
+                            for (int w = 0; w < 2; ++w) {
+                                if (h + 8 * (u + w) + 8 > ti.cols_valid) continue;
+                                uint4 o = y[u + w];
+                                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    float2 f = unpack_bf16x2(ow[e]);
+                                    f.x += s * __uint_as_float(r[8 * w + 2 * e]);
+                                    f.y += s * __uint_as_float(r[8 * w + 2 * e + 1]);
+                                    ow[e] = pack_bf16x2(f.x, f.y);
+                                }
+                                *reinterpret_cast<uint4*>(out + h + 8 * (u + w)) = o;
+                            }
+                        }
+                    }
+                }
+            } else {
+                // Weight gradients: row = hidden index (d_out for dB, d_in for dA), column = rank index.
+                const RedEntry re = p.red[ti.red_idx];
+                const AdapterDev ad = p.adapters[ti.adapter];
+                const int rank = ad.rank;
+                const int hid = ti.out_row + row;
+                const float s = ti.scale;
+                if (re.nsplit == 1) {
+                    for (int c = 0; c < ti.mma_n; c += 16) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(t_row + c, r);
+                        ptx::tmem_ld_wait();
+                        if (row_ok) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int k = c + e;
+                                if (k < rank) {
+                                    const float v = s * __uint_as_float(r[e]);
+                                    if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = v;
+                                    else ad.dA[(int64_t)k * p.M_total + hid] = v;
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    // Split along the tokens: write this split's partial, the last split of the
+                    // tile to arrive sums all partials in split order (deterministic) and stores.
+                    const int64_t slot_elems = (int64_t)kTileM * p.RP;
+                    float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems
+                                  + (int64_t)row * p.RP;
+                    for (int c = 0; c < ti.mma_n; c += 16) {
+                        uint32_t r[16];
+                        ptx::tmem_ld16(t_row + c, r);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<float4*>(mine + c + e) =
+                                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+                    }
+                    __threadfence();
+                    ptx::named_bar_sync(1, 128);
+                    if (threadIdx.x == 64) {
+                        const int old = atomicAdd(&p.counters[re.counter + ti.n0], 1);
+                        *red_flag = (old == re.nsplit - 1) ? 1 : 0;
+                    }
+                    ptx::named_bar_sync(1, 128);
+                    if (*red_flag) {
+                        __threadfence();
+                        if (row_ok) {
+                            for (int k = 0; k < rank; ++k) {
+                                float acc = 0.f;
+                                for (int sp = 0; sp < re.nsplit; ++sp)
+                                    acc += __ldcg(p.partials + ((int64_t)(re.slot + sp) * p.red_dtiles + ti.n0) * slot_elems
+                                                  + (int64_t)row * p.RP + k);
+                                const float v = s * acc;
+                                if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = v;
+                                else ad.dA[(int64_t)k * p.M_total + hid] = v;
+                            }
+                        }
+                        if (threadIdx.x == 64) p.counters[re.counter + ti.n0] = 0;
+                    }
+                    ptx::named_bar_sync(1, 128);
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
+            if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc<kTmemCols>(tmem_base);
+}
+
+// ---------------------------------------------------------------------------
+// Packing of the small per-adapter factors into the MMA-ready padded layouts.
+//   packA [n*RP][d_in]:  row i*RP + k = A_i[k][:]       (k < r_i), zero for r_i <= k < RP
+//   packBT[n*RP][d_out]: row i*RP + k = B_i[:][k]       (k < r_i), zero for r_i <= k < RP
+// ---------------------------------------------------------------------------
+__global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, int64_t d_in,
+                              __nv_bfloat16* __restrict__ packA) {
+    const int64_t vec_per_row = d_in / 8;
+    const int64_t total = (int64_t)n * RP * vec_per_row;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rowi = e / vec_per_row;
+        const int64_t v = e - rowi * vec_per_row;
+        const int i = (int)(rowi / RP);
+        const int k = (int)(rowi - (int64_t)i * RP);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (k < ad[i].rank)
+            val = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ad[i].A) + (int64_t)k * d_in)[v];
+        reinterpret_cast<uint4*>(packA + rowi * d_in)[v] = val;
+    }
+}
+
+// grid: (ceil(d_out/64), n); block 256.  Stages B_i[c0..c0+63][0..r) in shared memory.
+__global__ void __launch_bounds__(256) pack_bt_kernel(const AdapterDev* __restrict__ ad, int RP, int64_t d_out,
+                                                      __nv_bfloat16* __restrict__ packBT) {
+    __shared__ __nv_bfloat16 tile[64][kRankAlign * 4 + 2];  // up to rank 256
+    const int i = blockIdx.y;
+    const int64_t c0 = (int64_t)blockIdx.x * 64;
+    const int r = ad[i].rank;
+    const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(ad[i].B);
+    const int cols = (int)(d_out - c0 < 64 ? d_out - c0 : 64);
+    for (int e = threadIdx.x; e < cols * r; e += blockDim.x) {
+        const int cc = e / r, k = e - cc * r;
+        tile[cc][k] = B[(c0 + cc) * r + k];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < RP * 64; e += blockDim.x) {
+        const int k = e >> 6, cc = e & 63;
+        if (cc < cols) {
+            const __nv_bfloat16 v = (k < r) ? tile[cc][k] : __float2bfloat16_rn(0.f);
+            packBT[((int64_t)i * RP + k) * d_out + c0 + cc] = v;
+        }
+    }
+}
+
+}  // namespace plora

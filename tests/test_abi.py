@@ -1,0 +1,184 @@
+"""Host-side tests of the C ABI: it loads, exports what include/plora.h declares,
+rejects bad configurations and tables, and its schedule covers every token of
+every adapter exactly once.  No kernel is launched."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import packed_lora_fine_b200 as pl
+from packed_lora_fine_b200 import build as plbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    plbuild.build()
+    pl.load()
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "plora.h")).read()
+    return sorted(set(re.findall(r"PLORA_API\s+[\w\s\*]+?\b(plora_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 11
+    lib = ctypes.CDLL(pl.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(pl.EXPORTED)
+
+
+def test_status_strings_and_version():
+    for code, name in [(0, "PLORA_OK"), (1, "PLORA_ERR_INVALID_ARG"), (2, "PLORA_ERR_UNSUPPORTED"),
+                       (3, "PLORA_ERR_OOM"), (4, "PLORA_ERR_CUDA"), (5, "PLORA_ERR_TIMEOUT")]:
+        assert pl.status_string(code) == name
+    assert pl.plora_version() >= 100
+
+
+def cfg(d_in=64, d_out=64, dtype=pl.PLORA_BF16, max_adapters=8, max_rank=64, max_tokens=4096, flags=0):
+    return pl.plora_config(d_in, d_out, dtype, max_adapters, max_rank, flags, max_tokens)
+
+
+@pytest.mark.parametrize("c, want", [
+    (cfg(d_in=60), pl.PLORA_ERR_UNSUPPORTED),
+    (cfg(d_out=4), pl.PLORA_ERR_UNSUPPORTED),
+    (cfg(d_in=1 << 17), pl.PLORA_ERR_UNSUPPORTED),
+    (cfg(dtype=7), pl.PLORA_ERR_UNSUPPORTED),
+    (cfg(max_adapters=0), pl.PLORA_ERR_INVALID_ARG),
+    (cfg(max_rank=257), pl.PLORA_ERR_INVALID_ARG),
+    (cfg(max_rank=0), pl.PLORA_ERR_INVALID_ARG),
+    (cfg(max_tokens=0), pl.PLORA_ERR_INVALID_ARG),
+    (cfg(flags=2), pl.PLORA_ERR_INVALID_ARG),
+])
+def test_create_rejects_bad_config(c, want):
+    s, h = pl.plora_create_status(c)
+    assert s == want and not h
+
+
+def test_create_without_gpu_fails_loudly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    s, h = pl.plora_create_status(cfg())
+    assert s == pl.PLORA_ERR_CUDA and not h
+
+
+def fake_table(ranks, aligned=True, grads=True):
+    base = 0x7f0000000000
+    n = len(ranks)
+    A = [base + 4096 * (4 * i) for i in range(n)]
+    B = [base + 4096 * (4 * i + 1) for i in range(n)]
+    dA = [base + 4096 * (4 * i + 2) for i in range(n)] if grads else None
+    dB = [base + 4096 * (4 * i + 3) for i in range(n)] if grads else None
+    if not aligned:
+        A[0] += 8
+    return pl.make_table(ranks, [2.0] * n, A, B, dA, dB)
+
+
+def schedule(c, off, ranks, which, grads=False, tab=None):
+    s, v = pl.plora_debug_schedule(c, len(off) - 1, off, tab if tab is not None else fake_table(ranks), grads,
+                                   which)
+    assert s == pl.PLORA_OK, pl.status_string(s)
+    return v
+
+
+@pytest.mark.parametrize("off, ranks, want", [
+    ([1, 5], [4], pl.PLORA_ERR_INVALID_ARG),              # off[0] != 0
+    ([0, 9, 5], [4, 4], pl.PLORA_ERR_INVALID_ARG),        # decreasing
+    ([0, 5000], [4], pl.PLORA_ERR_INVALID_ARG),           # > max_tokens
+    ([0, 5], [0], pl.PLORA_ERR_INVALID_ARG),              # rank 0
+    ([0, 5], [65], pl.PLORA_ERR_INVALID_ARG),             # rank > max_rank
+    ([0] * 10, [4] * 9, pl.PLORA_ERR_INVALID_ARG),        # n > max_adapters
+])
+def test_bad_tables_rejected(off, ranks, want):
+    s, _ = pl.plora_debug_schedule(cfg(), len(off) - 1, off, fake_table(ranks), False, 0)
+    assert s == want
+
+
+def test_null_and_misaligned_pointers_rejected():
+    c = cfg()
+    s, _ = pl.plora_debug_schedule(c, 1, [0, 5], fake_table([4], aligned=False), False, 0)
+    assert s == pl.PLORA_ERR_INVALID_ARG
+    s, _ = pl.plora_debug_schedule(c, 1, [0, 5], fake_table([4], grads=False), True, 0)
+    assert s == pl.PLORA_ERR_INVALID_ARG            # backward needs dA, dB
+    s, _ = pl.plora_debug_schedule(c, 1, [0, 5], fake_table([4], grads=False), False, 0)
+    assert s == pl.PLORA_OK                         # forward ignores them
+    t = fake_table([4])
+    t[0].scale = float("nan")
+    s, _ = pl.plora_debug_schedule(c, 1, [0, 5], t, False, 0)
+    assert s == pl.PLORA_ERR_INVALID_ARG
+
+
+def random_segments(seed, n, lo, hi, zero_frac=0.2):
+    g = np.random.default_rng(seed)
+    counts = g.integers(lo, hi + 1, size=n)
+    counts[g.random(n) < zero_frac] = 0
+    off = np.zeros(n + 1, np.int64)
+    off[1:] = np.cumsum(counts)
+    ranks = g.choice([1, 3, 8, 16, 17, 64, 100, 256], size=n)
+    return off, ranks
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_token_tiles_cover_every_row_once(seed):
+    off, ranks = random_segments(seed, 40, 0, 700)
+    c = cfg(max_adapters=64, max_rank=256, max_tokens=int(off[-1]) + 1)
+    tiles = schedule(c, off, ranks, 0).reshape(-1, 4)
+    ad = schedule(c, off, ranks, 2).reshape(-1, 5)
+    RP, h_rows = schedule(c, off, ranks, 3)
+    owner = np.full(int(off[-1]), -1)
+    for a, rows, x, hrow in tiles:
+        assert 1 <= rows <= 128
+        assert np.all(owner[x:x + rows] == -1)
+        owner[x:x + rows] = a
+        assert off[a] <= x and x + rows <= off[a + 1]
+        assert hrow - ad[a, 2] == x - off[a]               # same offset inside the adapter's block
+        assert (x - off[a]) % 128 == 0
+    assert np.array_equal(owner, np.repeat(np.arange(len(ranks)), np.diff(off)))   # bit-exact map
+    # H/G blocks: each adapter's block is its token count rounded up to 128, packed in order
+    blocks = ((np.diff(off) + 127) // 128) * 128
+    assert np.array_equal(ad[:, 2], np.concatenate([[0], np.cumsum(blocks)[:-1]]))
+    assert h_rows == blocks.sum()
+    assert RP == ((max(ranks) + 63) // 64) * 64
+    assert np.array_equal(ad[:, 3], ((ranks + 15) // 16) * 16)
+    assert np.array_equal(ad[:, 4], ((ranks + 63) // 64) * 64)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_weight_grad_splits_cover_tokens_and_depend_only_on_count(seed):
+    off, ranks = random_segments(seed, 24, 0, 13000)
+    c = cfg(max_adapters=64, max_rank=256, max_tokens=int(off[-1]) + 1)
+    red = schedule(c, off, ranks, 1, grads=True).reshape(-1, 8)
+    ks = red[:, 3]
+    assert np.all(ks[:-1] >= ks[1:])                       # longest first
+    n = np.diff(off)
+    for i in range(len(ranks)):
+        e = red[red[:, 0] == i]
+        if n[i] == 0:
+            assert len(e) == 0
+            continue
+        e = e[np.argsort(e[:, 4])]
+        S = (n[i] + 4095) // 4096
+        assert len(e) == S and np.all(e[:, 5] == S) and np.array_equal(e[:, 4], np.arange(S))
+        assert np.array_equal(e[:, 1], off[i] + 4096 * np.arange(S))
+        lens = np.minimum(4096, n[i] - 4096 * np.arange(S))
+        assert np.array_equal(e[:, 3], (lens + 63) // 64)
+        assert (S == 1) == (e[0, 6] == -1)
+        # the same adapter alone gets the same splits
+        alone = schedule(c, [0, n[i]], [ranks[i]], 1, grads=True).reshape(-1, 8)
+        alone = alone[np.argsort(alone[:, 4])]
+        assert np.array_equal(alone[:, 3:6], e[:, 3:6])
+        assert np.array_equal(alone[:, 1], e[:, 1] - off[i])
+
+
+def test_empty_call_is_valid():
+    v = schedule(cfg(), [0], [], 0)
+    assert len(v) == 0
+    v = schedule(cfg(), [0, 0, 0], [3, 5], 1, grads=True)
+    assert len(v) == 0
