@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Packed LoRA forward + backward throughput on B200.
+
+One step = one plora_forward + one plora_backward (all eight products of the
+packed layer plus the factor packing) over the LLaMA-3-8B up_proj workload
+(4096 -> 14336, bf16, 32 adapters, ranks U{8..128}, long-tail token counts
+log-uniform in [512, 4096]).  Inputs are seeded synthetic tensors of that
+shape, resident in HBM before the timed region (larger than L2, so no flush).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU; each rank packs
+its own 32 adapters (adapters are independent, so the work shards with no
+data-path collective: weak scaling); the step time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on the host cores instead.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import plora_workloads as wl  # noqa: E402
+
+METRIC = "packed LoRA fwd+bwd tokens/sec on 1 B200 (32 adapters); % HBM / tensor roofline"
+UNIT = "tokens/s"
+WORKLOAD = "llama3-8b up_proj 4096->14336 bf16, 32 adapters r~U{8,16,32,64,128}, tokens~logU[512,4096]"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TC_KINDS = ("base_fwd", "base_dx")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=1003)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["llama_up32", "small"], default="llama_up32",
+                    help="small: 8 adapters of the same mix cut to 2048 tokens each (for profiler captures)")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_work(p):
+    """Per-launch algorithmic work of every kernel kind of one step: (flops, bytes)."""
+    n = p.counts.astype(np.float64)
+    r = p.ranks.astype(np.float64)
+    di, do = float(p.d_in), float(p.d_out)
+    T = float(p.T)
+    RP = math.ceil(max(p.ranks) / 64) * 64
+    w = {
+        "base_fwd": (2 * T * di * do, 2 * (T * di + di * do + T * do)),
+        "base_dx": (2 * T * di * do, 2 * (T * do + di * do + T * di)),
+        "shrink_x": (float(np.sum(2 * n * di * r)), float(np.sum(n * (2 * di + 2 * r) + 2 * r * di))),
+        "expand_y": (float(np.sum(2 * n * do * r)), float(np.sum(n * (4 * do + 2 * r) + 2 * r * do))),
+        "shrink_dy": (float(np.sum(2 * n * do * r)), float(np.sum(n * (2 * do + 2 * r) + 2 * r * do))),
+        "expand_dx": (float(np.sum(2 * n * di * r)), float(np.sum(n * (4 * di + 2 * r) + 2 * r * di))),
+        "wgrad_b": (float(np.sum(2 * n * do * r)), float(np.sum(n * (2 * do + 2 * r) + 4 * r * do))),
+        "wgrad_a": (float(np.sum(2 * n * di * r)), float(np.sum(n * (2 * di + 2 * r) + 4 * r * di))),
+        "pack_a": (0.0, float(np.sum(2 * r * di)) + 2 * len(r) * RP * di),
+        "pack_bt": (0.0, float(np.sum(2 * r * do)) + 2 * len(r) * RP * do),
+    }
+    return w
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="plora_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id, "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def reduce_max(x: float, dist) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_initialized():
+        return float(x)
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, dist) -> float:
+    if dist is None or not dist.is_initialized():
+        return float(x)
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_problem(seed: int, adapters: int, tokens_each: int):
+    """A bounded sample of the workload: the first `adapters` adapters of the 32-adapter mix,
+    each cut to `tokens_each` tokens, same layer shapes and distributions."""
+    ranks, counts, alphas = wl.config3_shape(seed)
+    k = adapters
+    return wl.make_problem("cfg3_sample", "bf16", 4096, 14336, ranks[:k], [tokens_each] * k, alphas[:k],
+                           wl.init_llm(4096), seed + 7777)
+
+
+def time_oracle(p, nthreads: int) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    oracle.full(p, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(seed: int) -> dict:
+    import oracle
+    oracle.build()
+    cores = host_cores()
+    nt = min(cores, oracle.num_procs())
+    p = oracle_sample_problem(seed, 8, 4)
+    time_oracle(oracle_sample_problem(seed, 1, 1), nt)  # load / page in
+    dt = time_oracle(p, nt)
+    return {"value": p.T / dt, "unit": UNIT, "cores": nt, "kind": "oracle",
+            "sample": f"fp64 oracle fwd+bwd (Y, dX, dA, dB) of {p.T} tokens: the first 8 adapters of the "
+                      f"32-adapter LLaMA-3-8B up_proj mix cut to 4 tokens each; {dt:.2f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    cores = host_cores()
+    nt = min(cores, oracle.num_procs())
+    # Size the per-step sample so the whole run stays within a few minutes.
+    probe = oracle_sample_problem(args.seed, 2, 2)
+    time_oracle(probe, nt)
+    t_tok = time_oracle(probe, nt) / probe.T
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    tokens_each = int(max(1, min(8, budget / t_tok / 8)))
+    p = oracle_sample_problem(args.seed, 8, tokens_each)
+    for _ in range(args.warmup):
+        time_oracle(p, nt)
+    total = 0.0
+    for _ in range(args.steps):
+        total += time_oracle(p, nt)
+    ms = 1000.0 * total / args.steps
+    value = p.T / (ms / 1000.0)
+    sample = (f"fp64 oracle fwd+bwd of {p.T} tokens per step (first 8 adapters of the 32-adapter mix, "
+              f"{tokens_each} tokens each) on {nt} host threads")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "adapters": 8, "tokens_per_step": p.T, "d_in": 4096,
+                       "d_out": 14336},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nt, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import packed_lora_fine_b200 as pl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        dist = None
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peaks_src = load_peaks()
+
+    if args.workload == "small":
+        ranks, counts, alphas = wl.config3_shape(args.seed)
+        p = wl.make_problem("cfg3_small", "bf16", 4096, 14336, ranks[:8], [2048] * 8, alphas[:8],
+                            wl.init_llm(4096), args.seed + 1000 * rank)
+    else:
+        p = wl.config3(seed=args.seed + 1000 * rank)
+    T = p.T
+
+    def tdev(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)
+
+    X, W, dY = tdev(p.X), tdev(p.W), tdev(p.dY)
+    A = [tdev(a) for a in p.A]
+    B = [tdev(b) for b in p.B]
+    Y = torch.empty((T, p.d_out), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((T, p.d_in), dtype=torch.bfloat16, device=dev)
+    dA = [torch.empty(a.shape, dtype=torch.float32, device=dev) for a in A]
+    dB = [torch.empty(b.shape, dtype=torch.float32, device=dev) for b in B]
+    eng = pl.PackedLoRA(p.d_in, p.d_out, "bf16", max_adapters=p.n_adapters, max_rank=int(max(p.ranks)),
+                        max_tokens=T)
+    tab_f = eng.table(p.scales, A, B)
+    tab_b = eng.table(p.scales, A, B, dA, dB)
+    saved = torch.empty(eng.saved_bytes(p.off, tab_f), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    st = stream.cuda_stream
+    n = p.n_adapters
+    off = np.ascontiguousarray(p.off, dtype=np.int64)
+
+    def step():
+        pl.plora_forward(eng.h, X.data_ptr(), W.data_ptr(), Y.data_ptr(), n, off, tab_f, saved.data_ptr(), st)
+        pl.plora_backward(eng.h, X.data_ptr(), W.data_ptr(), dY.data_ptr(), dX.data_ptr(), n, off, tab_b,
+                          saved.data_ptr(), st)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert pl.plora_check(eng.h, st) == pl.PLORA_OK
+    pl.plora_profile_read(eng.h)          # reset the counters
+    pl.plora_profile_enable(eng.h, True)
+
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    if not gpu_uuid.startswith("GPU-"):
+        gpu_uuid = "GPU-" + gpu_uuid
+    clocks = ClockSampler(gpu_uuid)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    prof = pl.plora_profile_read(eng.h)
+    pl.plora_profile_enable(eng.h, False)
+    assert pl.plora_check(eng.h, st) == pl.PLORA_OK
+    ms = reduce_max(ms_local, dist)
+    tokens_all = reduce_sum(T, dist)
+    value = tokens_all / (ms / 1000.0)
+
+    # Per-kernel roofline (device time from events bracketing each launch on its stream).
+    work = algorithmic_work(p)
+    kernels = {}
+    launches = 0
+    for kind, (cnt, tot) in prof.items():
+        launches += cnt
+        if cnt == 0:
+            continue
+        avg_ms = tot / cnt
+        fl, by = work.get(kind, (0.0, 0.0))
+        if kind in TC_KINDS:
+            ach = fl / (avg_ms / 1e3) / 1e12
+            kernels[kind] = {"launches": cnt, "avg_ms": avg_ms, "bound": "tensor", "achieved": ach,
+                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"]}
+        else:
+            ach = by / (avg_ms / 1e3) / 1e9
+            kernels[kind] = {"launches": cnt, "avg_ms": avg_ms, "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                             "frac": ach / peaks["hbm_gbs"]}
+    dom = max(kernels, key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
+    kd = kernels[dom]
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            tr = json.load(f)
+        e = tr.get(dom)
+        if e and e.get("source_sha") == source_sha():
+            traffic = e["bytes_per_launch"]
+    except Exception:
+        pass
+    peak_key = "bf16_tflops_sustained" if kd["bound"] == "tensor" else "hbm_gbs"
+    roofline = {"bound": kd["bound"], "achieved": kd["achieved"], "peak": peaks[peak_key], "unit": kd["unit"],
+                "frac": kd["frac"], "traffic": traffic, "kernel": dom,
+                "peak_source": f"{peaks_src} {peak_key}"}
+
+    # End to end through the C ABI with host buffers: every step copies X and dY in from pinned
+    # host memory, runs forward + backward, and copies every adapter's dA, dB out to pinned memory.
+    e2e = None
+    if not args.no_e2e:
+        hX = torch.empty(X.shape, dtype=X.dtype, pin_memory=True).copy_(X.cpu())
+        hdY = torch.empty(dY.shape, dtype=dY.dtype, pin_memory=True).copy_(dY.cpu())
+        hdA = [torch.empty(a.shape, dtype=torch.float32, pin_memory=True) for a in dA]
+        hdB = [torch.empty(b.shape, dtype=torch.float32, pin_memory=True) for b in dB]
+        h2d = hX.numel() * 2 + hdY.numel() * 2
+        d2h = sum(a.numel() * 4 for a in hdA) + sum(b.numel() * 4 for b in hdB)
+
+        def e2e_step():
+            X.copy_(hX, non_blocking=True)
+            dY.copy_(hdY, non_blocking=True)
+            step()
+            for a, h in zip(dA, hdA):
+                h.copy_(a, non_blocking=True)
+            for b, h in zip(dB, hdB):
+                h.copy_(b, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k2 = max(5, min(args.steps, 20))
+        e0.record(stream)
+        for _ in range(k2):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = reduce_max(e0.elapsed_time(e1) / k2, dist)
+        e2e = {"value": tokens_all / (ms_e2e / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": k2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.seed)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "adapters": n, "tokens_per_gpu": T, "global_tokens": int(tokens_all),
+                           "d_in": p.d_in, "d_out": p.d_out, "parallelism": f"adapter-sharded x{world}",
+                           "l2": "inputs larger than L2 (X 452 MB, dY 1.6 GB); no flush"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+                "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+                "kernels": kernels}
+        print(json.dumps(line), flush=True)
+    eng.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def source_sha() -> str:
+    """Hash of the kernel sources, to tell whether committed ncu counters still describe them."""
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "packed_lora_fine_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    sys.exit(main())
