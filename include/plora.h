@@ -226,6 +226,46 @@ PLORA_API plora_status plora_profile_enable(plora_handle h, int32_t enable);
 PLORA_API plora_status plora_profile_read(plora_handle h, int32_t capacity, int32_t* n_kinds,
                                           const char** names, int64_t* launches, double* total_ms);
 
+/*
+ * Allocation-free dB: dB_i = s_i H_i^T dY_i for every adapter -- the same
+ * product, schedule and results as the dB part of plora_backward -- without a
+ * handle and without allocating anything.  The paper has no counterpart; this
+ * entry point exists for callers that cannot allocate device memory: code
+ * running under a memory planner or a caching allocator that owns the whole
+ * device and forbids any other cudaMalloc, code that must not synchronise the
+ * device (cudaMalloc and cudaFree can), and hosts that hand a library only
+ * the tensors it works on.
+ *
+ * Its scratch (schedule, token-split partials, arrival counters, error flag)
+ * is one static device array of PLORA_STATIC_SCRATCH_BYTES that every GPU
+ * loading this library holds until the process exits.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * cfg: as for plora_create (bf16, no PLORA_FLAG_SIMT; the max_* fields bound
+ * the call).  dY: [T][d_out] bf16 device; saved: the buffer a plora_forward
+ * with the same off and adapter ranks filled; off, tab: host arrays as for
+ * plora_backward (only rank, scale and dB are read; dB must be non-NULL and
+ * 16-byte aligned, A and B must still be valid pointers).  Writes every dB_i.
+ *
+ * Returns PLORA_ERR_UNSUPPORTED if the call's schedule (64 bytes per adapter
+ * plus 32 bytes per 4096-token split) exceeds 1 MiB - 256 bytes, or if its
+ * split partials exceed the rest of the array: (splits of adapters longer
+ * than 4096 tokens) x ceil(d_out/128) x (4 + 128 x RP x 4) bytes must fit in
+ * PLORA_STATIC_SCRATCH_BYTES - 1 MiB, RP = max rank rounded up to 64.  Other errors as for
+ * plora_backward; a device wait that runs out of time is not reported
+ * (there is no handle to report it through).
+ *
+ * The first call on each device resolves the array's device address and sets
+ * the kernel up; make that first call before any stream capture.  Every call
+ * shares the one array and clears what must start at zero; calls whose work
+ * overlaps on the GPU (different streams, or different host threads) race on
+ * it and must be serialised by the caller.
+ */
+#define PLORA_STATIC_SCRATCH_BYTES (16u << 20)
+PLORA_API plora_status plora_grad_B_static(const plora_config* cfg, const void* dY, int32_t n_adapters,
+                                           const int64_t* off, const plora_adapter* tab, const void* saved,
+                                           void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 PLORA_API int32_t plora_version(void);
 

@@ -36,7 +36,8 @@ PLORA_MAX_ADAPTERS = 4096
 
 EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
-            "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read")
+            "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
+            "plora_grad_B_static")
 
 
 class plora_config(ctypes.Structure):
@@ -87,6 +88,8 @@ def load(path: str = LIB_PATH):
     lib.plora_profile_enable.restype = ctypes.c_int
     lib.plora_profile_read.argtypes = [H, I32, ctypes.POINTER(I32), P, P, P]
     lib.plora_profile_read.restype = ctypes.c_int
+    lib.plora_grad_B_static.argtypes = [ctypes.POINTER(plora_config), P, I32, P, P, P, P]
+    lib.plora_grad_B_static.restype = ctypes.c_int
     lib.plora_version.argtypes = []
     lib.plora_version.restype = ctypes.c_int32
     for fn in ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
@@ -217,6 +220,13 @@ def plora_profile_read(h: int) -> dict:
     ms = (ctypes.c_double * cap)()
     _raise(h, lib.plora_profile_read(h, cap, ctypes.byref(n), names, launches, ms))
     return {names[k].decode(): (int(launches[k]), float(ms[k])) for k in range(min(n.value, cap))}
+
+
+def plora_grad_B_static(cfg: plora_config, dY: int, n: int, off, tab, saved: int, stream: int = 0) -> int:
+    """dB of every adapter without allocating (scratch in a static device array). Returns the status."""
+    off = _offsets(off)
+    return int(load().plora_grad_B_static(ctypes.byref(cfg), dY, n, off.ctypes.data, ctypes.addressof(tab),
+                                          saved, stream))
 
 
 def plora_version() -> int:

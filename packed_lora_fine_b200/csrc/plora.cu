@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -814,3 +815,140 @@ plora_status plora_debug_schedule(const plora_config* cfg, int32_t n, const int6
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free variant of the dB weight-gradient product.
+//
+// Its scratch -- the adapter table and token splits the kernel reads, the split
+// partials, their arrival counters and the device error flag -- lives in one
+// file-scope device array instead of a handle's cudaMalloc'd workspace.  The
+// array is created with the module on every GPU that loads this library and
+// stays until the process exits.  Host code cannot use the array's name as a
+// device address (on the host it only stands for the symbol), so the first
+// call on each device looks the address up with cudaGetSymbolAddress and
+// passes that pointer to the kernel.
+// ===========================================================================
+namespace {
+
+constexpr size_t kStaticScratchBytes = PLORA_STATIC_SCRATCH_BYTES;
+constexpr size_t kStaticSchedBytes = (size_t)1 << 20;      // error flag + adapter table + splits
+constexpr int kStaticMaxDevices = 64;
+
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_plora_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+struct StaticDevice {
+    uint8_t* scratch = nullptr;   // device address of g_plora_static_scratch on this device
+    int num_sms = 0;
+};
+std::mutex g_static_mu;
+StaticDevice g_static_dev[kStaticMaxDevices];
+
+// Once per device, with that device current: resolve the array's device address, the
+// tensor-map encoder and the kernel's shared-memory limit.  None of these allocate.
+plora_status static_setup(int dev, StaticDevice& out) {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    StaticDevice& d = g_static_dev[dev];
+    if (!d.scratch) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_plora_static_scratch);
+        if (e != cudaSuccess || p == nullptr) return PLORA_ERR_CUDA;
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return PLORA_ERR_CUDA;
+        if (!get_encode()) return PLORA_ERR_CUDA;
+        e = cudaFuncSetAttribute(tc_kernel<Op::WgradB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+        if (e != cudaSuccess) return PLORA_ERR_CUDA;
+        d.num_sms = sms;
+        d.scratch = static_cast<uint8_t*>(p);
+    }
+    out = d;
+    return PLORA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void* dY, int32_t n, const int64_t* off,
+                                            const plora_adapter* tab, const void* saved, void* stream) {
+    if (!cfg) return PLORA_ERR_INVALID_ARG;
+    if (cfg->dtype != PLORA_BF16 || (cfg->flags & PLORA_FLAG_SIMT)) return PLORA_ERR_UNSUPPORTED;
+    if (cfg->d_in < 8 || cfg->d_out < 8 || cfg->d_in > 65536 || cfg->d_out > 65536 || cfg->d_in % 8 ||
+        cfg->d_out % 8)
+        return PLORA_ERR_UNSUPPORTED;
+    if (cfg->max_adapters < 1 || cfg->max_adapters > PLORA_MAX_ADAPTERS || cfg->max_rank < 1 ||
+        cfg->max_rank > PLORA_MAX_RANK || cfg->max_tokens < 1 || cfg->max_tokens > ((int64_t)1 << 30))
+        return PLORA_ERR_INVALID_ARG;
+    plora_ctx tmp;
+    tmp.cfg = *cfg;
+    tmp.esize = 2;
+    plora_status s = check_table(&tmp, n, off, tab, false);
+    if (s != PLORA_OK) return s;
+    for (int32_t i = 0; i < n; ++i)
+        if (!tab[i].dB || !aligned16(tab[i].dB)) return PLORA_ERR_INVALID_ARG;
+    const bool any_tokens = off[n] > 0;
+    if (any_tokens && (!dY || !saved)) return PLORA_ERR_INVALID_ARG;
+    if (!aligned16(dY) || (reinterpret_cast<uintptr_t>(saved) & 255u) != 0) return PLORA_ERR_INVALID_ARG;
+
+    HostPlan P;
+    build_plan(&tmp, n, off, tab, P);
+    const int64_t d_out = cfg->d_out;
+    const int32_t dtiles = (int32_t)ceil_div(d_out, kTileM);
+    // Scratch layout: [0,256) error flag | adapter table | splits  (within kStaticSchedBytes)
+    //                 | counters | partials                         (the rest of the array)
+    const size_t o_ad = 256;
+    const size_t o_red = align256(o_ad + P.ad.size() * sizeof(AdapterDev));
+    const size_t sched_end = align256(o_red + P.red.size() * sizeof(RedEntry));
+    const size_t o_cnt = kStaticSchedBytes;
+    const size_t o_part = align256(o_cnt + (size_t)P.slots * dtiles * sizeof(int32_t));
+    const size_t part_end = o_part + (size_t)P.slots * dtiles * kTileM * (size_t)P.RP * sizeof(float);
+    if (sched_end > kStaticSchedBytes || part_end > kStaticScratchBytes) return PLORA_ERR_UNSUPPORTED;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStaticMaxDevices) return PLORA_ERR_CUDA;
+    StaticDevice sd;
+    s = static_setup(dev, sd);
+    if (s != PLORA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // Adapters without tokens get dB = 0.
+    for (int32_t i : P.empty)
+        if (cudaMemsetAsync(tab[i].dB, 0, (size_t)tab[i].rank * d_out * sizeof(float), st) != cudaSuccess)
+            return PLORA_ERR_CUDA;
+    if (P.T == 0) return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
+
+    // The array keeps the previous call's contents: clear the error flag and the arrival
+    // counters, then copy this call's schedule in.
+    uint8_t* base = sd.scratch;
+    if (cudaMemsetAsync(base, 0, 256, st) != cudaSuccess) return PLORA_ERR_CUDA;
+    if (P.slots > 0 && cudaMemsetAsync(base + o_cnt, 0, (size_t)P.slots * dtiles * sizeof(int32_t), st) != cudaSuccess)
+        return PLORA_ERR_CUDA;
+    if (cudaMemcpyAsync(base + o_ad, P.ad.data(), P.ad.size() * sizeof(AdapterDev), cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(base + o_red, P.red.data(), P.red.size() * sizeof(RedEntry), cudaMemcpyHostToDevice, st) !=
+            cudaSuccess)
+        return PLORA_ERR_CUDA;
+
+    CUtensorMap mdY, mH;
+    if (!make_map(&mdY, dY, d_out, P.T, d_out, 64, 64) || !make_map(&mH, saved, P.RP, P.h_rows, P.RP, 64, 64))
+        return PLORA_ERR_CUDA;
+    TcParams p{};
+    p.RP = P.RP;
+    p.adapters = reinterpret_cast<const AdapterDev*>(base + o_ad);
+    p.red = reinterpret_cast<const RedEntry*>(base + o_red);
+    p.err_flag = reinterpret_cast<int*>(base);
+    p.timeout_ns = kTimeoutNs;
+    p.partials = reinterpret_cast<float*>(base + o_part);
+    p.counters = reinterpret_cast<int32_t*>(base + o_cnt);
+    p.group_m = 16;
+    p.M_total = (int32_t)d_out;
+    p.red_dtiles = dtiles;
+    p.num_tiles = (int32_t)P.red.size() * dtiles;
+    if (p.num_tiles > 0)
+        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, p);
+    return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
+}
