@@ -51,8 +51,13 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=1003)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["llama_up32", "small"], default="llama_up32",
-                    help="small: 8 adapters of the same mix cut to 2048 tokens each (for profiler captures)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run the expand products as separate passes (for comparison with the fused default)")
+    ap.add_argument("--suite", action="store_true",
+                    help="measure every workload (packed vs per-adapter sequential loop); one JSON line each")
+    ap.add_argument("--workload", choices=["llama_up32", "small", "layer_q"], default="llama_up32",
+                    help="small: 8 adapters of the same mix cut to 2048 tokens each; layer_q: the 4096x4096 q_proj "
+                         "of the one-layer workload, 16 adapters x 8192 tokens (both for profiler captures)")
     return ap.parse_args(argv)
 
 
@@ -232,6 +237,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.suite:
+        return run_suite(args)
 
     import torch
     import torch.distributed as dist
@@ -254,6 +261,8 @@ def main(argv=None):
         ranks, counts, alphas = wl.config3_shape(args.seed)
         p = wl.make_problem("cfg3_small", "bf16", 4096, 14336, ranks[:8], [2048] * 8, alphas[:8],
                             wl.init_llm(4096), args.seed + 1000 * rank)
+    elif args.workload == "layer_q":
+        p = wl.config4(seed=1004)[0]
     else:
         p = wl.config3(seed=args.seed + 1000 * rank)
     T = p.T
@@ -269,7 +278,7 @@ def main(argv=None):
     dA = [torch.empty(a.shape, dtype=torch.float32, device=dev) for a in A]
     dB = [torch.empty(b.shape, dtype=torch.float32, device=dev) for b in B]
     eng = pl.PackedLoRA(p.d_in, p.d_out, "bf16", max_adapters=p.n_adapters, max_rank=int(max(p.ranks)),
-                        max_tokens=T)
+                        max_tokens=T, unfused=args.unfused)
     tab_f = eng.table(p.scales, A, B)
     tab_b = eng.table(p.scales, A, B, dA, dB)
     saved = torch.empty(eng.saved_bytes(p.off, tab_f), dtype=torch.uint8, device=dev)
@@ -419,6 +428,141 @@ def source_sha() -> str:
             h.update(f.encode())
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+
+# ----------------------------------------------------------------------------- measurement suite
+def _suite_problem_shapes():
+    """(name, [(d_in, d_out), ...], ranks, counts, alphas) of every suite workload."""
+    out = []
+    r2 = [8, 8, 16, 16, 32, 32, 64, 64]
+    out.append(("qwen2.5-7b q_proj 3584x3584, 8 adapters", [(3584, 3584)], r2, [2048] * 8, [2.0 * x for x in r2]))
+    r3, c3, a3 = wl.config3_shape(1003)
+    out.append(("llama3-8b up_proj 4096x14336, 32 adapters (long tail)", [(4096, 14336)], list(r3), list(c3),
+                list(a3)))
+    r4 = list(wl.rng_for(1004, 1).choice(np.array([16, 32, 64]), size=16))
+    out.append(("llama3-8b layer: 7 projections, 16 adapters x 8192 tokens",
+                [(di, do) for _, di, do in wl.LLAMA3_LAYER], r4, [8192] * 16, [2.0 * x for x in r4]))
+    for k in (1, 2, 4, 8, 16, 32):
+        out.append((f"scaling 4096x4096 r16, {k} adapters x 2048 tokens", [(4096, 4096)], [16] * k, [2048] * k,
+                    [32.0] * k))
+    for which in ("i", "ii", "iii", "iv"):
+        p = wl.config5_mix(which)
+        out.append((f"degenerate mix {which} 4096x4096", [(4096, 4096)], [int(x) for x in p.ranks],
+                    [int(x) for x in p.counts], [float(x) for x in p.alphas]))
+    return out
+
+
+def run_suite(args):
+    """Packed fwd+bwd tokens/s and per-kernel roofline on every workload, next to the same kernels run
+    once per adapter (the naive sequential loop).  One JSON line per workload."""
+    import torch
+    import packed_lora_fine_b200 as pl
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    g = torch.Generator(device=dev)
+    g.manual_seed(args.seed)
+    st = torch.cuda.current_stream(dev)
+    for name, projs, ranks, counts, alphas in _suite_problem_shapes():
+        n = len(ranks)
+        off = np.zeros(n + 1, np.int64)
+        off[1:] = np.cumsum(counts)
+        T = int(off[-1])
+        scales = [a / r for a, r in zip(alphas, ranks)]
+        layers = []
+        for di, do in projs:
+            X = (torch.randn((T, di), generator=g, device=dev)).to(torch.bfloat16)
+            dY = (torch.randn((T, do), generator=g, device=dev)).to(torch.bfloat16)
+            W = (torch.randn((do, di), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+            bound = math.sqrt(6.0 / di)
+            A = [((torch.rand((r, di), generator=g, device=dev) * 2 - 1) * bound).to(torch.bfloat16) for r in ranks]
+            B = [(torch.randn((do, r), generator=g, device=dev) * 0.01).to(torch.bfloat16) for r in ranks]
+            eng = pl.PackedLoRA(di, do, "bf16", max_adapters=n, max_rank=max(ranks), max_tokens=max(T, 1))
+            Y = torch.empty((T, do), dtype=torch.bfloat16, device=dev)
+            dX = torch.empty((T, di), dtype=torch.bfloat16, device=dev)
+            dA = [torch.empty(a.shape, dtype=torch.float32, device=dev) for a in A]
+            dB = [torch.empty(b.shape, dtype=torch.float32, device=dev) for b in B]
+            tf = eng.table(scales, A, B)
+            tb = eng.table(scales, A, B, dA, dB)
+            saved = torch.empty(max(256, eng.saved_bytes(off, tf)), dtype=torch.uint8, device=dev)
+            # the sequential loop: one handle call per adapter on its own slice
+            seq = []
+            for i in range(n):
+                a, b = int(off[i]), int(off[i + 1])
+                o1 = np.array([0, b - a], np.int64)
+                t1f = eng.table([scales[i]], [A[i]], [B[i]])
+                t1b = eng.table([scales[i]], [A[i]], [B[i]], [dA[i]], [dB[i]])
+                sv = torch.empty(max(256, eng.saved_bytes(o1, t1f)), dtype=torch.uint8, device=dev)
+                seq.append((a, b, o1, t1f, t1b, sv))
+            layers.append(dict(X=X, dY=dY, W=W, A=A, B=B, eng=eng, Y=Y, dX=dX, tf=tf, tb=tb, saved=saved, seq=seq,
+                               di=di, do=do))
+
+        def packed_step():
+            for L in layers:
+                e = L["eng"]
+                pl.plora_forward(e.h, L["X"].data_ptr(), L["W"].data_ptr(), L["Y"].data_ptr(), n, off, L["tf"],
+                                 L["saved"].data_ptr(), st.cuda_stream)
+                pl.plora_backward(e.h, L["X"].data_ptr(), L["W"].data_ptr(), L["dY"].data_ptr(),
+                                  L["dX"].data_ptr(), n, off, L["tb"], L["saved"].data_ptr(), st.cuda_stream)
+
+        def seq_step():
+            for L in layers:
+                e = L["eng"]
+                esz = 2
+                for (a, b, o1, t1f, t1b, sv) in L["seq"]:
+                    xp = L["X"].data_ptr() + a * L["di"] * esz
+                    yp = L["Y"].data_ptr() + a * L["do"] * esz
+                    dyp = L["dY"].data_ptr() + a * L["do"] * esz
+                    dxp = L["dX"].data_ptr() + a * L["di"] * esz
+                    pl.plora_forward(e.h, xp, L["W"].data_ptr(), yp, 1, o1, t1f, sv.data_ptr(), st.cuda_stream)
+                    pl.plora_backward(e.h, xp, L["W"].data_ptr(), dyp, dxp, 1, o1, t1b, sv.data_ptr(),
+                                      st.cuda_stream)
+
+        def timed(fn, steps, profile=False):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            for L in layers:
+                pl.plora_profile_read(L["eng"].h)
+                pl.plora_profile_enable(L["eng"].h, profile)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for _ in range(steps):
+                fn()
+            e1.record(st)
+            torch.cuda.synchronize()
+            prof = {}
+            for L in layers:
+                for k, (c, ms) in pl.plora_profile_read(L["eng"].h).items():
+                    pc, pm = prof.get(k, (0, 0.0))
+                    prof[k] = (pc + c, pm + ms)
+                pl.plora_profile_enable(L["eng"].h, False)
+            return e0.elapsed_time(e1) / steps, prof
+
+        steps = max(5, min(args.steps, 30))
+        ms_p, prof = timed(packed_step, steps, profile=True)
+        ms_s, _ = timed(seq_step, max(3, steps // 3))
+        kern = {}
+        for k, (c, tot) in prof.items():
+            if c:
+                kern[k] = {"launches": c, "ms_per_step": tot / steps}
+        base_ms = sum(v["ms_per_step"] for k, v in kern.items() if k in TC_KINDS)
+        base_flops = sum(4.0 * T * L["di"] * L["do"] for L in layers)
+        line = {"suite": name, "tokens": T, "adapters": n, "projections": len(layers),
+                "packed_ms_per_step": ms_p, "packed_tokens_per_s": T / (ms_p / 1e3),
+                "sequential_ms_per_step": ms_s, "sequential_tokens_per_s": T / (ms_s / 1e3),
+                "packed_over_sequential": ms_s / ms_p,
+                "base_gemm_tflops": base_flops / (base_ms / 1e3) / 1e12 if base_ms else None,
+                "base_gemm_frac_of_sustained_peak": (base_flops / (base_ms / 1e3) / 1e12) / peaks["bf16_tflops_sustained"]
+                if base_ms else None,
+                "kernels_ms_per_step": {k: round(v["ms_per_step"], 4) for k, v in kern.items()}}
+        print(json.dumps(line), flush=True)
+        for L in layers:
+            L["eng"].close()
+        del layers
+        torch.cuda.empty_cache()
+    return 0
 
 
 if __name__ == "__main__":

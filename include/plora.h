@@ -47,7 +47,12 @@
  *
  * Errors.  Every argument is checked before anything is enqueued; on an
  * error nothing is written and the call returns a non-zero status, with a
- * message available from plora_last_error().  No C++ exception crosses this
+ * message available from plora_last_error().  This includes the memory:
+ * every tensor pointer must lie inside one device allocation that holds the
+ * tensor's whole extent (checked against the driver's allocation record,
+ * so at the granularity of cudaMalloc: a sub-allocator's slice is checked
+ * against its whole segment), else the call returns PLORA_ERR_INVALID_ARG
+ * and launches nothing.  No C++ exception crosses this
  * ABI.  An asynchronous device failure surfaces as PLORA_ERR_CUDA from the
  * call that observes it or from plora_check(); a device-side wait that ran
  * out of time surfaces as PLORA_ERR_TIMEOUT from plora_check().
@@ -87,7 +92,9 @@ typedef enum {
 
 /* plora_config.flags */
 enum {
-    PLORA_FLAG_SIMT = 1u  /* bf16 only: run the plain SIMT kernels instead of the tensor-core ones */
+    PLORA_FLAG_SIMT = 1u,     /* bf16 only: run the plain SIMT kernels instead of the tensor-core ones */
+    PLORA_FLAG_UNFUSED = 2u   /* tensor-core path: run the expand products (Y += s H B, dX += G A^T) as
+                                 separate read-modify-write passes instead of inside the base GEMMs */
 };
 
 /* Limits. */
@@ -141,7 +148,7 @@ PLORA_API plora_status plora_destroy(plora_handle h);
 /*
  * Size in bytes of the `saved` buffer that plora_forward fills and
  * plora_backward reads for this segment map and adapter table.  Its layout
- * is the library's (per-adapter blocks of X_i A_i rows, padded); read it
+ * is the library's (per-adapter zero-padded blocks of s_i X_i A_i rows); read it
  * only through plora_debug_unpack_saved.
  */
 PLORA_API plora_status plora_saved_bytes(plora_handle h, int32_t n_adapters, const int64_t* off,
@@ -183,7 +190,8 @@ PLORA_API const char* plora_status_string(plora_status s);
 PLORA_API const char* plora_last_error(plora_handle h);
 
 /*
- * Debug: copy adapter i's saved H_i = X_i A_i out of `saved` as fp32
+ * Debug: copy adapter i's saved activation H'_i = s_i X_i A_i (the scaled
+ * shrink, which both the expand and dB consume) out of `saved` as fp32
  * [n_i][r_i] into the device buffer H_out (16-byte aligned).
  */
 PLORA_API plora_status plora_debug_unpack_saved(plora_handle h, int32_t n_adapters, const int64_t* off,
@@ -201,8 +209,13 @@ PLORA_API plora_status plora_debug_unpack_saved(plora_handle h, int32_t n_adapte
  *              first H/G row, 64-token blocks, split index, split count,
  *              first partial slot (-1 if unsplit), first counter (-1);
  *   which = 2: adapters, 5 per adapter: first token row, tokens, first H/G
- *              row, rank rounded up to 16, rank rounded up to 64;
- *   which = 3: two values: the padded rank pitch RP and the H/G row count.
+ *              row (each adapter with tokens owns a block of 128 zero rows,
+ *              its rows rounded up to 128, then 128 zero rows), rank rounded
+ *              up to 16, rank rounded up to 64;
+ *   which = 3: two values: the padded rank pitch RP and the H/G row count;
+ *   which = 4: per global 128-row tile, the first index into the list of
+ *              which = 5 (plus the end), i.e. ceil(T/128) + 1 values;
+ *   which = 5: the adapters (with tokens) overlapping each global tile.
  * *count receives the number of int32 values the full answer needs.
  */
 PLORA_API plora_status plora_debug_schedule(const plora_config* cfg, int32_t n_adapters, const int64_t* off,
@@ -248,10 +261,10 @@ PLORA_API plora_status plora_profile_read(plora_handle h, int32_t capacity, int3
  * 16-byte aligned, A and B must still be valid pointers).  Writes every dB_i.
  *
  * Returns PLORA_ERR_UNSUPPORTED if the call's schedule (64 bytes per adapter
- * plus 32 bytes per 4096-token split) exceeds 1 MiB - 256 bytes, or if its
+ * plus 32 bytes per 16384-token split) exceeds 1 MiB - 256 bytes, or if its
  * split partials exceed the rest of the array: (splits of adapters longer
- * than 4096 tokens) x ceil(d_out/128) x (4 + 128 x RP x 4) bytes must fit in
- * PLORA_STATIC_SCRATCH_BYTES - 1 MiB, RP = max rank rounded up to 64.  Other errors as for
+ * than 16384 tokens) x ceil(d_out/128) x (4 + 128 x RP x 4) bytes must fit
+ * in PLORA_STATIC_SCRATCH_BYTES - 1 MiB, RP = max rank rounded up to 64.  Other errors as for
  * plora_backward; a device wait that runs out of time is not reported
  * (there is no handle to report it through).
  *

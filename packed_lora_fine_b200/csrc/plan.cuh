@@ -11,7 +11,7 @@ namespace plora {
 constexpr int kTileM = 128;     // token rows (or hidden rows) per tensor-core tile
 constexpr int kBlockK = 64;     // K elements per pipeline stage (128 bytes of bf16)
 constexpr int kRankAlign = 64;  // the padded rank width RP of the saved/G buffers is a multiple of this
-constexpr int kSplitTokens = 4096;  // weight-gradient split size along the tokens (fixed: deterministic)
+constexpr int kSplitTokens = 16384; // weight-gradient split size along the tokens (fixed: deterministic)
 
 // One adapter, as the kernels see it.
 struct AdapterDev {
@@ -51,6 +51,24 @@ struct RedEntry {
     int32_t counter;   // first arrival counter of the adapter (nsplit > 1), else -1
 };
 static_assert(sizeof(RedEntry) == 32, "RedEntry layout");
+
+// One adapter overlapping one global 128-row tile of a base GEMM (low-rank branch folded in).
+struct LoraSeg {
+    int32_t adapter;
+    int32_t h_y;       // H' / G row holding the tile's first token, inside the adapter's zero-padded block
+    int32_t rp16;      // rank rounded up to 16 (the K extent of the folded product)
+    int32_t pad_;
+};
+static_assert(sizeof(LoraSeg) == 16, "LoraSeg layout");
+
+// Per global 128-row tile of a base GEMM: the range of its LoraSeg entries, with the first two
+// inlined so that one 48-byte load gives everything in the common case.
+struct MTileRec {
+    int32_t q0, q1;    // entries mt_seg[q0 .. q1)
+    int32_t pad_[2];
+    LoraSeg s[2];      // mt_seg[q0], mt_seg[q0 + 1] (when present)
+};
+static_assert(sizeof(MTileRec) == 48, "MTileRec layout");
 
 // A generic strided product for the SIMT path:
 //   C(m, n) = alpha * sum_k A(m, k) B(k, n)  (+ C(m, n) if accumulate)

@@ -102,6 +102,33 @@ bool get_encode() {
     return true;
 }
 
+// [p, p + bytes) must lie inside one device allocation: every tensor pointer is checked against the
+// driver's record of the allocation that contains it, so that no kernel is ever launched on a host
+// pointer, an unallocated address or a buffer that is too small.
+PFN_cuMemGetAddressRange_v3020 g_range = nullptr;
+
+bool get_range_fn() {
+    if (g_range) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return false;
+    g_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+    return true;
+}
+
+bool in_device_allocation(const void* p, size_t bytes) {
+    if (bytes == 0) return true;
+    if (!p || !g_range) return false;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (g_range(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    if (a < base || a - base > size) return false;
+    return bytes <= size - (a - base);
+}
+
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
             kSimt, kKinds };
@@ -157,6 +184,9 @@ struct HostPlan {
     std::vector<TokTile> tok;
     std::vector<RedEntry> red;
     std::vector<int32_t> empty;    // adapters with no tokens
+    std::vector<int32_t> mt_off;   // per global 128-row tile: first entry in mt_seg (+ end)
+    std::vector<MTileRec> mt_rec;  // per global 128-row tile: the range, first two entries inlined
+    std::vector<LoraSeg> mt_seg;   // adapters overlapping each global tile
     int32_t slots = 0, counters = 0;
 };
 
@@ -215,11 +245,13 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
         a.rp16 = (int32_t)round_up(a.rank, 16);
         a.rp64 = (int32_t)round_up(a.rank, 64);
         a.pad_ = 0;
-        hrow += round_up(a.n, kTileM);
         if (a.n == 0) {
             P.empty.push_back(i);
             continue;
         }
+        // H' / G block: 128 zero rows, the adapter's rows rounded up to 128, 128 zero rows.
+        a.h_row = (int32_t)(hrow + kTileM);
+        hrow += round_up(a.n, kTileM) + 2 * kTileM;
         for (int32_t t = 0; t < a.n; t += kTileM)
             P.tok.push_back(TokTile{i, std::min(kTileM, a.n - t), a.x_row + t, a.h_row + t});
         // Weight-gradient splits: a function of this adapter's token count alone, so an
@@ -239,6 +271,26 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
         }
     }
     P.h_rows = hrow;
+    // Adapters overlapping each global 128-row tile (for the base GEMMs with the low-rank branch folded in).
+    const int64_t tiles_m = ceil_div(P.T, kTileM);
+    P.mt_off.assign(tiles_m + 1, 0);
+    int32_t first = 0;
+    for (int64_t mb = 0; mb < tiles_m; ++mb) {
+        const int64_t m0 = mb * kTileM, m1 = std::min<int64_t>(P.T, m0 + kTileM);
+        P.mt_off[mb] = (int32_t)P.mt_seg.size();
+        while (first < n && off[first + 1] <= m0) ++first;
+        for (int32_t j = first; j < n && off[j] < m1; ++j)
+            if (off[j + 1] > off[j])
+                P.mt_seg.push_back(LoraSeg{j, (int32_t)(P.ad[j].h_row + (m0 - off[j])), P.ad[j].rp16, 0});
+    }
+    P.mt_off[tiles_m] = (int32_t)P.mt_seg.size();
+    P.mt_rec.assign(tiles_m, MTileRec{});
+    for (int64_t mb = 0; mb < tiles_m; ++mb) {
+        MTileRec& r = P.mt_rec[mb];
+        r.q0 = P.mt_off[mb];
+        r.q1 = P.mt_off[mb + 1];
+        for (int k = 0; k < 2 && r.q0 + k < r.q1; ++k) r.s[k] = P.mt_seg[r.q0 + k];
+    }
     // Longest-first order of the weight-gradient work (the static persistent schedule
     // then deals items round-robin over the SMs).
     std::stable_sort(P.red.begin(), P.red.end(),
@@ -249,12 +301,51 @@ size_t saved_bytes_of(const plora_ctx* h, const HostPlan& P) {
     return (size_t)P.h_rows * (size_t)P.RP * h->esize;
 }
 
+// Extents of every tensor a call reads or writes (see include/plora.h for the layouts).
+struct TensorArgs {
+    const void* X = nullptr;
+    const void* W = nullptr;
+    const void* Y = nullptr;
+    const void* dY = nullptr;
+    const void* dX = nullptr;
+    const void* saved = nullptr;
+    bool adapters_AB = true;   // check each A_i, B_i
+    bool adapters_dA = false;  // check each dA_i
+    bool adapters_dB = false;  // check each dB_i
+};
+
+plora_status check_extents(plora_ctx* h, const HostPlan& P, const plora_adapter* tab, const TensorArgs& a) {
+    if (!get_range_fn()) return fail(h, PLORA_ERR_CUDA, "cuMemGetAddressRange is not available");
+    const size_t es = h->esize;
+    const size_t T = (size_t)P.T, di = (size_t)h->cfg.d_in, dout = (size_t)h->cfg.d_out;
+    struct Item { const void* p; size_t bytes; const char* name; };
+    const Item items[] = {{a.X, T * di * es, "X"}, {a.W, dout * di * es, "W"}, {a.Y, T * dout * es, "Y"},
+                          {a.dY, T * dout * es, "dY"}, {a.dX, T * di * es, "dX"},
+                          {a.saved, T ? saved_bytes_of(h, P) : 0, "saved"}};
+    for (const Item& it : items)
+        if (it.p && !in_device_allocation(it.p, it.bytes))
+            return fail(h, PLORA_ERR_INVALID_ARG, "%s is not a device buffer of %zu bytes", it.name, it.bytes);
+    for (int32_t i = 0; i < P.n; ++i) {
+        const size_t r = (size_t)tab[i].rank;
+        if (a.adapters_AB && (!in_device_allocation(tab[i].A, r * di * es) ||
+                              !in_device_allocation(tab[i].B, dout * r * es)))
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: A or B is not a device buffer of its size", i);
+        if (a.adapters_dA && !in_device_allocation(tab[i].dA, r * di * sizeof(float)))
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: dA is not a device buffer of its size", i);
+        if (a.adapters_dB && !in_device_allocation(tab[i].dB, dout * r * sizeof(float)))
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: dB is not a device buffer of its size", i);
+    }
+    return PLORA_OK;
+}
+
 // Copy the plan blob to the device through the staging ring. Returns device pointers.
 struct DevPlan {
     AdapterDev* ad = nullptr;
     TokTile* tok = nullptr;
     RedEntry* red = nullptr;
     SimtOp* ops = nullptr;
+    MTileRec* mt_rec = nullptr;
+    LoraSeg* mt_seg = nullptr;
     int slot = 0;
 };
 
@@ -275,6 +366,8 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     const size_t o_tok = put(P.tok.data(), P.tok.size() * sizeof(TokTile));
     const size_t o_red = put(P.red.data(), P.red.size() * sizeof(RedEntry));
     const size_t o_ops = put(ops.data(), ops.size() * sizeof(SimtOp));
+    const size_t o_mto = put(P.mt_rec.data(), P.mt_rec.size() * sizeof(MTileRec));
+    const size_t o_mtl = put(P.mt_seg.data(), P.mt_seg.size() * sizeof(LoraSeg));
     if (o > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "schedule exceeds the handle's staging size");
     uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
     e = cudaMemcpyAsync(d, h->h_blob[slot], o, cudaMemcpyHostToDevice, st);
@@ -283,6 +376,8 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     D.tok = reinterpret_cast<TokTile*>(d + o_tok);
     D.red = reinterpret_cast<RedEntry*>(d + o_red);
     D.ops = reinterpret_cast<SimtOp*>(d + o_ops);
+    D.mt_rec = reinterpret_cast<MTileRec*>(d + o_mto);
+    D.mt_seg = reinterpret_cast<LoraSeg*>(d + o_mtl);
     D.slot = slot;
     return PLORA_OK;
 }
@@ -325,13 +420,20 @@ void launch_simt(plora_ctx* h, const SimtOp* d_ops, int n_ops, int tiles, cudaSt
 // Tensor-core launches
 // ---------------------------------------------------------------------------
 template <Op OP>
-void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, cudaStream_t st) {
+void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const CUtensorMap& b2,
+               const TcParams& p, cudaStream_t st) {
     if (p.num_tiles <= 0) return;
     const int grid = std::min(p.num_tiles, h->num_sms);
     constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : OP == Op::BaseDx ? kBaseDx : OP == Op::ShrinkX ? kShrinkX
                        : OP == Op::ShrinkDy ? kShrinkDy : OP == Op::ExpandY ? kExpandY : OP == Op::ExpandDx ? kExpandDx
                        : OP == Op::WgradB ? kWgradB : kWgradA;
-    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, p); });
+    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p); });
+}
+
+// A deeper operand ring for ops whose B tile is narrower than 256 rows: A tile + RP rows of B.
+void narrow_ring(TcParams& p, int RP) {
+    p.stage_bytes = kABytes + RP * kBlockK * 2;
+    p.stages = std::min(kMaxStages, kRingBytes / p.stage_bytes);
 }
 
 template <Op OP>
@@ -350,6 +452,11 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     p.partials = h->at<float>(h->r_part);
     p.counters = h->at<int32_t>(h->r_cnt);
     p.group_m = 16;
+    p.mt_rec = D.mt_rec;
+    p.mt_seg = D.mt_seg;
+    p.fuse = 0;
+    p.stages = kStages;
+    p.stage_bytes = kStageBytes;
     return p;
 }
 
@@ -360,8 +467,11 @@ plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, cud
     const int64_t vecs = (int64_t)P.n * P.RP * (h->cfg.d_in / 8);
     const int grid_a = (int)std::min<int64_t>(ceil_div(vecs, 256), (int64_t)h->num_sms * 8);
     tracked(h, kPackA, st, [&] { pack_a_kernel<<<grid_a, 256, 0, st>>>(D.ad, P.n, P.RP, h->cfg.d_in, pa); });
-    dim3 gb((unsigned)ceil_div(h->cfg.d_out, 64), (unsigned)P.n);
-    tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, 0, st>>>(D.ad, P.RP, h->cfg.d_out, pb); });
+    dim3 gb((unsigned)ceil_div(h->cfg.d_out, 128), (unsigned)P.n);
+    int maxr = 1;
+    for (const AdapterDev& a : P.ad) maxr = std::max(maxr, a.rank);
+    const size_t smem_bt = (size_t)128 * (maxr + 2) * sizeof(__nv_bfloat16);
+    tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, smem_bt, st>>>(D.ad, P.RP, h->cfg.d_out, pb); });
     return PLORA_OK;
 }
 
@@ -398,7 +508,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     if (cfg->max_adapters < 1 || cfg->max_adapters > PLORA_MAX_ADAPTERS) return PLORA_ERR_INVALID_ARG;
     if (cfg->max_rank < 1 || cfg->max_rank > PLORA_MAX_RANK) return PLORA_ERR_INVALID_ARG;
     if (cfg->max_tokens < 1 || cfg->max_tokens > ((int64_t)1 << 30)) return PLORA_ERR_INVALID_ARG;
-    if (cfg->flags & ~(uint32_t)PLORA_FLAG_SIMT) return PLORA_ERR_INVALID_ARG;
+    if (cfg->flags & ~(uint32_t)(PLORA_FLAG_SIMT | PLORA_FLAG_UNFUSED)) return PLORA_ERR_INVALID_ARG;
 
     plora_ctx* h = new (std::nothrow) plora_ctx();
     if (!h) return PLORA_ERR_OOM;
@@ -417,7 +527,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     // Workspace sizing (all bounds follow from the config).
     const int64_t na = cfg->max_adapters;
     h->RPmax = (int)round_up(cfg->max_rank, kRankAlign);
-    h->max_h_rows = cfg->max_tokens + (int64_t)(kTileM - 1) * na;
+    h->max_h_rows = cfg->max_tokens + (int64_t)(3 * kTileM - 1) * na;
     const int64_t dtiles = std::max(ceil_div(cfg->d_in, kTileM), ceil_div(cfg->d_out, kTileM));
     h->max_slots = 2 * (cfg->max_tokens / kSplitTokens) + 1;
     h->max_counters = (cfg->max_tokens / (kSplitTokens + 1) + 1) * dtiles;
@@ -427,7 +537,9 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     h->blob_bytes = (size_t)round_up(na * (int64_t)sizeof(AdapterDev), 256) +
                     (size_t)round_up(tok_max * (int64_t)sizeof(TokTile), 256) +
                     (size_t)round_up(red_max * (int64_t)sizeof(RedEntry), 256) +
-                    (size_t)round_up(ops_max * (int64_t)sizeof(SimtOp), 256) + 1024;
+                    (size_t)round_up(ops_max * (int64_t)sizeof(SimtOp), 256) +
+                    (size_t)round_up((tok_max + 1) * (int64_t)sizeof(MTileRec), 256) +
+                    (size_t)round_up((tok_max + na) * (int64_t)sizeof(LoraSeg), 256) + 1024;
 
     size_t o = 0;
     auto carve = [&](Region& r, size_t bytes) {
@@ -461,6 +573,9 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
         if (e == cudaSuccess) e = set_tc_attr<Op::ExpandDx>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradB>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradA>();
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(pack_bt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     128 * (PLORA_MAX_RANK + 2) * (int)sizeof(__nv_bfloat16));
     }
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -522,6 +637,12 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     HostPlan P;
     build_plan(h, n, off, tab, P);
     if (P.T == 0) return PLORA_OK;
+    {
+        TensorArgs ta;
+        ta.X = X; ta.W = W; ta.Y = Y; ta.saved = saved;
+        s = check_extents(h, P, tab, ta);
+        if (s != PLORA_OK) return s;
+    }
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
 
     if (!h->tc) {
@@ -529,19 +650,19 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
         int32_t t1 = 0, t2 = 0;
         const bool f32 = h->cfg.dtype == PLORA_FP32;
         const size_t es = h->esize;
-        // K1: Y = X W.  K2: H_i = X_i A_i.
+        // K1: Y = X W.  K2: H'_i = s_i X_i A_i.
         add_op(ops, t1, X, d_in, 1, W, 1, d_in, Y, d_out, 1, P.T, d_out, d_in, 1.f, false, f32);
         for (const AdapterDev& a : P.ad) {
             if (a.n == 0) continue;
             add_op(ops, t1, (const uint8_t*)X + (size_t)a.x_row * d_in * es, d_in, 1, a.A, 1, d_in,
-                   (uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.n, a.rank, d_in, 1.f, false, f32);
+                   (uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.n, a.rank, d_in, a.scale, false, f32);
         }
         const int n1 = (int)ops.size();
-        // K3: Y_i += s_i H_i B_i.
+        // K3: Y_i += H'_i B_i.
         for (const AdapterDev& a : P.ad) {
             if (a.n == 0) continue;
             add_op(ops, t2, (const uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.B, 1, a.rank,
-                   (uint8_t*)Y + (size_t)a.x_row * d_out * es, d_out, 1, a.n, d_out, a.rank, a.scale, true, f32);
+                   (uint8_t*)Y + (size_t)a.x_row * d_out * es, d_out, 1, a.n, d_out, a.rank, 1.f, true, f32);
         }
         DevPlan D;
         s = upload(h, P, ops, st, D);
@@ -561,36 +682,43 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
     pack_factors(h, P, D, st);
-    CUtensorMap mX, mW, mPA, mH, mPB;
+    CUtensorMap mX, mW, mPA, mHk, mPB, mPB16;
     bool ok = make_map(&mX, X, d_in, P.T, d_in, 64, kTileM) &&
               make_map(&mW, W, d_in, d_out, d_in, 64, kTileN) &&
               make_map(&mPA, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, P.RP) &&
-              make_map(&mH, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
-              make_map(&mPB, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 64);
+              make_map(&mHk, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_map(&mPB, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 64) &&
+              make_map(&mPB16, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 16);
     if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
-    TcParams p = base_params(h, P, D);
-    // K1: Y = X W over all packed tokens.
-    p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_out; p.K_total = (int32_t)d_in;
-    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_out, kTileN);
-    p.num_tiles = p.tiles_m * p.tiles_n;
-    p.b_box_rows = kTileN;
-    p.out = Y; p.out_ld = d_out;
-    launch_tc<Op::BaseFwd>(h, mX, mW, p, st);
-    // K2: H_i = X_i A_i per 128-token tile.
+    const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
+    // K2: H'_i = s_i X_i A_i per 128-token tile (into the zero-padded blocks of `saved`).
     TcParams q = base_params(h, P, D);
     q.K_total = (int32_t)d_in;
     q.num_tiles = (int32_t)P.tok.size();
     q.b_box_rows = P.RP;
     q.out = saved; q.out_ld = P.RP;
-    launch_tc<Op::ShrinkX>(h, mX, mPA, q, st);
-    // K3: Y_i += s_i H_i B_i.
-    TcParams r = base_params(h, P, D);
-    r.N_total = (int32_t)d_out;
-    r.tiles_n = (int32_t)ceil_div(d_out, kTileN);
-    r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
-    r.out = Y; r.out_ld = d_out;
-    launch_tc<Op::ExpandY>(h, mH, mPB, r, st);
+    narrow_ring(q, P.RP);
+    launch_tc<Op::ShrinkX>(h, mX, mPA, mX, mPA, q, st);
+    // K1 (+K3): Y = X W over all packed tokens; fused, each tile also accumulates H'_j B_j of
+    // every adapter j overlapping it, so Y is written once.
+    TcParams p = base_params(h, P, D);
+    p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_out; p.K_total = (int32_t)d_in;
+    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_out, kTileN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.b_box_rows = kTileN;
+    p.out = Y; p.out_ld = d_out;
+    p.fuse = fused ? 1 : 0;
+    launch_tc<Op::BaseFwd>(h, mX, mW, mHk, mPB16, p, st);
+    if (!fused) {
+        // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
+        TcParams r = base_params(h, P, D);
+        r.N_total = (int32_t)d_out;
+        r.tiles_n = (int32_t)ceil_div(d_out, kTileN);
+        r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
+        r.out = Y; r.out_ld = d_out;
+        launch_tc<Op::ExpandY>(h, mHk, mPB, mHk, mPB, r, st);
+    }
     return finish(h, D, st);
 }
 
@@ -612,6 +740,14 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     HostPlan P;
     build_plan(h, n, off, tab, P);
+    {
+        TensorArgs ta;
+        if (P.T > 0) { ta.X = X; ta.W = W; ta.dY = dY; ta.dX = dX; ta.saved = saved; }
+        ta.adapters_AB = P.T > 0;
+        ta.adapters_dA = ta.adapters_dB = true;
+        s = check_extents(h, P, tab, ta);
+        if (s != PLORA_OK) return s;
+    }
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
     // Adapters without tokens: their weight gradients are zero.
     for (int32_t i : P.empty) {
@@ -627,7 +763,7 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
         int32_t t1 = 0, t2 = 0;
         const bool f32 = h->cfg.dtype == PLORA_FP32;
         const size_t es = h->esize;
-        // Phase 1 -- K4: dX = dY W^T; K5: G_i = s_i dY_i B_i^T; K7: dB_i = s_i dY_i^T H_i.
+        // Phase 1 -- K4: dX = dY W^T; K5: G_i = s_i dY_i B_i^T; K7: dB_i = dY_i^T H'_i.
         if (dX) add_op(ops, t1, dY, d_out, 1, W, d_in, 1, dX, d_in, 1, P.T, d_in, d_out, 1.f, false, f32);
         for (const AdapterDev& a : P.ad) {
             if (a.n == 0) continue;
@@ -635,7 +771,7 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
                    (uint8_t*)G + (size_t)a.h_row * P.RP * es, P.RP, 1, a.n, a.rank, d_out, a.scale, false, f32);
             add_op(ops, t1, (const uint8_t*)dY + (size_t)a.x_row * d_out * es, 1, d_out,
                    (const uint8_t*)saved + (size_t)a.h_row * P.RP * es, P.RP, 1, a.dB, a.rank, 1, d_out, a.rank,
-                   a.n, a.scale, false, true);
+                   a.n, 1.f, false, true);
         }
         const int n1 = (int)ops.size();
         // Phase 2 -- K6: dX_i += G_i A_i^T; K8: dA_i = X_i^T G_i.
@@ -665,7 +801,7 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
     pack_factors(h, P, D, st);
-    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_k, mG_k, mG_mn, mPA_mn, mH_mn, mX_mn;
+    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_k, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn;
     bool ok = make_map(&mdY_k, dY, d_out, P.T, d_out, 64, kTileM) &&
               make_map(&mdY_mn, dY, d_out, P.T, d_out, 64, 64) &&
               make_map(&mW_mn, W, d_in, d_out, d_in, 64, 64) &&
@@ -673,46 +809,53 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
               make_map(&mG_k, G, P.RP, P.h_rows, P.RP, 64, kTileM) &&
               make_map(&mG_mn, G, P.RP, P.h_rows, P.RP, 64, 64) &&
               make_map(&mPA_mn, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
+              make_map(&mPA16, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
               make_map(&mH_mn, saved, P.RP, P.h_rows, P.RP, 64, 64) &&
               make_map(&mX_mn, X, d_in, P.T, d_in, 64, 64);
     if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
-    if (dX) {
-        // K4: dX = dY W^T.
-        TcParams p = base_params(h, P, D);
-        p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
-        p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
-        p.num_tiles = p.tiles_m * p.tiles_n;
-        p.out = dX; p.out_ld = d_in;
-        launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, p, st);
-    }
-    // K5: G_i = s_i dY_i B_i^T.
+    const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
+    // K5: G_i = s_i dY_i B_i^T per 128-token tile (into the zero-padded workspace blocks).
     TcParams q = base_params(h, P, D);
     q.K_total = (int32_t)d_out;
     q.num_tiles = (int32_t)P.tok.size();
     q.b_box_rows = P.RP;
     q.out = G; q.out_ld = P.RP;
-    launch_tc<Op::ShrinkDy>(h, mdY_k, mPB_k, q, st);
+    narrow_ring(q, P.RP);
+    launch_tc<Op::ShrinkDy>(h, mdY_k, mPB_k, mdY_k, mPB_k, q, st);
     if (dX) {
-        // K6: dX_i += G_i A_i^T.
-        TcParams r = base_params(h, P, D);
-        r.N_total = (int32_t)d_in;
-        r.tiles_n = (int32_t)ceil_div(d_in, kTileN);
-        r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
-        r.out = dX; r.out_ld = d_in;
-        launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, r, st);
+        // K4 (+K6): dX = dY W^T; fused, each tile also accumulates G_j A_j^T of every adapter j
+        // overlapping it, so dX is written once.
+        TcParams p = base_params(h, P, D);
+        p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
+        p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
+        p.num_tiles = p.tiles_m * p.tiles_n;
+        p.out = dX; p.out_ld = d_in;
+        p.fuse = fused ? 1 : 0;
+        launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, p, st);
+        if (!fused) {
+            // K6 as its own pass: dX_i += G_i A_i^T (read-modify-write of dX).
+            TcParams r = base_params(h, P, D);
+            r.N_total = (int32_t)d_in;
+            r.tiles_n = (int32_t)ceil_div(d_in, kTileN);
+            r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
+            r.out = dX; r.out_ld = d_in;
+            launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, mG_k, mPA_mn, r, st);
+        }
     }
-    // K7: dB_i = s_i dY_i^T H_i; K8: dA_i = X_i^T G_i (sums over each adapter's tokens).
+    // K7: dB_i = H'_i^T dY_i; K8: dA_i = X_i^T G_i (sums over each adapter's tokens).
     TcParams wb = base_params(h, P, D);
     wb.M_total = (int32_t)d_out;
     wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
     wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
-    launch_tc<Op::WgradB>(h, mdY_mn, mH_mn, wb, st);
+    narrow_ring(wb, P.RP);
+    launch_tc<Op::WgradB>(h, mdY_mn, mH_mn, mdY_mn, mH_mn, wb, st);
     TcParams wa = base_params(h, P, D);
     wa.M_total = (int32_t)d_in;
     wa.red_dtiles = (int32_t)ceil_div(d_in, kTileM);
     wa.num_tiles = (int32_t)P.red.size() * wa.red_dtiles;
-    launch_tc<Op::WgradA>(h, mX_mn, mG_mn, wa, st);
+    narrow_ring(wa, P.RP);
+    launch_tc<Op::WgradA>(h, mX_mn, mG_mn, mX_mn, mG_mn, wa, st);
     return finish(h, D, st);
 }
 
@@ -743,6 +886,16 @@ plora_status plora_debug_unpack_saved(plora_handle h, int32_t n, const int64_t* 
     build_plan(h, n, off, tab, P);
     const AdapterDev& a = P.ad[i];
     if (a.n == 0) return PLORA_OK;
+    {
+        TensorArgs ta;
+        ta.saved = saved;
+        ta.adapters_AB = false;
+        s = check_extents(h, P, tab, ta);
+        if (s == PLORA_OK && !in_device_allocation(H_out, (size_t)a.n * a.rank * sizeof(float)))
+            s = fail(h, PLORA_ERR_INVALID_ARG, "H_out is not a device buffer of %zu bytes",
+                     (size_t)a.n * a.rank * sizeof(float));
+        if (s != PLORA_OK) return s;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int grid = (int)std::min<int64_t>(ceil_div((int64_t)a.n * a.rank, 256), 1024);
     if (h->cfg.dtype == PLORA_FP32)
@@ -806,6 +959,10 @@ plora_status plora_debug_schedule(const plora_config* cfg, int32_t n, const int6
         for (const AdapterDev& a : P.ad) v.insert(v.end(), {a.x_row, a.n, a.h_row, a.rp16, a.rp64});
     } else if (which == 3) {
         v = {P.RP, (int32_t)P.h_rows};
+    } else if (which == 4) {
+        v = P.mt_off;
+    } else if (which == 5) {
+        for (const LoraSeg& g : P.mt_seg) v.push_back(g.adapter);
     } else {
         return PLORA_ERR_INVALID_ARG;
     }
@@ -913,6 +1070,14 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     StaticDevice sd;
     s = static_setup(dev, sd);
     if (s != PLORA_OK) return s;
+    {
+        TensorArgs ta;
+        if (P.T > 0) { ta.dY = dY; ta.saved = saved; }
+        ta.adapters_AB = false;
+        ta.adapters_dB = true;
+        s = check_extents(&tmp, P, tab, ta);
+        if (s != PLORA_OK) return s;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     // Adapters without tokens get dB = 0.
@@ -948,7 +1113,8 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     p.M_total = (int32_t)d_out;
     p.red_dtiles = dtiles;
     p.num_tiles = (int32_t)P.red.size() * dtiles;
+    narrow_ring(p, P.RP);
     if (p.num_tiles > 0)
-        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, p);
+        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, mdY, mH, p);
     return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
 }

@@ -47,14 +47,16 @@ template <Op OP> struct OpTraits {
     static constexpr bool kWgrad = (OP == Op::WgradB || OP == Op::WgradA);
 };
 
-constexpr int kStages = 4;
+constexpr int kStages = 4;                        // stages of the largest (48 KB) layout
+constexpr int kMaxStages = 8;                     // ring slots when the op's stages are smaller
 constexpr int kTileN = 256;                       // N of the base / expand tiles (TMEM columns)
 constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB: 128 rows x 64 bf16
 constexpr int kBBytesMax = kTileN * kBlockK * 2;  // 32 KB: 256 rows x 64 bf16
 constexpr int kStageBytes = kABytes + kBBytesMax;
 constexpr int kTmemCols = 512;                    // two 256-column fp32 accumulators
 constexpr int kTcThreads = 192;
-constexpr int kTcSmemBytes = kStages * kStageBytes + 1024 /* align */ + 256 /* barriers */;
+constexpr int kRingBytes = kStages * kStageBytes; // 192 KB of operand ring
+constexpr int kTcSmemBytes = kRingBytes + 1024 /* align */ + 256 /* barriers */;
 
 struct TcParams {
     int32_t M_total;        // Base: T; Wgrad: d (rows of dB_i or columns of dA_i)
@@ -74,12 +76,20 @@ struct TcParams {
     int32_t* counters;      // Wgrad split arrival counters
     int* err_flag;
     uint64_t timeout_ns;
+    // Base ops with the low-rank branch folded in (fuse != 0): for global m-tile mb, the
+    // adapters overlapping its 128 rows are mt_seg[mt_rec[mb].q0 .. mt_rec[mb].q1).
+    const MTileRec* mt_rec;
+    const LoraSeg* mt_seg;
+    int32_t fuse;
+    int32_t stages;         // operand ring depth (<= kMaxStages)
+    int32_t stage_bytes;    // bytes per ring stage: A tile + this op's largest B tile
 };
 
 struct TileInfo {
     int32_t a_x, a_y, b_x, b_y;
     int32_t kblocks, last_ksteps, mma_n, nb_boxes;
     int32_t adapter, out_row, rows_valid, n0, cols_valid, red_idx;
+    int32_t mtile;
     float scale;
 };
 
@@ -101,6 +111,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         const int r = t - g * per_group;
         const int mb = first_m + r % gm;
         const int nb = r / gm;
+        ti.mtile = mb;
         ti.a_x = 0;
         ti.a_y = mb * kTileM;
         if constexpr (OP == Op::BaseFwd) { ti.b_x = 0; ti.b_y = nb * kTileN; }
@@ -125,7 +136,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         ti.rows_valid = tt.rows;
         ti.n0 = 0;
         ti.cols_valid = p.RP;
-        ti.scale = (OP == Op::ShrinkDy) ? ad.scale : 1.f;
+        ti.scale = ad.scale;   // H' = s X A and G = s dY B^T carry the adapter's scale
     } else if constexpr (Tr::kExpand) {
         const int mt = t / p.tiles_n;
         const int nb = t - mt * p.tiles_n;
@@ -145,7 +156,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         ti.rows_valid = tt.rows;
         ti.n0 = nb * kTileN;
         ti.cols_valid = min(kTileN, p.N_total - ti.n0);
-        ti.scale = (OP == Op::ExpandY) ? ad.scale : 1.f;
+        ti.scale = 1.f;        // H' and G already carry the scale
     } else {
         const int e = t / p.red_dtiles;
         const int db = t - e * p.red_dtiles;
@@ -164,9 +175,24 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         ti.rows_valid = min(kTileM, p.M_total - ti.out_row);
         ti.n0 = db;  // the d-tile index (for partial slots)
         ti.cols_valid = ad.rank;
-        ti.scale = (OP == Op::WgradB) ? ad.scale : 1.f;
+        ti.scale = 1.f;        // H' and G already carry the scale
     }
     return ti;
+}
+
+// The folded low-rank record of base tile t (empty when not folding or past the end).
+template <Op OP>
+__device__ __forceinline__ MTileRec load_mtile(const TcParams& p, int t) {
+    MTileRec r;
+    r.q0 = r.q1 = 0;
+    if (OpTraits<OP>::kBase && p.fuse && t < p.num_tiles) {
+        const TileInfo ti = decode_tile<OP>(p, t);
+        r = p.mt_rec[ti.mtile];
+    }
+    return r;
+}
+__device__ __forceinline__ LoraSeg mtile_seg(const TcParams& p, const MTileRec& r, int q) {
+    return q - r.q0 < 2 ? r.s[q - r.q0] : p.mt_seg[q];
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -181,17 +207,19 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
 template <Op OP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const TcParams p) {
+          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
     using Tr = OpTraits<OP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-    uint64_t* full_bar = bars;                    // [kStages]
-    uint64_t* empty_bar = bars + kStages;         // [kStages]
-    uint64_t* accf_bar = bars + 2 * kStages;      // [2]
-    uint64_t* acce_bar = bars + 2 * kStages + 2;  // [2]
-    uint64_t* drain_bar = bars + 2 * kStages + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+    uint64_t* full_bar = bars;                       // [kMaxStages]
+    uint64_t* empty_bar = bars + kMaxStages;         // [kMaxStages]
+    uint64_t* accf_bar = bars + 2 * kMaxStages;      // [2]
+    uint64_t* acce_bar = bars + 2 * kMaxStages + 2;  // [2]
+    uint64_t* drain_bar = bars + 2 * kMaxStages + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 5);
+    const int nst = p.stages;                        // ring depth of this launch
+    const int stb = p.stage_bytes;                   // bytes per stage (multiple of 1024)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* red_flag = reinterpret_cast<int*>(tmem_slot + 2);
 
@@ -199,7 +227,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < nst; ++s) {
             ptx::mbar_init(&full_bar[s], 1);
             ptx::mbar_init(&empty_bar[s], 1);
         }
@@ -214,6 +242,10 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     if (warp == 0 && lane == 0) {
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
+        if (Tr::kBase && p.fuse) {
+            ptx::tma_prefetch_desc(&tmA2);
+            ptx::tma_prefetch_desc(&tmB2);
+        }
     }
     if (warp == 1) {
         ptx::tmem_alloc<kTmemCols>(tmem_slot);
@@ -232,13 +264,17 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             uint32_t phase = 0;
             uint32_t armed = 0, armed_par = 0;
             bool ok = true;
+            MTileRec lr_next = load_mtile<OP>(p, blockIdx.x);
             for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
                 const TileInfo ti = decode_tile<OP>(p, t);
                 const uint32_t b_bytes = Tr::kBmn ? (uint32_t)ti.nb_boxes * 8192u
                                                   : (uint32_t)p.b_box_rows * 128u;
+                // Folded low-rank branch: this tile's record was fetched one tile ahead.
+                const MTileRec lr = lr_next;
+                lr_next = load_mtile<OP>(p, t + gridDim.x);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
-                    uint8_t* sA = smem + stage * kStageBytes;
+                    uint8_t* sA = smem + stage * stb;
                     uint8_t* sB = sA + kABytes;
                     ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + b_bytes);
                     armed |= 1u << stage;
@@ -256,11 +292,36 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     } else {
                         ptx::tma_load_2d(sB, &tmB, &full_bar[stage], ti.b_x + kb * kBlockK, ti.b_y);
                     }
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++stage == nst) { stage = 0; phase ^= 1u; }
+                }
+                if constexpr (Tr::kBase) {
+                    // Low-rank branch folded into the same accumulator: for every adapter j whose
+                    // tokens overlap this m-tile, K-steps over its rank with A = its H' (or G) rows,
+                    // read at the tile's row offset inside j's zero-padded block (rows outside j's
+                    // segment load as zeros), and B = its packed factor (MN-major, 16-row boxes so
+                    // that only the rank's rows are staged).
+                    for (int q = lr.q0; q < lr.q1 && ok; ++q) {
+                        const LoraSeg sg = mtile_seg(p, lr, q);
+                        for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
+                            const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
+                            if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
+                            uint8_t* sA = smem + stage * stb;
+                            uint8_t* sB = sA + kABytes;
+                            ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + 4u * (uint32_t)R * 128u);
+                            armed |= 1u << stage;
+                            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                            ptx::tma_load_2d(sA, &tmA2, &full_bar[stage], kb * kBlockK, sg.h_y);
+                            for (int h = 0; h < 4; ++h)
+                                for (int r16 = 0; r16 < R; r16 += 16)
+                                    ptx::tma_load_2d(sB + h * R * 128 + r16 * 128, &tmB2, &full_bar[stage],
+                                                     ti.n0 + 64 * h, sg.adapter * p.RP + kb * kBlockK + r16);
+                            if (++stage == nst) { stage = 0; phase ^= 1u; }
+                        }
+                    }
                 }
             }
             // Drain: every load this thread issued must have landed before the CTA exits.
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < nst; ++s)
                 if (armed & (1u << s)) {
                     int dummy = 0;
                     ptx::mbar_wait(&full_bar[s], (armed_par >> s) & 1u, &dummy, lim, p.err_flag);
@@ -274,16 +335,19 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             int abuf = 0;
             uint32_t aphase = 0;
             bool ok = true;
+            MTileRec lr_next = load_mtile<OP>(p, blockIdx.x);
             for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
                 const TileInfo ti = decode_tile<OP>(p, t);
                 const uint32_t idesc = ptx::idesc_bf16_f32(kTileM, ti.mma_n, Tr::kAmn, Tr::kBmn);
+                const MTileRec lr = lr_next;
+                lr_next = load_mtile<OP>(p, t + gridDim.x);
                 if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, lim, p.err_flag)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    const uint32_t sA = ptx::smem_u32(smem + stage * kStageBytes);
+                    const uint32_t sA = ptx::smem_u32(smem + stage * stb);
                     const uint32_t sB = sA + kABytes;
                     const int steps = (kb == ti.kblocks - 1) ? ti.last_ksteps : 4;
                     for (int ks = 0; ks < steps; ++ks) {
@@ -294,7 +358,27 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                         ptx::tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | ks) ? 1u : 0u);
                     }
                     ptx::tc_commit(&empty_bar[stage]);
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++stage == nst) { stage = 0; phase ^= 1u; }
+                }
+                if constexpr (Tr::kBase) {
+                    const uint32_t idesc_lr = ptx::idesc_bf16_f32(kTileM, kTileN, false, true);
+                    for (int q = lr.q0; q < (ok ? lr.q1 : lr.q0); ++q) {
+                        const LoraSeg sg = mtile_seg(p, lr, q);
+                        for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
+                            const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
+                            if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, lim, p.err_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            const uint32_t sA = ptx::smem_u32(smem + stage * stb);
+                            const uint32_t sB = sA + kABytes;
+                            for (int ks = 0; ks < R / 16; ++ks)
+                                ptx::tc_mma_f16(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024),
+                                                ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024),
+                                                idesc_lr, 1u);
+                            ptx::tc_commit(&empty_bar[stage]);
+                            if (++stage == nst) { stage = 0; phase ^= 1u; }
+                        }
+                        if (!ok) break;
+                    }
                 }
                 if (!ok) break;
                 ptx::tc_commit(&accf_bar[abuf]);
@@ -361,6 +445,25 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     *reinterpret_cast<uint4*>(out + c) = v0;
                     *reinterpret_cast<uint4*>(out + c + 8) = v1;
                 }
+                // The adapter's block has 128 zero rows before and after its (128-rounded) rows, so that a
+                // base tile straddling the segment can read it at any row offset; the first and the last
+                // tile of the adapter write them.
+                const AdapterDev ad = p.adapters[ti.adapter];
+                const bool first = ti.out_row == ad.h_row;
+                const bool last = ti.out_row + kTileM >= ad.h_row + ad.n;
+                if (first || last) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.out);
+                    if (first) {
+                        uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(ad.h_row - kTileM + row) * p.out_ld);
+                        for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                    }
+                    if (last) {
+                        const int tail = ad.h_row + ((ad.n + kTileM - 1) / kTileM) * kTileM;
+                        uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(tail + row) * p.out_ld);
+                        for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                    }
+                }
             } else if constexpr (Tr::kExpand) {
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
                 const float s = ti.scale;
@@ -422,17 +525,16 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     // Split along the tokens: write this split's partial, the last split of the
                     // tile to arrive sums all partials in split order (deterministic) and stores.
                     const int64_t slot_elems = (int64_t)kTileM * p.RP;
-                    float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems
-                                  + (int64_t)row * p.RP;
+                    // partial layout [slot][d-tile][rank column][128 rows]: a warp's lanes touch
+                    // consecutive rows, so both the writes here and the reduction below coalesce.
+                    float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems + row;
                     for (int c = 0; c < ti.mma_n; c += 16) {
                         uint32_t r[16];
                         ptx::tmem_ld16(t_row + c, r);
                         ptx::tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            *reinterpret_cast<float4*>(mine + c + e) =
-                                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+                        for (int e = 0; e < 16; ++e)
+                            if (c + e < rank) mine[(int64_t)(c + e) * kTileM] = __uint_as_float(r[e]);
                     }
                     __threadfence();
                     ptx::named_bar_sync(1, 128);
@@ -444,14 +546,30 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     if (*red_flag) {
                         __threadfence();
                         if (row_ok) {
-                            for (int k = 0; k < rank; ++k) {
-                                float acc = 0.f;
-                                for (int sp = 0; sp < re.nsplit; ++sp)
-                                    acc += __ldcg(p.partials + ((int64_t)(re.slot + sp) * p.red_dtiles + ti.n0) * slot_elems
-                                                  + (int64_t)row * p.RP + k);
-                                const float v = s * acc;
-                                if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = v;
-                                else ad.dA[(int64_t)k * p.M_total + hid] = v;
+                            const float* first = p.partials + ((int64_t)re.slot * p.red_dtiles + ti.n0) * slot_elems + row;
+                            const int64_t split_stride = (int64_t)p.red_dtiles * slot_elems;
+                            for (int k0 = 0; k0 < rank; k0 += 8) {
+                                // 8 ranks at a time: all of a split's loads are in flight together,
+                                // the sum still runs over the splits in order.
+                                float acc[8];
+#pragma unroll
+                                for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+                                for (int sp = 0; sp < re.nsplit; ++sp) {
+                                    float v[8];
+#pragma unroll
+                                    for (int u = 0; u < 8; ++u)
+                                        v[u] = (k0 + u < rank) ? __ldcg(first + sp * split_stride + (int64_t)(k0 + u) * kTileM) : 0.f;
+#pragma unroll
+                                    for (int u = 0; u < 8; ++u) acc[u] += v[u];
+                                }
+#pragma unroll
+                                for (int u = 0; u < 8; ++u) {
+                                    const int k = k0 + u;
+                                    if (k < rank) {
+                                        if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = s * acc[u];
+                                        else ad.dA[(int64_t)k * p.M_total + hid] = s * acc[u];
+                                    }
+                                }
                             }
                         }
                         if (threadIdx.x == 64) p.counters[re.counter + ti.n0] = 0;
@@ -474,8 +592,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
 // ---------------------------------------------------------------------------
 // Packing of the small per-adapter factors into the MMA-ready padded layouts.
-//   packA [n*RP][d_in]:  row i*RP + k = A_i[k][:]       (k < r_i), zero for r_i <= k < RP
-//   packBT[n*RP][d_out]: row i*RP + k = B_i[:][k]       (k < r_i), zero for r_i <= k < RP
+//   packA [n*RP][d_in]:  row i*RP + k = A_i[k][:]       (k < r_i), zero for r_i <= k < rp16_i
+//   packBT[n*RP][d_out]: row i*RP + k = B_i[:][k]       (k < r_i), zero for r_i <= k < rp16_i
+// Rows rp16_i <= k < RP are never read by an MMA and are left unwritten.
 // ---------------------------------------------------------------------------
 __global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, int64_t d_in,
                               __nv_bfloat16* __restrict__ packA) {
@@ -486,6 +605,7 @@ __global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, 
         const int64_t v = e - rowi * vec_per_row;
         const int i = (int)(rowi / RP);
         const int k = (int)(rowi - (int64_t)i * RP);
+        if (k >= ad[i].rp16) continue;   // rows past the MMA extent are never read
         uint4 val = make_uint4(0, 0, 0, 0);
         if (k < ad[i].rank)
             val = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ad[i].A) + (int64_t)k * d_in)[v];
@@ -493,25 +613,43 @@ __global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, 
     }
 }
 
-// grid: (ceil(d_out/64), n); block 256.  Stages B_i[c0..c0+63][0..r) in shared memory.
+// grid: (ceil(d_out/128), n); block 256.  Stages B_i[c0..c0+127][0..r) in shared memory (dynamic,
+// 128 x (r + 2) bf16), then writes rows k < rp16 of packBT, 128 columns each.
 __global__ void __launch_bounds__(256) pack_bt_kernel(const AdapterDev* __restrict__ ad, int RP, int64_t d_out,
                                                       __nv_bfloat16* __restrict__ packBT) {
-    __shared__ __nv_bfloat16 tile[64][kRankAlign * 4 + 2];  // up to rank 256
+    extern __shared__ __nv_bfloat16 tile[];
     const int i = blockIdx.y;
-    const int64_t c0 = (int64_t)blockIdx.x * 64;
+    const int64_t c0 = (int64_t)blockIdx.x * 128;
     const int r = ad[i].rank;
+    const int ld = r + 2;
     const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(ad[i].B);
-    const int cols = (int)(d_out - c0 < 64 ? d_out - c0 : 64);
-    for (int e = threadIdx.x; e < cols * r; e += blockDim.x) {
-        const int cc = e / r, k = e - cc * r;
-        tile[cc][k] = B[(c0 + cc) * r + k];
+    const int cols = (int)(d_out - c0 < 128 ? d_out - c0 : 128);
+    if ((r & 7) == 0) {
+        // rows of B are 16-byte multiples: 16-byte loads, 8 ranks each
+        const int vr = r >> 3;
+        const uint4* src = reinterpret_cast<const uint4*>(B + c0 * r);
+        for (int e = threadIdx.x; e < cols * vr; e += blockDim.x) {
+            const int cc = e / vr, v = e - cc * vr;
+            const uint4 q = src[e];
+            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&q);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) tile[cc * ld + v * 8 + u] = h[u];
+        }
+    } else {
+        for (int e = threadIdx.x; e < cols * r; e += blockDim.x) {
+            const int cc = e / r, k = e - cc * r;
+            tile[cc * ld + k] = B[(c0 + cc) * r + k];
+        }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < RP * 64; e += blockDim.x) {
-        const int k = e >> 6, cc = e & 63;
+    const int rows = ad[i].rp16;   // rows past the MMA extent are never read
+    for (int e = threadIdx.x; e < rows * 64; e += blockDim.x) {
+        const int k = e >> 6, cc = (e & 63) * 2;
         if (cc < cols) {
-            const __nv_bfloat16 v = (k < r) ? tile[cc][k] : __float2bfloat16_rn(0.f);
-            packBT[((int64_t)i * RP + k) * d_out + c0 + cc] = v;
+            __nv_bfloat162 v;
+            v.x = (k < r) ? tile[cc * ld + k] : __float2bfloat16_rn(0.f);
+            v.y = (k < r) ? tile[(cc + 1) * ld + k] : __float2bfloat16_rn(0.f);
+            *reinterpret_cast<__nv_bfloat162*>(packBT + ((int64_t)i * RP + k) * d_out + c0 + cc) = v;
         }
     }
 }

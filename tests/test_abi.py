@@ -54,7 +54,7 @@ def cfg(d_in=64, d_out=64, dtype=pl.PLORA_BF16, max_adapters=8, max_rank=64, max
     (cfg(max_rank=257), pl.PLORA_ERR_INVALID_ARG),
     (cfg(max_rank=0), pl.PLORA_ERR_INVALID_ARG),
     (cfg(max_tokens=0), pl.PLORA_ERR_INVALID_ARG),
-    (cfg(flags=2), pl.PLORA_ERR_INVALID_ARG),
+    (cfg(flags=4), pl.PLORA_ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_config(c, want):
     s, h = pl.plora_create_status(c)
@@ -141,10 +141,22 @@ def test_token_tiles_cover_every_row_once(seed):
         assert hrow - ad[a, 2] == x - off[a]               # same offset inside the adapter's block
         assert (x - off[a]) % 128 == 0
     assert np.array_equal(owner, np.repeat(np.arange(len(ranks)), np.diff(off)))   # bit-exact map
-    # H/G blocks: each adapter's block is its token count rounded up to 128, packed in order
-    blocks = ((np.diff(off) + 127) // 128) * 128
-    assert np.array_equal(ad[:, 2], np.concatenate([[0], np.cumsum(blocks)[:-1]]))
+    # H/G blocks: every adapter with tokens owns 128 zero rows, its rows rounded up to 128 and
+    # 128 zero rows, packed in order; the first H/G row of its data follows the leading pad.
+    n = np.diff(off)
+    blocks = np.where(n > 0, ((n + 127) // 128) * 128 + 256, 0)
+    starts = np.concatenate([[0], np.cumsum(blocks)[:-1]])
+    assert np.array_equal(ad[n > 0, 2], starts[n > 0] + 128)
     assert h_rows == blocks.sum()
+    # adapters overlapping each global 128-row tile
+    mto = schedule(c, off, ranks, 4)
+    mtl = schedule(c, off, ranks, 5)
+    T = int(off[-1])
+    assert len(mto) == (T + 127) // 128 + 1 and mto[0] == 0 and mto[-1] == len(mtl)
+    for mb in range((T + 127) // 128):
+        m0, m1 = 128 * mb, min(T, 128 * mb + 128)
+        want = [j for j in range(len(ranks)) if n[j] > 0 and off[j] < m1 and off[j + 1] > m0]
+        assert list(mtl[mto[mb]:mto[mb + 1]]) == want
     assert RP == ((max(ranks) + 63) // 64) * 64
     assert np.array_equal(ad[:, 3], ((ranks + 15) // 16) * 16)
     assert np.array_equal(ad[:, 4], ((ranks + 63) // 64) * 64)
@@ -152,7 +164,7 @@ def test_token_tiles_cover_every_row_once(seed):
 
 @pytest.mark.parametrize("seed", range(4))
 def test_weight_grad_splits_cover_tokens_and_depend_only_on_count(seed):
-    off, ranks = random_segments(seed, 24, 0, 13000)
+    off, ranks = random_segments(seed, 24, 0, 40000)
     c = cfg(max_adapters=64, max_rank=256, max_tokens=int(off[-1]) + 1)
     red = schedule(c, off, ranks, 1, grads=True).reshape(-1, 8)
     ks = red[:, 3]
@@ -164,10 +176,10 @@ def test_weight_grad_splits_cover_tokens_and_depend_only_on_count(seed):
             assert len(e) == 0
             continue
         e = e[np.argsort(e[:, 4])]
-        S = (n[i] + 4095) // 4096
+        S = (n[i] + 16383) // 16384
         assert len(e) == S and np.all(e[:, 5] == S) and np.array_equal(e[:, 4], np.arange(S))
-        assert np.array_equal(e[:, 1], off[i] + 4096 * np.arange(S))
-        lens = np.minimum(4096, n[i] - 4096 * np.arange(S))
+        assert np.array_equal(e[:, 1], off[i] + 16384 * np.arange(S))
+        lens = np.minimum(16384, n[i] - 16384 * np.arange(S))
         assert np.array_equal(e[:, 3], (lens + 63) // 64)
         assert (S == 1) == (e[0, 6] == -1)
         # the same adapter alone gets the same splits

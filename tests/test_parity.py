@@ -54,26 +54,36 @@ MIXES = [
 
 
 @pytest.mark.parametrize("k", range(len(MIXES)))
-@pytest.mark.parametrize("path", ["tc", "simt", "fp32"])
+@pytest.mark.parametrize("path", ["tc", "tc_unfused", "simt", "fp32"])
 def test_small_mixes(k, path):
     d_in, d_out, ranks, counts = MIXES[k]
     p = mix(100 + k, "fp32" if path == "fp32" else "bf16", d_in, d_out, ranks, counts)
-    errs, bad = compare(p, run(p, simt=(path == "simt")), full_oracle(p), tol(p))
+    errs, bad = compare(p, run(p, simt=(path == "simt"), unfused=(path == "tc_unfused")), full_oracle(p), tol(p))
     assert not bad, (bad, errs)
 
 
-def test_lora_delta_with_zero_base():
+@pytest.mark.parametrize("unfused", [False, True])
+def test_lora_delta_with_zero_base(unfused):
     """W = 0: Y and dX hold only the LoRA terms, so the bf16 check sees them at full sensitivity."""
-    for k in (1, 2):
+    for k in (1, 2, 3):
         d_in, d_out, ranks, counts = MIXES[k]
         p = wl.with_zero_W(mix(200 + k, "bf16", d_in, d_out, ranks, counts))
-        errs, bad = compare(p, run(p), full_oracle(p), BF16_TOL)
+        errs, bad = compare(p, run(p, unfused=unfused), full_oracle(p), BF16_TOL)
         assert not bad, (bad, errs)
+
+
+def test_many_adapters_in_one_tile():
+    """1- and 2-token adapters: a 128-row tile of the base GEMM overlaps many adapters."""
+    counts = [1, 2, 1, 0, 3, 1, 130, 1, 1, 5, 1, 2, 250, 1]
+    ranks = [1, 8, 16, 4, 64, 3, 32, 256, 2, 17, 1, 8, 100, 5]
+    p = wl.with_zero_W(mix(250, "bf16", 264, 392, ranks, counts))
+    errs, bad = compare(p, run(p), full_oracle(p), BF16_TOL)
+    assert not bad, (bad, errs)
 
 
 def test_weight_grad_split_path():
     """Adapters longer than the split size exercise the split partials and their fixed-order reduction."""
-    p = mix(300, "bf16", 256, 384, [16, 96, 8], [9000, 4097, 300])
+    p = mix(300, "bf16", 256, 384, [16, 96, 8], [34000, 16385, 300])
     errs, bad = compare(p, run(p), full_oracle(p), BF16_TOL)
     assert not bad, (bad, errs)
 
@@ -118,17 +128,17 @@ def test_B_zero_gives_base_and_zero_dA_exactly():
     assert not bad, bad
 
 
-@pytest.mark.parametrize("path", ["tc", "simt"])
+@pytest.mark.parametrize("path", ["tc", "tc_unfused", "simt"])
 def test_packed_equals_alone_bit_exact(path):
-    d_in, d_out, ranks, counts = (384, 520, [1, 16, 100, 64, 8], [300, 129, 0, 4500, 1])
+    d_in, d_out, ranks, counts = (384, 520, [1, 16, 100, 64, 8], [300, 129, 0, 16500, 1])
     p = mix(500, "bf16", d_in, d_out, ranks, counts)
-    g = run(p, simt=(path == "simt"))
+    g = run(p, simt=(path == "simt"), unfused=(path == "tc_unfused"))
     for i in range(p.n_adapters):
         a, b = int(p.off[i]), int(p.off[i + 1])
         q = dataclasses.replace(p, off=np.array([0, b - a], np.int64), ranks=p.ranks[i:i + 1],
                                 alphas=p.alphas[i:i + 1], scales=p.scales[i:i + 1], X=p.X[a:b],
                                 A=[p.A[i]], B=[p.B[i]], dY=p.dY[a:b])
-        h = run(q, simt=(path == "simt"))
+        h = run(q, simt=(path == "simt"), unfused=(path == "tc_unfused"))
         assert np.array_equal(h["Y"], g["Y"][a:b]), i
         assert np.array_equal(h["dX"], g["dX"][a:b]), i
         assert np.array_equal(h["dA"][0], g["dA"][i]), i
@@ -136,7 +146,7 @@ def test_packed_equals_alone_bit_exact(path):
 
 
 def test_repeat_runs_bit_identical():
-    p = mix(600, "bf16", 520, 328, [1, 3, 17, 64, 100], [1, 127, 129, 0, 5000])
+    p = mix(600, "bf16", 520, 328, [1, 3, 17, 64, 100], [1, 127, 129, 0, 17000])
     dev = DeviceProblem(p)
     a, b = run(p, dev=dev), run(p, dev=dev)
     for k in ("Y", "dX"):
@@ -159,7 +169,7 @@ def test_saved_activations_match_oracle_H():
         pl.plora_debug_unpack_saved(eng.h, p.n_adapters, p.off, tab, saved.data_ptr(), i, H.data_ptr())
         torch.cuda.synchronize()
         if n:
-            ref = o["H"][p.off[i]:p.off[i + 1], :r]
+            ref = float(p.scales[i]) * o["H"][p.off[i]:p.off[i + 1], :r]   # saved holds s_i X_i A_i
             assert rel_err(H.cpu().numpy()[:n], ref) <= BF16_TOL
     eng.close()
 
@@ -185,6 +195,11 @@ def test_invalid_call_writes_nothing():
     s = pl.plora_forward(eng.h, d.X.data_ptr() + 2, d.W.data_ptr(), Y.data_ptr(), 2, p.off, tab,
                          saved.data_ptr(), 0, check=False)
     assert s == pl.PLORA_ERR_INVALID_ARG
+    # a host pointer: refused by the extent check, nothing launched
+    host_X = np.zeros((p.T, 256), np.uint16)
+    s = pl.plora_forward(eng.h, host_X.ctypes.data, d.W.data_ptr(), Y.data_ptr(), 2, p.off, tab, saved.data_ptr(),
+                         0, check=False)
+    assert s == pl.PLORA_ERR_INVALID_ARG and "X is not a device buffer" in pl.plora_last_error(eng.h)
     torch.cuda.synchronize()
     assert bool(torch.all(Y == 7.0))
     assert pl.plora_check(eng.h, 0) == pl.PLORA_OK

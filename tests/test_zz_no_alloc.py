@@ -25,10 +25,10 @@ import packed_lora_fine_b200 as pl  # noqa: E402
 
 
 def _problem():
-    # Two adapters longer than the 4096-token split (so split partials and arrival
+    # Two adapters longer than the 16384-token split (so split partials and arrival
     # counters are used), a short one and an empty one.
     r = np.array([16, 96, 8, 24])
-    return wl.make_problem("noalloc", "bf16", 256, 384, r, [9000, 4097, 300, 0], 2.0 * r,
+    return wl.make_problem("noalloc", "bf16", 256, 384, r, [34000, 16385, 300, 0], 2.0 * r,
                            wl.init_llm(256), 4242)
 
 
@@ -60,10 +60,16 @@ def test_static_grad_B_matches_backward_twice():
 
 
 def test_static_grad_B_rejects_oversized_calls():
-    # 300 000 tokens in one adapter: 74 splits x 3 d-tiles x 128 x 256 x 4 bytes > the static array.
-    cfg = pl.plora_config(256, 384, pl.PLORA_BF16, 1, 256, 0, 300000)
-    tab = pl.make_table([256], [1.0], [1 << 20], [1 << 21], [1 << 22], [1 << 23])
-    st = pl.plora_grad_B_static(cfg, 1 << 24, 1, np.array([0, 300000], np.int64), tab, 1 << 25, 0)
+    """Calls whose split partials cannot fit the static array are refused before any device work.
+    The precondition is computed here from the documented limit first, so that a change of the
+    library's constants can never turn this into a launch on the placeholder pointers below."""
+    split, d_out, rank, tokens = 16384, 65536, 256, 40000
+    splits = -(-tokens // split)
+    partial_bytes = splits * (-(-d_out // 128)) * (4 + 128 * rank * 4)
+    assert splits > 1 and partial_bytes > 8 * (pl.PLORA_STATIC_SCRATCH_BYTES)
+    cfg = pl.plora_config(256, d_out, pl.PLORA_BF16, 1, rank, 0, tokens)
+    tab = pl.make_table([rank], [1.0], [1 << 20], [1 << 21], [1 << 22], [1 << 23])
+    st = pl.plora_grad_B_static(cfg, 1 << 24, 1, np.array([0, tokens], np.int64), tab, 1 << 25, 0)
     assert st == pl.PLORA_ERR_UNSUPPORTED
     cfg32 = pl.plora_config(256, 384, pl.PLORA_FP32, 1, 256, 0, 1000)
     st = pl.plora_grad_B_static(cfg32, 1 << 24, 1, np.array([0, 1000], np.int64), tab, 1 << 25, 0)
