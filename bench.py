@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="run the expand products as separate passes (for comparison with the fused default)")
+    ap.add_argument("--base-pair", action="store_true",
+                    help="base GEMMs on SM pairs (cta_group::2) instead of single SMs")
     ap.add_argument("--suite", action="store_true",
                     help="measure every workload (packed vs per-adapter sequential loop); one JSON line each")
     ap.add_argument("--workload", choices=["llama_up32", "small", "layer_q"], default="llama_up32",
@@ -278,7 +280,7 @@ def main(argv=None):
     dA = [torch.empty(a.shape, dtype=torch.float32, device=dev) for a in A]
     dB = [torch.empty(b.shape, dtype=torch.float32, device=dev) for b in B]
     eng = pl.PackedLoRA(p.d_in, p.d_out, "bf16", max_adapters=p.n_adapters, max_rank=int(max(p.ranks)),
-                        max_tokens=T, unfused=args.unfused)
+                        max_tokens=T, unfused=args.unfused, base_pair=args.base_pair)
     tab_f = eng.table(p.scales, A, B)
     tab_b = eng.table(p.scales, A, B, dA, dB)
     saved = torch.empty(eng.saved_bytes(p.off, tab_f), dtype=torch.uint8, device=dev)

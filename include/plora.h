@@ -93,8 +93,10 @@ typedef enum {
 /* plora_config.flags */
 enum {
     PLORA_FLAG_SIMT = 1u,     /* bf16 only: run the plain SIMT kernels instead of the tensor-core ones */
-    PLORA_FLAG_UNFUSED = 2u   /* tensor-core path: run the expand products (Y += s H B, dX += G A^T) as
+    PLORA_FLAG_UNFUSED = 2u,  /* tensor-core path: run the expand products (Y += s H B, dX += G A^T) as
                                  separate read-modify-write passes instead of inside the base GEMMs */
+    PLORA_FLAG_BASE_PAIR = 4u /* tensor-core path: base GEMMs on SM pairs (256-row tiles, tcgen05
+                                 cta_group::2, half the B staging per SM) instead of single SMs */
 };
 
 /* Limits. */
@@ -209,13 +211,13 @@ PLORA_API plora_status plora_debug_unpack_saved(plora_handle h, int32_t n_adapte
  *              first H/G row, 64-token blocks, split index, split count,
  *              first partial slot (-1 if unsplit), first counter (-1);
  *   which = 2: adapters, 5 per adapter: first token row, tokens, first H/G
- *              row (each adapter with tokens owns a block of 128 zero rows,
- *              its rows rounded up to 128, then 128 zero rows), rank rounded
+ *              row (each adapter with tokens owns a block of 256 zero rows,
+ *              its rows rounded up to 128, then 256 zero rows), rank rounded
  *              up to 16, rank rounded up to 64;
  *   which = 3: two values: the padded rank pitch RP and the H/G row count;
- *   which = 4: per global 128-row tile, the first index into the list of
- *              which = 5 (plus the end), i.e. ceil(T/128) + 1 values;
- *   which = 5: the adapters (with tokens) overlapping each global tile.
+ *   which = 4: per global 256-row tile of the base GEMMs, the first index
+ *              into the list of which = 5 (plus the end): ceil(T/256) + 1 values;
+ *   which = 5: the adapters (with tokens) overlapping each such tile.
  * *count receives the number of int32 values the full answer needs.
  */
 PLORA_API plora_status plora_debug_schedule(const plora_config* cfg, int32_t n_adapters, const int64_t* off,

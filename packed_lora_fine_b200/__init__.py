@@ -32,6 +32,7 @@ PLORA_BF16 = 0
 PLORA_FP32 = 1
 PLORA_FLAG_SIMT = 1
 PLORA_FLAG_UNFUSED = 2
+PLORA_FLAG_BASE_PAIR = 4
 PLORA_MAX_RANK = 256
 PLORA_MAX_ADAPTERS = 4096
 PLORA_STATIC_SCRATCH_BYTES = 16 << 20
@@ -245,12 +246,13 @@ class PackedLoRA:
     """
 
     def __init__(self, d_in, d_out, dtype="bf16", max_adapters=64, max_rank=PLORA_MAX_RANK,
-                 max_tokens=1 << 16, simt=False, unfused=False):
+                 max_tokens=1 << 16, simt=False, unfused=False, base_pair=False):
         self.d_in, self.d_out = int(d_in), int(d_out)
         self.dtype = dtype
         self.h = plora_create(self.d_in, self.d_out, PLORA_BF16 if dtype == "bf16" else PLORA_FP32,
                               max_adapters, max_rank, max_tokens,
-                              (PLORA_FLAG_SIMT if simt else 0) | (PLORA_FLAG_UNFUSED if unfused else 0))
+                              (PLORA_FLAG_SIMT if simt else 0) | (PLORA_FLAG_UNFUSED if unfused else 0)
+                              | (PLORA_FLAG_BASE_PAIR if base_pair else 0))
 
     def close(self):
         if self.h:

@@ -12,6 +12,8 @@ constexpr int kTileM = 128;     // token rows (or hidden rows) per tensor-core t
 constexpr int kBlockK = 64;     // K elements per pipeline stage (128 bytes of bf16)
 constexpr int kRankAlign = 64;  // the padded rank width RP of the saved/G buffers is a multiple of this
 constexpr int kSplitTokens = 16384; // weight-gradient split size along the tokens (fixed: deterministic)
+constexpr int kLoraPad = 256;       // zero rows before and after each adapter's H' / G block
+constexpr int kLoraTileM = 256;     // base-GEMM rows per overlap record (one CTA-pair tile)
 
 // One adapter, as the kernels see it.
 struct AdapterDev {

@@ -21,6 +21,7 @@
 #include "plan.cuh"
 #include "simt.cuh"
 #include "tc.cuh"
+#include "tc_pair.cuh"
 
 using namespace plora;
 
@@ -45,6 +46,7 @@ struct plora_ctx {
     int64_t max_slots = 0, max_counters = 0;
     size_t blob_bytes = 0;
     bool tc = false;           // tensor-core path (bf16 without PLORA_FLAG_SIMT)
+    int pairs_fwd = 0, pairs_dx = 0;   // co-resident SM pairs for the pair-tile base GEMMs
 
     uint8_t* ws = nullptr;     // one device allocation, carved into regions
     size_t ws_bytes = 0;
@@ -250,8 +252,8 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
             continue;
         }
         // H' / G block: 128 zero rows, the adapter's rows rounded up to 128, 128 zero rows.
-        a.h_row = (int32_t)(hrow + kTileM);
-        hrow += round_up(a.n, kTileM) + 2 * kTileM;
+        a.h_row = (int32_t)(hrow + kLoraPad);
+        hrow += round_up(a.n, kTileM) + 2 * kLoraPad;
         for (int32_t t = 0; t < a.n; t += kTileM)
             P.tok.push_back(TokTile{i, std::min(kTileM, a.n - t), a.x_row + t, a.h_row + t});
         // Weight-gradient splits: a function of this adapter's token count alone, so an
@@ -272,11 +274,11 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
     }
     P.h_rows = hrow;
     // Adapters overlapping each global 128-row tile (for the base GEMMs with the low-rank branch folded in).
-    const int64_t tiles_m = ceil_div(P.T, kTileM);
+    const int64_t tiles_m = ceil_div(P.T, kLoraTileM);
     P.mt_off.assign(tiles_m + 1, 0);
     int32_t first = 0;
     for (int64_t mb = 0; mb < tiles_m; ++mb) {
-        const int64_t m0 = mb * kTileM, m1 = std::min<int64_t>(P.T, m0 + kTileM);
+        const int64_t m0 = mb * kLoraTileM, m1 = std::min<int64_t>(P.T, m0 + kLoraTileM);
         P.mt_off[mb] = (int32_t)P.mt_seg.size();
         while (first < n && off[first + 1] <= m0) ++first;
         for (int32_t j = first; j < n && off[j] < m1; ++j)
@@ -430,6 +432,60 @@ void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const C
     tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p); });
 }
 
+// Base GEMMs on SM pairs: a cluster of two CTAs per 256x256 tile, persistent over the pairs that
+// can be resident at once (a GPC with an odd number of free SMs leaves one unpaired).
+template <Op OP>
+cudaLaunchConfig_t pair_config(int pairs, cudaStream_t st, cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kTcSmemBytes;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+template <Op OP>
+void launch_pair(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                 const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+    if (p.num_tiles <= 0) return;
+    const int resident = OP == Op::BaseFwd ? h->pairs_fwd : h->pairs_dx;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config<OP>(std::min(p.num_tiles, resident), st, attr);
+    constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : kBaseDx;
+    tracked(h, kind, st, [&] { cudaLaunchKernelEx(&cfg, tc_pair_kernel<OP>, a, b, a2, b2, p); });
+}
+
+template <Op OP>
+cudaError_t pair_setup(int& pairs) {
+    cudaError_t e = cudaFuncSetAttribute(tc_pair_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_pair_kernel<OP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config<OP>(1, nullptr, attr);
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, tc_pair_kernel<OP>, &cfg);
+    if (e != cudaSuccess) return e;
+    pairs = clusters;
+    return pairs > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+// Pair-tile parameters of a base GEMM over T rows: 256-row m-tiles, 32 KB stages, a 6-deep ring.
+void pair_params(TcParams& p, int64_t T, int64_t N) {
+    p.tiles_m = (int32_t)ceil_div(T, 2 * kTileM);
+    p.tiles_n = (int32_t)ceil_div(N, kTileN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.group_m = 8;
+    p.stage_bytes = kPairStageBytes;
+    p.stages = std::min(kMaxStages, kRingBytes / kPairStageBytes);
+}
+
 // A deeper operand ring for ops whose B tile is narrower than 256 rows: A tile + RP rows of B.
 void narrow_ring(TcParams& p, int RP) {
     p.stage_bytes = kABytes + RP * kBlockK * 2;
@@ -508,7 +564,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     if (cfg->max_adapters < 1 || cfg->max_adapters > PLORA_MAX_ADAPTERS) return PLORA_ERR_INVALID_ARG;
     if (cfg->max_rank < 1 || cfg->max_rank > PLORA_MAX_RANK) return PLORA_ERR_INVALID_ARG;
     if (cfg->max_tokens < 1 || cfg->max_tokens > ((int64_t)1 << 30)) return PLORA_ERR_INVALID_ARG;
-    if (cfg->flags & ~(uint32_t)(PLORA_FLAG_SIMT | PLORA_FLAG_UNFUSED)) return PLORA_ERR_INVALID_ARG;
+    if (cfg->flags & ~(uint32_t)(PLORA_FLAG_SIMT | PLORA_FLAG_UNFUSED | PLORA_FLAG_BASE_PAIR)) return PLORA_ERR_INVALID_ARG;
 
     plora_ctx* h = new (std::nothrow) plora_ctx();
     if (!h) return PLORA_ERR_OOM;
@@ -527,7 +583,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     // Workspace sizing (all bounds follow from the config).
     const int64_t na = cfg->max_adapters;
     h->RPmax = (int)round_up(cfg->max_rank, kRankAlign);
-    h->max_h_rows = cfg->max_tokens + (int64_t)(3 * kTileM - 1) * na;
+    h->max_h_rows = cfg->max_tokens + (int64_t)(kTileM - 1 + 2 * kLoraPad) * na;
     const int64_t dtiles = std::max(ceil_div(cfg->d_in, kTileM), ceil_div(cfg->d_out, kTileM));
     h->max_slots = 2 * (cfg->max_tokens / kSplitTokens) + 1;
     h->max_counters = (cfg->max_tokens / (kSplitTokens + 1) + 1) * dtiles;
@@ -573,6 +629,8 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
         if (e == cudaSuccess) e = set_tc_attr<Op::ExpandDx>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradB>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradA>();
+        if (e == cudaSuccess) e = pair_setup<Op::BaseFwd>(h->pairs_fwd);
+        if (e == cudaSuccess) e = pair_setup<Op::BaseDx>(h->pairs_dx);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(pack_bt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      128 * (PLORA_MAX_RANK + 2) * (int)sizeof(__nv_bfloat16));
@@ -682,9 +740,10 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
     pack_factors(h, P, D, st);
-    CUtensorMap mX, mW, mPA, mHk, mPB, mPB16;
+    CUtensorMap mX, mW, mW128, mPA, mHk, mPB, mPB16;
     bool ok = make_map(&mX, X, d_in, P.T, d_in, 64, kTileM) &&
               make_map(&mW, W, d_in, d_out, d_in, 64, kTileN) &&
+              make_map(&mW128, W, d_in, d_out, d_in, 64, kTileM) &&
               make_map(&mPA, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, P.RP) &&
               make_map(&mHk, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
               make_map(&mPB, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 64) &&
@@ -709,7 +768,12 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     p.b_box_rows = kTileN;
     p.out = Y; p.out_ld = d_out;
     p.fuse = fused ? 1 : 0;
-    launch_tc<Op::BaseFwd>(h, mX, mW, mHk, mPB16, p, st);
+    if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
+        pair_params(p, P.T, d_out);
+        launch_pair<Op::BaseFwd>(h, mX, mW128, mHk, mPB16, p, st);
+    } else {
+        launch_tc<Op::BaseFwd>(h, mX, mW, mHk, mPB16, p, st);
+    }
     if (!fused) {
         // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
         TcParams r = base_params(h, P, D);
@@ -832,7 +896,12 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
         p.num_tiles = p.tiles_m * p.tiles_n;
         p.out = dX; p.out_ld = d_in;
         p.fuse = fused ? 1 : 0;
-        launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, p, st);
+        if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
+            pair_params(p, P.T, d_in);
+            launch_pair<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, p, st);
+        } else {
+            launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, p, st);
+        }
         if (!fused) {
             // K6 as its own pass: dX_i += G_i A_i^T (read-modify-write of dX).
             TcParams r = base_params(h, P, D);

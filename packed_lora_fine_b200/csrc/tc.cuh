@@ -187,12 +187,20 @@ __device__ __forceinline__ MTileRec load_mtile(const TcParams& p, int t) {
     r.q0 = r.q1 = 0;
     if (OpTraits<OP>::kBase && p.fuse && t < p.num_tiles) {
         const TileInfo ti = decode_tile<OP>(p, t);
-        r = p.mt_rec[ti.mtile];
+        r = p.mt_rec[ti.mtile / (kLoraTileM / kTileM)];
+        // a 128-row tile reads its half of the 256-row record's rows
+        const int shift = (ti.mtile % (kLoraTileM / kTileM)) * kTileM;
+        r.s[0].h_y += shift;
+        r.s[1].h_y += shift;
+        r.pad_[0] = shift;
     }
     return r;
 }
 __device__ __forceinline__ LoraSeg mtile_seg(const TcParams& p, const MTileRec& r, int q) {
-    return q - r.q0 < 2 ? r.s[q - r.q0] : p.mt_seg[q];
+    if (q - r.q0 < 2) return r.s[q - r.q0];
+    LoraSeg s = p.mt_seg[q];
+    s.h_y += r.pad_[0];
+    return s;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -445,8 +453,8 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     *reinterpret_cast<uint4*>(out + c) = v0;
                     *reinterpret_cast<uint4*>(out + c + 8) = v1;
                 }
-                // The adapter's block has 128 zero rows before and after its (128-rounded) rows, so that a
-                // base tile straddling the segment can read it at any row offset; the first and the last
+                // The adapter's block has kLoraPad zero rows before and after its (128-rounded) rows, so that
+                // a base tile straddling the segment can read it at any row offset; the first and the last
                 // tile of the adapter write them.
                 const AdapterDev ad = p.adapters[ti.adapter];
                 const bool first = ti.out_row == ad.h_row;
@@ -454,14 +462,16 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 if (first || last) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
                     __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.out);
-                    if (first) {
-                        uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(ad.h_row - kTileM + row) * p.out_ld);
-                        for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
-                    }
-                    if (last) {
-                        const int tail = ad.h_row + ((ad.n + kTileM - 1) / kTileM) * kTileM;
-                        uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(tail + row) * p.out_ld);
-                        for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                    const int tail = ad.h_row + ((ad.n + kTileM - 1) / kTileM) * kTileM;
+                    for (int pr = row; pr < kLoraPad; pr += kTileM) {
+                        if (first) {
+                            uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(ad.h_row - kLoraPad + pr) * p.out_ld);
+                            for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                        }
+                        if (last) {
+                            uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(tail + pr) * p.out_ld);
+                            for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                        }
                     }
                 }
             } else if constexpr (Tr::kExpand) {

@@ -38,7 +38,7 @@ class DeviceProblem:
         self.B = [to_dev(b, p, device) for b in p.B]
 
 
-def run(p, simt=False, dev=None, want_dX=True, engine=None, max_tokens=None, unfused=False):
+def run(p, simt=False, dev=None, want_dX=True, engine=None, max_tokens=None, unfused=False, base_pair=False):
     """One packed forward + backward through the C ABI. Returns numpy float64 outputs."""
     import torch
     import packed_lora_fine_b200 as pl
@@ -47,7 +47,8 @@ def run(p, simt=False, dev=None, want_dX=True, engine=None, max_tokens=None, unf
     if own:
         engine = pl.PackedLoRA(p.d_in, p.d_out, p.dtype, max_adapters=max(1, p.n_adapters),
                                max_rank=int(max(p.ranks)) if p.n_adapters else 1,
-                               max_tokens=max_tokens or max(1, p.T), simt=simt, unfused=unfused)
+                               max_tokens=max_tokens or max(1, p.T), simt=simt, unfused=unfused,
+                               base_pair=base_pair)
     off = p.off
     Y, saved = engine.forward(d.X, d.W, off, p.scales, d.A, d.B)
     dX, dA, dB = engine.backward(d.X, d.W, d.dY, off, p.scales, d.A, d.B, saved, want_dX=want_dX)

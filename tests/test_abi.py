@@ -54,7 +54,7 @@ def cfg(d_in=64, d_out=64, dtype=pl.PLORA_BF16, max_adapters=8, max_rank=64, max
     (cfg(max_rank=257), pl.PLORA_ERR_INVALID_ARG),
     (cfg(max_rank=0), pl.PLORA_ERR_INVALID_ARG),
     (cfg(max_tokens=0), pl.PLORA_ERR_INVALID_ARG),
-    (cfg(flags=4), pl.PLORA_ERR_INVALID_ARG),
+    (cfg(flags=8), pl.PLORA_ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_config(c, want):
     s, h = pl.plora_create_status(c)
@@ -141,20 +141,20 @@ def test_token_tiles_cover_every_row_once(seed):
         assert hrow - ad[a, 2] == x - off[a]               # same offset inside the adapter's block
         assert (x - off[a]) % 128 == 0
     assert np.array_equal(owner, np.repeat(np.arange(len(ranks)), np.diff(off)))   # bit-exact map
-    # H/G blocks: every adapter with tokens owns 128 zero rows, its rows rounded up to 128 and
-    # 128 zero rows, packed in order; the first H/G row of its data follows the leading pad.
+    # H/G blocks: every adapter with tokens owns 256 zero rows, its rows rounded up to 128 and
+    # 256 zero rows, packed in order; the first H/G row of its data follows the leading pad.
     n = np.diff(off)
-    blocks = np.where(n > 0, ((n + 127) // 128) * 128 + 256, 0)
+    blocks = np.where(n > 0, ((n + 127) // 128) * 128 + 512, 0)
     starts = np.concatenate([[0], np.cumsum(blocks)[:-1]])
-    assert np.array_equal(ad[n > 0, 2], starts[n > 0] + 128)
+    assert np.array_equal(ad[n > 0, 2], starts[n > 0] + 256)
     assert h_rows == blocks.sum()
-    # adapters overlapping each global 128-row tile
+    # adapters overlapping each global 256-row tile of the base GEMMs
     mto = schedule(c, off, ranks, 4)
     mtl = schedule(c, off, ranks, 5)
     T = int(off[-1])
-    assert len(mto) == (T + 127) // 128 + 1 and mto[0] == 0 and mto[-1] == len(mtl)
-    for mb in range((T + 127) // 128):
-        m0, m1 = 128 * mb, min(T, 128 * mb + 128)
+    assert len(mto) == (T + 255) // 256 + 1 and mto[0] == 0 and mto[-1] == len(mtl)
+    for mb in range((T + 255) // 256):
+        m0, m1 = 256 * mb, min(T, 256 * mb + 256)
         want = [j for j in range(len(ranks)) if n[j] > 0 and off[j] < m1 and off[j + 1] > m0]
         assert list(mtl[mto[mb]:mto[mb + 1]]) == want
     assert RP == ((max(ranks) + 63) // 64) * 64

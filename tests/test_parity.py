@@ -54,11 +54,12 @@ MIXES = [
 
 
 @pytest.mark.parametrize("k", range(len(MIXES)))
-@pytest.mark.parametrize("path", ["tc", "tc_unfused", "simt", "fp32"])
+@pytest.mark.parametrize("path", ["tc", "tc_pair", "tc_unfused", "simt", "fp32"])
 def test_small_mixes(k, path):
     d_in, d_out, ranks, counts = MIXES[k]
     p = mix(100 + k, "fp32" if path == "fp32" else "bf16", d_in, d_out, ranks, counts)
-    errs, bad = compare(p, run(p, simt=(path == "simt"), unfused=(path == "tc_unfused")), full_oracle(p), tol(p))
+    g = run(p, simt=(path == "simt"), unfused=(path == "tc_unfused"), base_pair=(path == "tc_pair"))
+    errs, bad = compare(p, g, full_oracle(p), tol(p))
     assert not bad, (bad, errs)
 
 
@@ -72,12 +73,13 @@ def test_lora_delta_with_zero_base(unfused):
         assert not bad, (bad, errs)
 
 
-def test_many_adapters_in_one_tile():
-    """1- and 2-token adapters: a 128-row tile of the base GEMM overlaps many adapters."""
+@pytest.mark.parametrize("base_pair", [False, True])
+def test_many_adapters_in_one_tile(base_pair):
+    """1- and 2-token adapters: a base-GEMM tile overlaps many adapters."""
     counts = [1, 2, 1, 0, 3, 1, 130, 1, 1, 5, 1, 2, 250, 1]
     ranks = [1, 8, 16, 4, 64, 3, 32, 256, 2, 17, 1, 8, 100, 5]
     p = wl.with_zero_W(mix(250, "bf16", 264, 392, ranks, counts))
-    errs, bad = compare(p, run(p), full_oracle(p), BF16_TOL)
+    errs, bad = compare(p, run(p, base_pair=base_pair), full_oracle(p), BF16_TOL)
     assert not bad, (bad, errs)
 
 
@@ -128,17 +130,17 @@ def test_B_zero_gives_base_and_zero_dA_exactly():
     assert not bad, bad
 
 
-@pytest.mark.parametrize("path", ["tc", "tc_unfused", "simt"])
+@pytest.mark.parametrize("path", ["tc", "tc_pair", "tc_unfused", "simt"])
 def test_packed_equals_alone_bit_exact(path):
     d_in, d_out, ranks, counts = (384, 520, [1, 16, 100, 64, 8], [300, 129, 0, 16500, 1])
     p = mix(500, "bf16", d_in, d_out, ranks, counts)
-    g = run(p, simt=(path == "simt"), unfused=(path == "tc_unfused"))
+    g = run(p, simt=(path == "simt"), unfused=(path == "tc_unfused"), base_pair=(path == "tc_pair"))
     for i in range(p.n_adapters):
         a, b = int(p.off[i]), int(p.off[i + 1])
         q = dataclasses.replace(p, off=np.array([0, b - a], np.int64), ranks=p.ranks[i:i + 1],
                                 alphas=p.alphas[i:i + 1], scales=p.scales[i:i + 1], X=p.X[a:b],
                                 A=[p.A[i]], B=[p.B[i]], dY=p.dY[a:b])
-        h = run(q, simt=(path == "simt"), unfused=(path == "tc_unfused"))
+        h = run(q, simt=(path == "simt"), unfused=(path == "tc_unfused"), base_pair=(path == "tc_pair"))
         assert np.array_equal(h["Y"], g["Y"][a:b]), i
         assert np.array_equal(h["dX"], g["dX"][a:b]), i
         assert np.array_equal(h["dA"][0], g["dA"][i]), i
