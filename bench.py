@@ -363,8 +363,10 @@ def main(argv=None):
                 "frac": kd["frac"], "traffic": traffic, "kernel": dom,
                 "peak_source": f"{peaks_src} {peak_key}"}
 
-    # End to end through the C ABI with host buffers: every step copies X and dY in from pinned
-    # host memory, runs forward + backward, and copies every adapter's dA, dB out to pinned memory.
+    # End to end through the C ABI with host buffers, pipelined like a training loop: every step
+    # copies its X and dY in from pinned host memory (copy stream), runs forward + backward (compute
+    # stream), and copies every adapter's dA, dB out to pinned host memory (copy-out stream).  Inputs
+    # and gradients are double-buffered, so step k+1's inputs stream in while step k computes.
     e2e = None
     if not args.no_e2e:
         hX = torch.empty(X.shape, dtype=X.dtype, pin_memory=True).copy_(X.cpu())
@@ -373,31 +375,61 @@ def main(argv=None):
         hdB = [torch.empty(b.shape, dtype=torch.float32, pin_memory=True) for b in dB]
         h2d = hX.numel() * 2 + hdY.numel() * 2
         d2h = sum(a.numel() * 4 for a in hdA) + sum(b.numel() * 4 for b in hdB)
+        Xb = [X, torch.empty_like(X)]
+        dYb = [dY, torch.empty_like(dY)]
+        dAb = [dA, [torch.empty_like(a) for a in dA]]
+        dBb = [dB, [torch.empty_like(b) for b in dB]]
+        tabs = [tab_b, eng.table(p.scales, A, B, dAb[1], dBb[1])]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()
+        in_done = [ev(), ev()]
+        used = [ev(), ev()]      # compute of the step that last read / wrote buffer b is done
+        out_done = [ev(), ev()]  # copy-out of buffer b's gradients is done
+        for e_ in used + out_done:
+            e_.record(stream)
 
-        def e2e_step():
-            X.copy_(hX, non_blocking=True)
-            dY.copy_(hdY, non_blocking=True)
-            step()
-            for a, h in zip(dA, hdA):
-                h.copy_(a, non_blocking=True)
-            for b, h in zip(dB, hdB):
-                h.copy_(b, non_blocking=True)
+        def e2e_step(k):
+            b = k % 2
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(used[b])
+                Xb[b].copy_(hX, non_blocking=True)
+                dYb[b].copy_(hdY, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            stream.wait_event(out_done[b])
+            pl.plora_forward(eng.h, Xb[b].data_ptr(), W.data_ptr(), Y.data_ptr(), n, off, tab_f, saved.data_ptr(),
+                             st)
+            pl.plora_backward(eng.h, Xb[b].data_ptr(), W.data_ptr(), dYb[b].data_ptr(), dX.data_ptr(), n, off,
+                              tabs[b], saved.data_ptr(), st)
+            used[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(used[b])
+                for a, h in zip(dAb[b], hdA):
+                    h.copy_(a, non_blocking=True)
+                for g_, h in zip(dBb[b], hdB):
+                    h.copy_(g_, non_blocking=True)
+                out_done[b].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        for k in range(2):
+            e2e_step(k)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         k2 = max(5, min(args.steps, 20))
         e0.record(stream)
-        for _ in range(k2):
-            e2e_step()
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        for k in range(k2):
+            e2e_step(k)
+        stream.wait_stream(s_out)
+        stream.wait_stream(s_in)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
         ms_e2e = reduce_max(e0.elapsed_time(e1) / k2, dist)
         e2e = {"value": tokens_all / (ms_e2e / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": k2}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": ms_e2e, "steps": k2,
+               "pipeline": "H2D of step k+1 overlaps compute of step k (double-buffered inputs and gradients)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -481,7 +481,7 @@ void pair_params(TcParams& p, int64_t T, int64_t N) {
     p.tiles_m = (int32_t)ceil_div(T, 2 * kTileM);
     p.tiles_n = (int32_t)ceil_div(N, kTileN);
     p.num_tiles = p.tiles_m * p.tiles_n;
-    p.group_m = 8;
+    p.group_m = 16;   // the same 4096-row window in 256-row pair tiles
     p.stage_bytes = kPairStageBytes;
     p.stages = std::min(kMaxStages, kRingBytes / kPairStageBytes);
 }
@@ -507,7 +507,7 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     p.timeout_ns = kTimeoutNs;
     p.partials = h->at<float>(h->r_part);
     p.counters = h->at<int32_t>(h->r_cnt);
-    p.group_m = 16;
+    p.group_m = 32;   // 32 x 128 rows: a 4096-row window of A stays in L2 while W streams past it
     p.mt_rec = D.mt_rec;
     p.mt_seg = D.mt_seg;
     p.fuse = 0;

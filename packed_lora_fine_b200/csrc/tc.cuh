@@ -56,7 +56,8 @@ constexpr int kStageBytes = kABytes + kBBytesMax;
 constexpr int kTmemCols = 512;                    // two 256-column fp32 accumulators
 constexpr int kTcThreads = 192;
 constexpr int kRingBytes = kStages * kStageBytes; // 192 KB of operand ring
-constexpr int kTcSmemBytes = kRingBytes + 1024 /* align */ + 256 /* barriers */;
+constexpr int kEpiStageFloats = 32 * 33;          // per epilogue warp: a 32 x 32 fp32 chunk (padded rows)
+constexpr int kTcSmemBytes = kRingBytes + 1024 /* align */ + 256 /* barriers */ + 4 * kEpiStageFloats * 4;
 
 struct TcParams {
     int32_t M_total;        // Base: T; Wgrad: d (rows of dB_i or columns of dA_i)
@@ -230,6 +231,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int stb = p.stage_bytes;                   // bytes per stage (multiple of 1024)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* red_flag = reinterpret_cast<int*>(tmem_slot + 2);
+    float* epi_stage = reinterpret_cast<float*>(smem + kRingBytes + 256);   // [4 warps][32][33]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -514,7 +516,38 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                 const int rank = ad.rank;
                 const int hid = ti.out_row + row;
                 const float s = ti.scale;
-                if (re.nsplit == 1) {
+                if (re.nsplit == 1 && OP == Op::WgradB) {
+                    // dB_i's 128-row tile is one contiguous block ([row][rank]); stage 32 x 32 chunks of
+                    // this warp's rows in shared memory and store them with consecutive lanes on
+                    // consecutive addresses.
+                    float* stg = epi_stage + q * kEpiStageFloats;
+                    const int row0 = ti.out_row + q * 32;                 // first hidden row of this warp
+                    const int nrows = min(32, p.M_total - row0);
+                    float* blk = ad.dB + (int64_t)row0 * rank;
+                    for (int c0 = 0; c0 < ti.mma_n && c0 < rank; c0 += 32) {
+                        uint32_t r[16];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            ptx::tmem_ld16(t_row + c0 + 16 * hh, r);
+                            ptx::tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) stg[lane * 33 + 16 * hh + e] = s * __uint_as_float(r[e]);
+                        }
+                        __syncwarp();
+                        const int ncols = min(32, rank - c0);
+                        if (rank <= 32) {
+                            // the whole [nrows][rank] block is contiguous: linear stores
+                            for (int idx = lane; idx < nrows * rank; idx += 32) {
+                                const int rr = idx / rank, cc = idx - rr * rank;
+                                blk[idx] = stg[rr * 33 + cc];
+                            }
+                        } else {
+                            for (int rr = 0; rr < nrows; ++rr)
+                                if (lane < ncols) blk[(int64_t)rr * rank + c0 + lane] = stg[rr * 33 + lane];
+                        }
+                        __syncwarp();
+                    }
+                } else if (re.nsplit == 1) {
                     for (int c = 0; c < ti.mma_n; c += 16) {
                         uint32_t r[16];
                         ptx::tmem_ld16(t_row + c, r);
@@ -523,11 +556,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
                                 const int k = c + e;
-                                if (k < rank) {
-                                    const float v = s * __uint_as_float(r[e]);
-                                    if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = v;
-                                    else ad.dA[(int64_t)k * p.M_total + hid] = v;
-                                }
+                                if (k < rank) ad.dA[(int64_t)k * p.M_total + hid] = s * __uint_as_float(r[e]);
                             }
                         }
                     }
