@@ -583,7 +583,33 @@ def run_suite(args):
                 kern[k] = {"launches": c, "ms_per_step": tot / steps}
         base_ms = sum(v["ms_per_step"] for k, v in kern.items() if k in TC_KINDS)
         base_flops = sum(4.0 * T * L["di"] * L["do"] for L in layers)
-        line = {"suite": name, "tokens": T, "adapters": n, "projections": len(layers),
+        adamw = None
+        if len(layers) == 1:
+            # the optimizer step of the same adapters: fp32 masters and moments, grads from the step above
+            L = layers[0]
+            f32 = lambda t_: torch.zeros(t_.shape, dtype=torch.float32, device=dev)
+            Am = [a.float() for a in L["A"]]
+            Bm = [b.float() for b in L["B"]]
+            mA, vA = [f32(a) for a in L["A"]], [f32(a) for a in L["A"]]
+            mB, vB = [f32(b) for b in L["B"]], [f32(b) for b in L["B"]]
+            hps = [dict(lr=1e-4, step=1) for _ in range(n)]
+            sts = pl.make_adamw_states(hps, [x.data_ptr() for x in Am], [x.data_ptr() for x in Bm],
+                                       [x.data_ptr() for x in mA], [x.data_ptr() for x in vA],
+                                       [x.data_ptr() for x in mB], [x.data_ptr() for x in vB])
+            e = L["eng"]
+            for _ in range(3):
+                pl.plora_adamw_step(e.h, n, L["tb"], sts, st.cuda_stream)
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(st)
+            for _ in range(20):
+                pl.plora_adamw_step(e.h, n, L["tb"], sts, st.cuda_stream)
+            a1.record(st)
+            torch.cuda.synchronize()
+            ms_a = a0.elapsed_time(a1) / 20
+            elems = sum(int(r) * (L["di"] + L["do"]) for r in ranks)
+            adamw = {"ms": ms_a, "elements": elems, "hbm_frac": elems * 30 / (ms_a / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        line = {"suite": name, "tokens": T, "adapters": n, "projections": len(layers), "adamw_step": adamw,
                 "packed_ms_per_step": ms_p, "packed_tokens_per_s": T / (ms_p / 1e3),
                 "sequential_ms_per_step": ms_s, "sequential_tokens_per_s": T / (ms_s / 1e3),
                 "packed_over_sequential": ms_s / ms_p,

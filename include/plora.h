@@ -225,6 +225,42 @@ PLORA_API plora_status plora_debug_schedule(const plora_config* cfg, int32_t n_a
                                             int32_t* out, int64_t capacity, int64_t* count);
 
 /*
+ * Optimizer state of one adapter for plora_adamw_step.  All arrays are fp32 device
+ * buffers shaped like the adapter's factors (A: [r][d_in], B: [d_out][r]), 16-byte
+ * aligned, updated in place.  A_master / B_master hold the fp32 parameters; with an
+ * fp32 handle they may be NULL, and then the table's A / B are the fp32 parameters.
+ */
+typedef struct {
+    float lr;            /* this step's learning rate for this adapter (after any schedule) */
+    float beta1, beta2;  /* in [0, 1) */
+    float eps;           /* > 0 */
+    float weight_decay;  /* decoupled: p <- p (1 - lr weight_decay) */
+    int32_t step;        /* 1-based count of this adapter's updates, for bias correction */
+    float* A_master;
+    float* B_master;
+    float* mA;
+    float* vA;
+    float* mB;
+    float* vB;
+} plora_adamw_state;
+
+/*
+ * One AdamW step for every adapter in one launch (the optimizer update that follows the
+ * backward in LoRA fine-tuning; "LLM+LoRA微调加速技术原理解析", m.youleyou.com, the PEFT
+ * training loop with torch.optim.AdamW).  Per element of A_i and B_i, with g = dA_i / dB_i
+ * from the table (fp32), in fp32:
+ *     p <- p (1 - lr wd);   m <- b1 m + (1 - b1) g;   v <- b2 v + (1 - b2) g^2;
+ *     p <- p - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * then the table's A_i / B_i (the layer's parameters in the handle's dtype) receive p,
+ * rounded to nearest even for bf16.  Adapters are independent: each has its own state.
+ * tab: host plora_adapter[n] (rank, A, B written, dA, dB read); st: host
+ * plora_adamw_state[n].  Errors as for plora_backward (every pointer is checked against
+ * its device allocation before anything is launched).
+ */
+PLORA_API plora_status plora_adamw_step(plora_handle h, int32_t n_adapters, const plora_adapter* tab,
+                                        const plora_adamw_state* st, void* stream);
+
+/*
  * Profiling.  The handle always counts its kernel launches per kernel kind.
  * With profiling enabled, it also brackets every launch with CUDA events on
  * the launching stream and sums each kernel's device time.

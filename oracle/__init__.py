@@ -13,7 +13,9 @@ Pinned by ``tests/test_oracle.py`` against properties the mathematics fixes:
 weight merging (X (W + s A B) as one library matmul), B = 0, rank-1 closed
 forms, packed == each adapter alone, linearity in s, exact central finite
 differences of <dY, Y>, a hand-derived integer example and the segment
-signature.  No function here is "parity unpinned".
+signature.  ``adamw`` (the optimizer step of the LoRA training loop) is pinned by
+torch.optim.AdamW in float64 and by its first-step and zero-gradient closed forms.
+No function here is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -57,6 +59,9 @@ def _load():
                                              pp, i64, _P, i64, _P, ci]
         for fn in ("oracle_forward", "oracle_input_grad", "oracle_weight_grads"):
             getattr(_lib, fn).restype = ctypes.c_int
+        d = ctypes.c_double
+        _lib.oracle_adamw.argtypes = [i64, _P, _P, _P, _P, d, d, d, d, d, ci]
+        _lib.oracle_adamw.restype = None
         _lib.oracle_num_procs.restype = ctypes.c_int
     return _lib
 
@@ -159,6 +164,19 @@ def weight_grads(p, nthreads: int = 1, cols_a: Optional[np.ndarray] = None,
                             ctypes.c_int64(0 if cols_b is None else len(cb)), None if cols_b is None else cb.ctypes.data,
                             ctypes.c_int(nthreads))
     return {"dA": dA, "dB": dB}
+
+
+def adamw(p, m, v, g, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, step=1):
+    """One AdamW step in float64 on copies of p, m, v (any shape); returns (p, m, v)."""
+    lib = _load()
+    p = np.array(p, dtype=np.float64, copy=True, order="C")
+    m = np.array(m, dtype=np.float64, copy=True, order="C")
+    v = np.array(v, dtype=np.float64, copy=True, order="C")
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    assert p.shape == m.shape == v.shape == g.shape
+    lib.oracle_adamw(ctypes.c_int64(p.size), p.ctypes.data, m.ctypes.data, v.ctypes.data, g.ctypes.data,
+                     float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), int(step))
+    return p, m, v
 
 
 def full(p, nthreads: int = 1) -> Dict:

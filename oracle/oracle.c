@@ -228,3 +228,24 @@ int oracle_weight_grads(int dtype, int64_t d_in, int64_t d_out, int32_t n, const
     }
     return 0;
 }
+
+/*
+ * One AdamW step on n elements, in double (TEST INFRASTRUCTURE, like the rest of this file).
+ * The LoRA fine-tuning loop on "LLM+LoRA微调加速技术原理解析" (m.youleyou.com, the PEFT example)
+ * updates the adapters with torch.optim.AdamW; the pages print no formula, so this follows that
+ * optimizer's documented algorithm (Adam with decoupled weight decay), in its order:
+ *   p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+ *   p <- p - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ */
+void oracle_adamw(int64_t n, double* p, double* m, double* v, const double* g, double lr, double beta1,
+                  double beta2, double eps, double weight_decay, int step) {
+    const double bc1 = 1.0 - pow(beta1, (double)step);
+    const double bc2 = 1.0 - pow(beta2, (double)step);
+    for (int64_t e = 0; e < n; ++e) {
+        p[e] = p[e] * (1.0 - lr * weight_decay);
+        m[e] = beta1 * m[e] + (1.0 - beta1) * g[e];
+        v[e] = beta2 * v[e] + (1.0 - beta2) * g[e] * g[e];
+        const double denom = sqrt(v[e]) / sqrt(bc2) + eps;
+        p[e] = p[e] - (lr / bc1) * m[e] / denom;
+    }
+}

@@ -40,7 +40,7 @@ PLORA_STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
-            "plora_grad_B_static")
+            "plora_grad_B_static", "plora_adamw_step")
 
 
 class plora_config(ctypes.Structure):
@@ -52,6 +52,13 @@ class plora_config(ctypes.Structure):
 class plora_adapter(ctypes.Structure):
     _fields_ = [("rank", ctypes.c_int32), ("scale", ctypes.c_float), ("A", ctypes.c_void_p),
                 ("B", ctypes.c_void_p), ("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p)]
+
+
+class plora_adamw_state(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int32),
+                ("A_master", ctypes.c_void_p), ("B_master", ctypes.c_void_p), ("mA", ctypes.c_void_p),
+                ("vA", ctypes.c_void_p), ("mB", ctypes.c_void_p), ("vB", ctypes.c_void_p)]
 
 
 class PloraError(RuntimeError):
@@ -91,6 +98,8 @@ def load(path: str = LIB_PATH):
     lib.plora_profile_enable.restype = ctypes.c_int
     lib.plora_profile_read.argtypes = [H, I32, ctypes.POINTER(I32), P, P, P]
     lib.plora_profile_read.restype = ctypes.c_int
+    lib.plora_adamw_step.argtypes = [H, I32, P, P, P]
+    lib.plora_adamw_step.restype = ctypes.c_int
     lib.plora_grad_B_static.argtypes = [ctypes.POINTER(plora_config), P, I32, P, P, P, P]
     lib.plora_grad_B_static.restype = ctypes.c_int
     lib.plora_version.argtypes = []
@@ -232,6 +241,31 @@ def plora_grad_B_static(cfg: plora_config, dY: int, n: int, off, tab, saved: int
                                           saved, stream))
 
 
+def make_adamw_states(hparams, A_master, B_master, mA, vA, mB, vB):
+    """Host plora_adamw_state[] from per-adapter dicts (lr, beta1, beta2, eps, weight_decay, step) and device
+    pointers (ints; A_master / B_master may be None for an fp32 handle)."""
+    n = len(hparams)
+    st = (plora_adamw_state * max(1, n))()
+    for i, hp in enumerate(hparams):
+        st[i].lr = float(hp["lr"])
+        st[i].beta1 = float(hp.get("beta1", 0.9))
+        st[i].beta2 = float(hp.get("beta2", 0.999))
+        st[i].eps = float(hp.get("eps", 1e-8))
+        st[i].weight_decay = float(hp.get("weight_decay", 0.01))
+        st[i].step = int(hp["step"])
+        st[i].A_master = A_master[i] if A_master is not None else None
+        st[i].B_master = B_master[i] if B_master is not None else None
+        st[i].mA, st[i].vA, st[i].mB, st[i].vB = mA[i], vA[i], mB[i], vB[i]
+    return st
+
+
+def plora_adamw_step(h: int, n: int, tab, states, stream: int = 0, check: bool = True) -> int:
+    s = load().plora_adamw_step(h, n, ctypes.addressof(tab), ctypes.addressof(states), stream)
+    if check:
+        _raise(h, s)
+    return s
+
+
 def plora_version() -> int:
     return int(load().plora_version())
 
@@ -301,3 +335,37 @@ class PackedLoRA:
         plora_backward(self.h, X.data_ptr(), W.data_ptr(), dY.data_ptr(), dX.data_ptr() if want_dX else None,
                        n, off, tab, saved.data_ptr(), st)
         return dX, dA, dB
+
+
+# ---------------------------------------------------------------- autograd
+def packed_lora(engine: "PackedLoRA", X, W, off, scales, A, B):
+    """Y = X W + s_i (X_i A_i) B_i for every packed adapter, differentiable in X, A_i and B_i
+    (W is the frozen base weight and gets no gradient).  A[i] is lora_A.weight ([r_i][d_in]),
+    B[i] is lora_B.weight ([d_out][r_i]), W is nn.Linear.weight ([d_out][d_in]); `off` holds
+    the host segment offsets of the packed rows of X.  The backward runs plora_backward; the
+    fp32 weight gradients are returned in each parameter's dtype."""
+    import torch
+
+    class _PackedLoRAFn(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, X_, W_, *AB):
+            n = len(off) - 1
+            A_, B_ = list(AB[:n]), list(AB[n:])
+            Y, saved = engine.forward(X_.contiguous(), W_.contiguous(), off, scales, A_, B_)
+            ctx.save_for_backward(X_, W_, saved, *AB)
+            return Y
+
+        @staticmethod
+        def backward(ctx, dY):
+            X_, W_, saved, *AB = ctx.saved_tensors
+            n = len(off) - 1
+            A_, B_ = list(AB[:n]), list(AB[n:])
+            dX, dA, dB = engine.backward(X_, W_, dY.contiguous(), off, scales, A_, B_, saved,
+                                         want_dX=ctx.needs_input_grad[0])
+            gA = [g.to(a.dtype) for g, a in zip(dA, A_)]
+            gB = [g.to(b.dtype) for g, b in zip(dB, B_)]
+            return (dX, None, *gA, *gB)
+
+    if W.requires_grad:
+        raise ValueError("packed_lora: the base weight W is frozen; pass W with requires_grad=False")
+    return _PackedLoRAFn.apply(X, W, *A, *B)

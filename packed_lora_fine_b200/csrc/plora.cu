@@ -22,6 +22,7 @@
 #include "simt.cuh"
 #include "tc.cuh"
 #include "tc_pair.cuh"
+#include "adamw.cuh"
 
 using namespace plora;
 
@@ -133,9 +134,9 @@ bool in_device_allocation(const void* p, size_t bytes) {
 
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
-            kSimt, kKinds };
+            kSimt, kAdamw, kKinds };
 const char* const kKindNames[kKinds] = {"pack_a", "pack_bt", "base_fwd", "shrink_x", "expand_y", "base_dx",
-                                        "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm"};
+                                        "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw"};
 
 cudaEvent_t take_event(plora_ctx* h) {
     if (!h->pool.empty()) {
@@ -384,6 +385,27 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     return PLORA_OK;
 }
 
+// Copy two host arrays to the device through the staging ring (same slot discipline as upload()).
+plora_status upload_parts(plora_ctx* h, const void* a, size_t na, const void* b, size_t nb, cudaStream_t st,
+                          uint8_t** da, uint8_t** db, int* slot_out) {
+    const int slot = h->next_slot;
+    h->next_slot = (h->next_slot + 1) % kSlots;
+    cudaError_t e = cudaEventSynchronize(h->ev[slot]);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize(staging slot)");
+    const size_t ob = (size_t)round_up((int64_t)na, 256);
+    const size_t total = ob + nb;
+    if (total > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "optimizer tables exceed the staging size");
+    if (na) memcpy(h->h_blob[slot], a, na);
+    if (nb) memcpy(h->h_blob[slot] + ob, b, nb);
+    uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
+    e = cudaMemcpyAsync(d, h->h_blob[slot], total, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync(optimizer tables)");
+    *da = d;
+    *db = d + ob;
+    *slot_out = slot;
+    return PLORA_OK;
+}
+
 plora_status finish(plora_ctx* h, const DevPlan& D, cudaStream_t st) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
@@ -596,6 +618,11 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
                     (size_t)round_up(ops_max * (int64_t)sizeof(SimtOp), 256) +
                     (size_t)round_up((tok_max + 1) * (int64_t)sizeof(MTileRec), 256) +
                     (size_t)round_up((tok_max + na) * (int64_t)sizeof(LoraSeg), 256) + 1024;
+    // The AdamW step's tables (segments and chunks) travel through the same staging ring.
+    const int64_t adamw_chunks = 2 * na + na * (int64_t)cfg->max_rank * (cfg->d_in + cfg->d_out) / kAdamwChunk;
+    h->blob_bytes = std::max(h->blob_bytes, (size_t)round_up(2 * na * (int64_t)sizeof(AdamwSeg), 256) +
+                                                (size_t)round_up(adamw_chunks * (int64_t)sizeof(AdamwChunk), 256) +
+                                                1024);
 
     size_t o = 0;
     auto carve = [&](Region& r, size_t bytes) {
@@ -974,6 +1001,86 @@ plora_status plora_debug_unpack_saved(plora_handle h, int32_t n, const int64_t* 
                                                                  a.rank, H_out);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PLORA_OK : cuda_fail(h, e, "unpack launch");
+}
+
+plora_status plora_adamw_step(plora_handle h, int32_t n, const plora_adapter* tab, const plora_adamw_state* st,
+                              void* stream) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    if (n < 0 || n > h->cfg.max_adapters)
+        return fail(h, PLORA_ERR_INVALID_ARG, "n_adapters=%d outside [0, max_adapters=%d]", n, h->cfg.max_adapters);
+    if (n == 0) return PLORA_OK;
+    if (!tab || !st) return fail(h, PLORA_ERR_INVALID_ARG, "adapter table or optimizer state is NULL");
+    if (!get_range_fn()) return fail(h, PLORA_ERR_CUDA, "cuMemGetAddressRange is not available");
+    const bool bf16 = h->cfg.dtype == PLORA_BF16;
+    const size_t di = (size_t)h->cfg.d_in, dout = (size_t)h->cfg.d_out;
+    std::vector<AdamwSeg> segs;
+    std::vector<AdamwChunk> chunks;
+    for (int32_t i = 0; i < n; ++i) {
+        const plora_adapter& a = tab[i];
+        const plora_adamw_state& o = st[i];
+        if (a.rank < 1 || a.rank > h->cfg.max_rank)
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: rank %d outside [1, max_rank=%d]", i, a.rank,
+                        h->cfg.max_rank);
+        if (!(o.beta1 >= 0.f && o.beta1 < 1.f) || !(o.beta2 >= 0.f && o.beta2 < 1.f) || !(o.eps > 0.f) ||
+            !std::isfinite(o.eps) || !std::isfinite(o.lr) || !std::isfinite(o.weight_decay) || o.step < 1)
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: invalid AdamW hyper-parameters", i);
+        if (bf16 && (!o.A_master || !o.B_master))
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: a bf16 handle needs fp32 master copies", i);
+        if (!bf16 && (o.A_master || o.B_master))
+            return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: an fp32 handle updates A and B in place", i);
+        const size_t r = (size_t)a.rank;
+        const size_t es = h->esize;
+        float* pA = bf16 ? o.A_master : const_cast<float*>(static_cast<const float*>(a.A));
+        float* pB = bf16 ? o.B_master : const_cast<float*>(static_cast<const float*>(a.B));
+        const void* ptrs[] = {a.A, a.B, a.dA, a.dB, pA, pB, o.mA, o.vA, o.mB, o.vB};
+        const size_t bytes[] = {r * di * es, dout * r * es, r * di * 4, dout * r * 4, r * di * 4, dout * r * 4,
+                                r * di * 4, r * di * 4, dout * r * 4, dout * r * 4};
+        for (int k = 0; k < 10; ++k) {
+            if (!ptrs[k] || !aligned16(ptrs[k]))
+                return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: a parameter, gradient or state pointer is NULL "
+                            "or not 16-byte aligned", i);
+            if (!in_device_allocation(ptrs[k], bytes[k]))
+                return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: a parameter, gradient or state buffer is not a "
+                            "device buffer of its size", i);
+        }
+        const double b1 = o.beta1, b2 = o.beta2;
+        const double bc1 = 1.0 - std::pow(b1, (double)o.step);
+        const double bc2 = 1.0 - std::pow(b2, (double)o.step);
+        AdamwSeg sg{};
+        sg.decay = (float)(1.0 - (double)o.lr * (double)o.weight_decay);
+        sg.step_size = (float)((double)o.lr / bc1);
+        sg.beta1 = o.beta1;
+        sg.beta2 = o.beta2;
+        sg.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
+        sg.eps = o.eps;
+        AdamwSeg sa = sg, sb = sg;
+        sa.p = pA; sa.m = o.mA; sa.v = o.vA; sa.g = a.dA; sa.out = bf16 ? const_cast<void*>(a.A) : nullptr;
+        sa.n = (int64_t)(r * di);
+        sb.p = pB; sb.m = o.mB; sb.v = o.vB; sb.g = a.dB; sb.out = bf16 ? const_cast<void*>(a.B) : nullptr;
+        sb.n = (int64_t)(dout * r);
+        for (const AdamwSeg& x : {sa, sb}) {
+            const int32_t id = (int32_t)segs.size();
+            segs.push_back(x);
+            for (int64_t e = 0; e < x.n; e += kAdamwChunk) chunks.push_back(AdamwChunk{id, 0, e});
+        }
+    }
+    cudaError_t ce = cudaSetDevice(h->device);
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    uint8_t *dsegs = nullptr, *dchunks = nullptr;
+    int slot = 0;
+    plora_status s = upload_parts(h, segs.data(), segs.size() * sizeof(AdamwSeg), chunks.data(),
+                                  chunks.size() * sizeof(AdamwChunk), cs, &dsegs, &dchunks, &slot);
+    if (s != PLORA_OK) return s;
+    const unsigned grid = (unsigned)chunks.size();
+    tracked(h, kAdamw, cs, [&] {
+        adamw_kernel<<<grid, 256, 0, cs>>>(reinterpret_cast<const AdamwSeg*>(dsegs),
+                                           reinterpret_cast<const AdamwChunk*>(dchunks));
+    });
+    DevPlan D;
+    D.slot = slot;
+    return finish(h, D, cs);
 }
 
 plora_status plora_profile_enable(plora_handle h, int32_t enable) {

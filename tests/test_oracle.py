@@ -264,3 +264,46 @@ def test_input_rounding_is_round_to_nearest_even():
     assert back[0] == 1.0 and back[1] == 1.0 and back[2] == 1.0 + 2 ** -6
     assert back[3] == -2.5
     assert abs(back[4] - 3.0e-3) <= 3.0e-3 * 2 ** -8
+
+
+# ----------------------------------------------------------------------------- AdamW step
+ADAMW_CASES = [dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01),
+               dict(lr=3e-2, beta1=0.8, beta2=0.99, eps=1e-6, weight_decay=0.0),
+               dict(lr=5e-4, beta1=0.0, beta2=0.5, eps=1e-3, weight_decay=0.1)]
+
+
+@pytest.mark.parametrize("hp", ADAMW_CASES)
+def test_adamw_matches_torch_adamw_in_float64(hp):
+    """Special case = library routine: torch.optim.AdamW on float64 tensors, several steps."""
+    torch = pytest.importorskip("torch")
+    g = np.random.default_rng(5)
+    p0 = g.standard_normal((7, 13))
+    tp = torch.tensor(p0, dtype=torch.float64, requires_grad=True)
+    opt = torch.optim.AdamW([tp], lr=hp["lr"], betas=(hp["beta1"], hp["beta2"]), eps=hp["eps"],
+                            weight_decay=hp["weight_decay"])
+    p, m, v = p0.copy(), np.zeros_like(p0), np.zeros_like(p0)
+    for t in range(1, 6):
+        grad = g.standard_normal(p0.shape) * (0.1 * t)
+        tp.grad = torch.tensor(grad, dtype=torch.float64)
+        opt.step()
+        p, m, v = oracle.adamw(p, m, v, grad, step=t, **hp)
+        st = opt.state[tp]
+        assert np.max(np.abs(p - tp.detach().numpy())) <= 1e-12 * max(1.0, np.max(np.abs(p)))
+        assert np.max(np.abs(m - st["exp_avg"].numpy())) <= 1e-14
+        assert np.max(np.abs(v - st["exp_avg_sq"].numpy())) <= 1e-14
+
+
+def test_adamw_first_step_closed_form():
+    """From zero moments, step 1: m_hat = g and sqrt(v_hat) = |g|, so p1 = p0 (1 - lr wd) - lr g / (|g| + eps)."""
+    g = np.random.default_rng(6)
+    p0, grad = g.standard_normal(50), g.standard_normal(50)
+    lr, wd, eps = 0.01, 0.05, 1e-4
+    p1, m1, v1 = oracle.adamw(p0, np.zeros(50), np.zeros(50), grad, lr=lr, weight_decay=wd, eps=eps, step=1)
+    assert np.allclose(p1, p0 * (1 - lr * wd) - lr * grad / (np.abs(grad) + eps), rtol=1e-13, atol=1e-15)
+    assert np.allclose(m1, 0.1 * grad, rtol=1e-15) and np.allclose(v1, 0.001 * grad * grad, rtol=1e-12)
+
+
+def test_adamw_zero_gradient_is_pure_decay():
+    p0 = np.random.default_rng(7).standard_normal(40)
+    p1, m1, v1 = oracle.adamw(p0, np.zeros(40), np.zeros(40), np.zeros(40), lr=0.1, weight_decay=0.2, step=3)
+    assert np.array_equal(p1, p0 * (1 - 0.1 * 0.2)) and not np.any(m1) and not np.any(v1)
