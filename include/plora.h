@@ -317,6 +317,16 @@ PLORA_API plora_status plora_grad_B_static(const plora_config* cfg, const void* 
                                            const int64_t* off, const plora_adapter* tab, const void* saved,
                                            void* stream);
 
+/*
+ * Debug / failure detection: launch one CTA whose bounded wait is on a barrier that
+ * nothing ever arrives at, through the same bounded-wait code the kernels use, with a
+ * limit of timeout_ns (1 ms .. 10 s).  The wait runs out, the kernel records
+ * PLORA_ERR_TIMEOUT in the handle's device error flag and returns; the next
+ * plora_check(h, stream) reports PLORA_ERR_TIMEOUT (and clears the flag).  No trap, no
+ * fault, no hang: the context stays usable.
+ */
+PLORA_API plora_status plora_debug_timeout_probe(plora_handle h, int64_t timeout_ns, void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 PLORA_API int32_t plora_version(void);
 

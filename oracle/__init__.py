@@ -45,25 +45,51 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def _lib_setup(lib):
+    i64, i32, ci = ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    pp = ctypes.POINTER(_P)
+    lib.oracle_forward.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, _P, pp, pp, i64, _P, _P, _P, i64, ci]
+    lib.oracle_input_grad.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, pp, pp, _P, i64, _P, _P, _P, i64, ci]
+    lib.oracle_weight_grads.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, pp, pp, _P, pp, pp, i64, _P, i64, _P,
+                                        ci]
+    for fn in ("oracle_forward", "oracle_input_grad", "oracle_weight_grads"):
+        getattr(lib, fn).restype = ctypes.c_int
+    d = ctypes.c_double
+    lib.oracle_adamw.argtypes = [i64, _P, _P, _P, _P, d, d, d, d, d, ci]
+    lib.oracle_adamw.restype = None
+    lib.oracle_num_procs.restype = ctypes.c_int
+
+
 def _load():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
-        i64, i32, ci = ctypes.c_int64, ctypes.c_int32, ctypes.c_int
-        pp = ctypes.POINTER(_P)
-        _lib.oracle_forward.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, _P, pp, pp, i64, _P,
-                                        _P, _P, i64, ci]
-        _lib.oracle_input_grad.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, pp, pp, _P, i64, _P,
-                                           _P, _P, i64, ci]
-        _lib.oracle_weight_grads.argtypes = [ci, i64, i64, i32, _P, _P, _P, _P, pp, pp, _P, pp,
-                                             pp, i64, _P, i64, _P, ci]
-        for fn in ("oracle_forward", "oracle_input_grad", "oracle_weight_grads"):
-            getattr(_lib, fn).restype = ctypes.c_int
-        d = ctypes.c_double
-        _lib.oracle_adamw.argtypes = [i64, _P, _P, _P, _P, d, d, d, d, d, ci]
-        _lib.oracle_adamw.restype = None
-        _lib.oracle_num_procs.restype = ctypes.c_int
+        lib = ctypes.CDLL(build())
+        _lib_setup(lib)
+        _lib = lib
     return _lib
+
+
+class use_library:
+    """Test hook: run the oracle functions on another build of oracle.c (for example a copy with a
+    planted mistake), inside a `with` block."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        _load()
+        self.saved = _lib
+        _lib = None
+        lib = ctypes.CDLL(self.path)
+        _lib_setup(lib)
+        _lib = lib
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
 
 
 def num_procs() -> int:

@@ -40,7 +40,7 @@ PLORA_STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
-            "plora_grad_B_static", "plora_adamw_step")
+            "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe")
 
 
 class plora_config(ctypes.Structure):
@@ -98,6 +98,8 @@ def load(path: str = LIB_PATH):
     lib.plora_profile_enable.restype = ctypes.c_int
     lib.plora_profile_read.argtypes = [H, I32, ctypes.POINTER(I32), P, P, P]
     lib.plora_profile_read.restype = ctypes.c_int
+    lib.plora_debug_timeout_probe.argtypes = [H, I64, P]
+    lib.plora_debug_timeout_probe.restype = ctypes.c_int
     lib.plora_adamw_step.argtypes = [H, I32, P, P, P]
     lib.plora_adamw_step.restype = ctypes.c_int
     lib.plora_grad_B_static.argtypes = [ctypes.POINTER(plora_config), P, I32, P, P, P, P]
@@ -264,6 +266,10 @@ def plora_adamw_step(h: int, n: int, tab, states, stream: int = 0, check: bool =
     if check:
         _raise(h, s)
     return s
+
+
+def plora_debug_timeout_probe(h: int, timeout_ns: int, stream: int = 0) -> int:
+    return int(load().plora_debug_timeout_probe(h, int(timeout_ns), stream))
 
 
 def plora_version() -> int:

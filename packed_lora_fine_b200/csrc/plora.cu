@@ -132,6 +132,20 @@ bool in_device_allocation(const void* p, size_t bytes) {
     return bytes <= size - (a - base);
 }
 
+// A wait that is never satisfied: exercises the bounded-wait timeout path and the error flag.
+__global__ void timeout_probe_kernel(int* err_flag, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns, err_flag);
+    __syncthreads();
+}
+
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
             kSimt, kAdamw, kKinds };
@@ -1081,6 +1095,17 @@ plora_status plora_adamw_step(plora_handle h, int32_t n, const plora_adapter* ta
     DevPlan D;
     D.slot = slot;
     return finish(h, D, cs);
+}
+
+plora_status plora_debug_timeout_probe(plora_handle h, int64_t timeout_ns, void* stream) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    if (timeout_ns < 1000000 || timeout_ns > 10000000000LL)
+        return fail(h, PLORA_ERR_INVALID_ARG, "timeout_ns=%lld outside [1 ms, 10 s]", (long long)timeout_ns);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    timeout_probe_kernel<<<1, 32, 0, st>>>(h->at<int>(h->r_err), (uint64_t)timeout_ns);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PLORA_OK : cuda_fail(h, e, "timeout probe launch");
 }
 
 plora_status plora_profile_enable(plora_handle h, int32_t enable) {
