@@ -80,7 +80,7 @@ def algorithmic_work(p):
     r = p.ranks.astype(np.float64)
     di, do = float(p.d_in), float(p.d_out)
     T = float(p.T)
-    RP = math.ceil(max(p.ranks) / 64) * 64
+    rp16 = np.ceil(r / 16) * 16
     w = {
         "base_fwd": (2 * T * di * do, 2 * (T * di + di * do + T * do)),
         "base_dx": (2 * T * di * do, 2 * (T * do + di * do + T * di)),
@@ -90,8 +90,10 @@ def algorithmic_work(p):
         "expand_dx": (float(np.sum(2 * n * di * r)), float(np.sum(n * (4 * di + 2 * r) + 2 * r * di))),
         "wgrad_b": (float(np.sum(2 * n * do * r)), float(np.sum(n * (2 * do + 2 * r) + 4 * r * do))),
         "wgrad_a": (float(np.sum(2 * n * di * r)), float(np.sum(n * (2 * di + 2 * r) + 4 * r * di))),
-        "pack_a": (0.0, float(np.sum(2 * r * di)) + 2 * len(r) * RP * di),
-        "pack_bt": (0.0, float(np.sum(2 * r * do)) + 2 * len(r) * RP * do),
+        # packs read each factor once and write rows (A, B^T) or columns (B) up to rp16
+        "pack_a": (0.0, float(np.sum(2 * r * di + 2 * rp16 * di))),
+        "pack_b": (0.0, float(np.sum(2 * r * do + 2 * rp16 * do))),
+        "pack_bt": (0.0, float(np.sum(2 * r * do + 2 * rp16 * do))),
     }
     return w
 

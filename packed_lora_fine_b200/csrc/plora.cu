@@ -148,9 +148,10 @@ __global__ void timeout_probe_kernel(int* err_flag, uint64_t limit_ns) {
 
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
-            kSimt, kAdamw, kKinds };
+            kSimt, kAdamw, kPackB, kKinds };
 const char* const kKindNames[kKinds] = {"pack_a", "pack_bt", "base_fwd", "shrink_x", "expand_y", "base_dx",
-                                        "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw"};
+                                        "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw",
+                                        "pack_b"};
 
 cudaEvent_t take_event(plora_ctx* h) {
     if (!h->pool.empty()) {
@@ -552,16 +553,28 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     return p;
 }
 
-plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, cudaStream_t st) {
+// Stages the factors in the layouts the tensor-core operands want: A as [n RP][d_in] (rows
+// padded to RP) always; B either row-padded, [n d_out][RP] (the fused forward's K-major expand
+// operand), or transposed, [n RP][d_out] (the shrink of the backward and the unfused expand).
+enum class BPack { RowPadded, Transposed };
+
+plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, BPack bp, cudaStream_t st) {
     if (P.n == 0) return PLORA_OK;
     __nv_bfloat16* pa = h->at<__nv_bfloat16>(h->r_packA);
     __nv_bfloat16* pb = h->at<__nv_bfloat16>(h->r_packBT);
+    const int64_t grid_cap = (int64_t)h->num_sms * 8;
     const int64_t vecs = (int64_t)P.n * P.RP * (h->cfg.d_in / 8);
-    const int grid_a = (int)std::min<int64_t>(ceil_div(vecs, 256), (int64_t)h->num_sms * 8);
+    const int grid_a = (int)std::min<int64_t>(ceil_div(vecs, 256), grid_cap);
     tracked(h, kPackA, st, [&] { pack_a_kernel<<<grid_a, 256, 0, st>>>(D.ad, P.n, P.RP, h->cfg.d_in, pa); });
+    if (bp == BPack::RowPadded) {
+        int maxr16 = 16; for (const AdapterDev& a : P.ad) maxr16 = std::max(maxr16, a.rp16);
+        const int64_t per_adapter = h->cfg.d_out * (maxr16 / 8);
+        dim3 grid_b((unsigned)std::min<int64_t>(ceil_div(per_adapter, 256), 65535), (unsigned)P.n);
+        tracked(h, kPackB, st, [&] { pack_b_kernel<<<grid_b, 256, 0, st>>>(D.ad, P.RP, (int)h->cfg.d_out, pb); });
+        return PLORA_OK;
+    }
     dim3 gb((unsigned)ceil_div(h->cfg.d_out, 128), (unsigned)P.n);
-    int maxr = 1;
-    for (const AdapterDev& a : P.ad) maxr = std::max(maxr, a.rank);
+    int maxr = 1; for (const AdapterDev& a : P.ad) maxr = std::max(maxr, a.rank);
     const size_t smem_bt = (size_t)128 * (maxr + 2) * sizeof(__nv_bfloat16);
     tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, smem_bt, st>>>(D.ad, P.RP, h->cfg.d_out, pb); });
     return PLORA_OK;
@@ -780,18 +793,22 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     DevPlan D;
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
-    pack_factors(h, P, D, st);
-    CUtensorMap mX, mW, mW128, mPA, mHk, mPB, mPB16;
+    const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
+    pack_factors(h, P, D, fused ? BPack::RowPadded : BPack::Transposed, st);
+    // mPB: the transposed B pack (unfused expand, MN-major); mPBk / mPBk128: the row-padded B
+    // pack (fused expand, K-major; 256 rows for the 1-SM tile, 128 per CTA of an SM pair).
+    CUtensorMap mX, mW, mW128, mPA, mHk, mPB, mPBk, mPBk128;
+    const void* pb = h->at<void>(h->r_packBT);
     bool ok = make_map(&mX, X, d_in, P.T, d_in, 64, kTileM) &&
               make_map(&mW, W, d_in, d_out, d_in, 64, kTileN) &&
               make_map(&mW128, W, d_in, d_out, d_in, 64, kTileM) &&
               make_map(&mPA, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, P.RP) &&
               make_map(&mHk, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
-              make_map(&mPB, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 64) &&
-              make_map(&mPB16, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, 16);
+              (fused ? make_map(&mPBk, pb, P.RP, (uint64_t)P.n * d_out, P.RP, 64, kTileN) &&
+                       make_map(&mPBk128, pb, P.RP, (uint64_t)P.n * d_out, P.RP, 64, kTileM)
+                     : make_map(&mPB, pb, d_out, (uint64_t)P.n * P.RP, d_out, 64, 64));
     if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
-    const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
     // K2: H'_i = s_i X_i A_i per 128-token tile (into the zero-padded blocks of `saved`).
     TcParams q = base_params(h, P, D);
     q.K_total = (int32_t)d_in;
@@ -811,9 +828,9 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     p.fuse = fused ? 1 : 0;
     if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
         pair_params(p, P.T, d_out);
-        launch_pair<Op::BaseFwd>(h, mX, mW128, mHk, mPB16, p, st);
+        launch_pair<Op::BaseFwd>(h, mX, mW128, mHk, fused ? mPBk128 : mW128, p, st);
     } else {
-        launch_tc<Op::BaseFwd>(h, mX, mW, mHk, mPB16, p, st);
+        launch_tc<Op::BaseFwd>(h, mX, mW, mHk, fused ? mPBk : mW, p, st);
     }
     if (!fused) {
         // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
@@ -905,7 +922,7 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     DevPlan D;
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
-    pack_factors(h, P, D, st);
+    pack_factors(h, P, D, BPack::Transposed, st);
     CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_k, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn;
     bool ok = make_map(&mdY_k, dY, d_out, P.T, d_out, 64, kTileM) &&
               make_map(&mdY_mn, dY, d_out, P.T, d_out, 64, 64) &&

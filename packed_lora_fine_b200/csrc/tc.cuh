@@ -12,6 +12,7 @@
 //   ShrinkX    H_i = X_i A_i       (per 128-token tile)   X      K-major          A pack     K-major
 //   ShrinkDy   G_i = s_i dY_i B_i^T                       dY     K-major          B^T pack   K-major
 //   ExpandY    Y_i += s_i H_i B_i                         H      K-major          B^T pack   MN-major
+//              (folded into BaseFwd instead: B row-padded pack, K-major)
 //   ExpandDx   dX_i += G_i A_i^T                          G      K-major          A pack     MN-major
 //   WgradB     dB_i = s_i dY_i^T H_i (sum over tokens)    dY     MN-major         H          MN-major
 //   WgradA     dA_i = X_i^T G_i      (sum over tokens)    X      MN-major         G          MN-major
@@ -308,8 +309,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     // Low-rank branch folded into the same accumulator: for every adapter j whose
                     // tokens overlap this m-tile, K-steps over its rank with A = its H' (or G) rows,
                     // read at the tile's row offset inside j's zero-padded block (rows outside j's
-                    // segment load as zeros), and B = its packed factor (MN-major, 16-row boxes so
-                    // that only the rank's rows are staged).
+                    // segment load as zeros).  B has the base B's major-ness: for Y, rows n0.. of
+                    // j's row-padded B (K-major, one 256 x 64 box); for dX, j's packed A
+                    // (MN-major, 16-row boxes so that only the rank's rows are staged).
                     for (int q = lr.q0; q < lr.q1 && ok; ++q) {
                         const LoraSeg sg = mtile_seg(p, lr, q);
                         for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
@@ -317,14 +319,20 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                             if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
                             uint8_t* sA = smem + stage * stb;
                             uint8_t* sB = sA + kABytes;
-                            ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + 4u * (uint32_t)R * 128u);
+                            const uint32_t lb_bytes = Tr::kBmn ? 4u * (uint32_t)R * 128u : (uint32_t)kTileN * 128u;
+                            ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + lb_bytes);
                             armed |= 1u << stage;
                             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                             ptx::tma_load_2d(sA, &tmA2, &full_bar[stage], kb * kBlockK, sg.h_y);
-                            for (int h = 0; h < 4; ++h)
-                                for (int r16 = 0; r16 < R; r16 += 16)
-                                    ptx::tma_load_2d(sB + h * R * 128 + r16 * 128, &tmB2, &full_bar[stage],
-                                                     ti.n0 + 64 * h, sg.adapter * p.RP + kb * kBlockK + r16);
+                            if constexpr (Tr::kBmn) {
+                                for (int h = 0; h < 4; ++h)
+                                    for (int r16 = 0; r16 < R; r16 += 16)
+                                        ptx::tma_load_2d(sB + h * R * 128 + r16 * 128, &tmB2, &full_bar[stage],
+                                                         ti.n0 + 64 * h, sg.adapter * p.RP + kb * kBlockK + r16);
+                            } else {
+                                ptx::tma_load_2d(sB, &tmB2, &full_bar[stage], kb * kBlockK,
+                                                 sg.adapter * p.N_total + ti.n0);
+                            }
                             if (++stage == nst) { stage = 0; phase ^= 1u; }
                         }
                     }
@@ -371,7 +379,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                     if (++stage == nst) { stage = 0; phase ^= 1u; }
                 }
                 if constexpr (Tr::kBase) {
-                    const uint32_t idesc_lr = ptx::idesc_bf16_f32(kTileM, kTileN, false, true);
+                    const uint32_t idesc_lr = ptx::idesc_bf16_f32(kTileM, kTileN, false, Tr::kBmn);
                     for (int q = lr.q0; q < (ok ? lr.q1 : lr.q0); ++q) {
                         const LoraSeg sg = mtile_seg(p, lr, q);
                         for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
@@ -380,10 +388,12 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
                             ptx::tc_fence_after();
                             const uint32_t sA = ptx::smem_u32(smem + stage * stb);
                             const uint32_t sB = sA + kABytes;
-                            for (int ks = 0; ks < R / 16; ++ks)
-                                ptx::tc_mma_f16(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024),
-                                                ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024),
+                            for (int ks = 0; ks < R / 16; ++ks) {
+                                const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024)
+                                                                : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
+                                ptx::tc_mma_f16(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024), bdesc,
                                                 idesc_lr, 1u);
+                            }
                             ptx::tc_commit(&empty_bar[stage]);
                             if (++stage == nst) { stage = 0; phase ^= 1u; }
                         }
@@ -649,6 +659,38 @@ __global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, 
         if (k < ad[i].rank)
             val = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ad[i].A) + (int64_t)k * d_in)[v];
         reinterpret_cast<uint4*>(packA + rowi * d_in)[v] = val;
+    }
+}
+
+// Row-padded copy of every B for the fused forward (the expand's B operand, K-major like W):
+// packB[(i d_out + c) RP + k] = B_i[c][k] for k < r_i, 0 for r_i <= k < rp16_i; columns at or
+// past rp16_i are never multiplied and stay unwritten.  grid.y = adapter; one thread per 16-byte
+// chunk of the rp16_i columns, so consecutive threads read consecutive bytes of B_i.
+__global__ void __launch_bounds__(256) pack_b_kernel(const AdapterDev* __restrict__ ad, int RP, int d_out,
+                                                     __nv_bfloat16* __restrict__ packB) {
+    const int i = blockIdx.y;
+    const int r = ad[i].rank;
+    const unsigned vc = (unsigned)ad[i].rp16 / 8u;          // chunks per row
+    const unsigned total = (unsigned)d_out * vc;
+    const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(ad[i].B);
+    __nv_bfloat16* dst = packB + (int64_t)i * d_out * RP;
+    for (unsigned e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+        const unsigned c = e / vc;
+        const int ch = (int)(e - c * vc);
+        const __nv_bfloat16* src = B + (int64_t)c * r;
+        uint4 val;
+        if ((r & 7) == 0 && ch * 8 < r) {
+            val = reinterpret_cast<const uint4*>(src)[ch];
+        } else {
+            __nv_bfloat16 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int k = ch * 8 + u;
+                v[u] = k < r ? src[k] : __float2bfloat16_rn(0.f);
+            }
+            val = *reinterpret_cast<const uint4*>(v);
+        }
+        *reinterpret_cast<uint4*>(dst + (int64_t)c * RP + ch * 8) = val;
     }
 }
 

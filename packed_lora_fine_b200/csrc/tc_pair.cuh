@@ -131,7 +131,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     if (++stage == nst) { stage = 0; phase ^= 1u; }
                 }
                 // Folded low-rank branch: A = this CTA's 128 rows of adapter j's zero-padded block,
-                // B = this CTA's 128 columns of j's packed factor (16-row MN-major boxes).
+                // B = this CTA's 128 columns of j's factor, with the base B's major-ness (Y: the
+                // row-padded B, one K-major 128 x 64 box; dX: packed A, 16-row MN-major boxes).
                 for (int q = lr.q0; q < lr.q1 && ok; ++q) {
                     const LoraSeg sg = mtile_seg(p, lr, q);
                     for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
@@ -140,16 +141,21 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         uint8_t* sA = smem + stage * stb;
                         uint8_t* sB = sA + kABytes;
                         if (leader) {
-                            ptx::mbar_arrive_expect_tx(&full_bar[stage], 2u * (a_bytes + 2u * (uint32_t)R * 128u));
+                            const uint32_t lb_bytes = kBmn ? 2u * (uint32_t)R * 128u : (uint32_t)kABytes;
+                            ptx::mbar_arrive_expect_tx(&full_bar[stage], 2u * (a_bytes + lb_bytes));
                             armed |= 1u << stage;
                             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                         }
                         const uint32_t fb = ptx::pair_leader_addr(&full_bar[stage]);
                         ptx::tma_load_2d_pair(sA, &tmA2, fb, kb * kBlockK, sg.h_y + (int)crank * kTileM);
-                        for (int h = 0; h < 2; ++h)
-                            for (int r16 = 0; r16 < R; r16 += 16)
-                                ptx::tma_load_2d_pair(sB + h * R * 128 + r16 * 128, &tmB2, fb, b_col + 64 * h,
-                                                      sg.adapter * p.RP + kb * kBlockK + r16);
+                        if constexpr (kBmn) {
+                            for (int h = 0; h < 2; ++h)
+                                for (int r16 = 0; r16 < R; r16 += 16)
+                                    ptx::tma_load_2d_pair(sB + h * R * 128 + r16 * 128, &tmB2, fb, b_col + 64 * h,
+                                                          sg.adapter * p.RP + kb * kBlockK + r16);
+                        } else {
+                            ptx::tma_load_2d_pair(sB, &tmB2, fb, kb * kBlockK, sg.adapter * p.N_total + b_col);
+                        }
                         if (++stage == nst) { stage = 0; phase ^= 1u; }
                     }
                 }
@@ -172,7 +178,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t aphase = 0;
             bool ok = true;
             const uint32_t idesc = ptx::idesc_bf16_f32(kPairTileM, kTileN, false, kBmn);
-            const uint32_t idesc_lr = ptx::idesc_bf16_f32(kPairTileM, kTileN, false, true);
+            const uint32_t idesc_lr = ptx::idesc_bf16_f32(kPairTileM, kTileN, false, kBmn);
             MTileRec lr_next = rec_of(pair);
             for (int t = pair; t < p.num_tiles && ok; t += npairs) {
                 const MTileRec lr = lr_next;
@@ -202,10 +208,12 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         ptx::tc_fence_after();
                         const uint32_t sA = ptx::smem_u32(smem + stage * stb);
                         const uint32_t sB = sA + kABytes;
-                        for (int ks = 0; ks < R / 16; ++ks)
-                            ptx::tc_mma_f16_pair(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024),
-                                                 ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024),
+                        for (int ks = 0; ks < R / 16; ++ks) {
+                            const uint64_t bdesc = kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024)
+                                                        : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
+                            ptx::tc_mma_f16_pair(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024), bdesc,
                                                  idesc_lr, 1u);
+                        }
                         ptx::tc_commit_pair_both(&empty_bar[stage]);
                         if (++stage == nst) { stage = 0; phase ^= 1u; }
                     }
