@@ -95,6 +95,8 @@ def algorithmic_work(p):
         "pack_b": (0.0, float(np.sum(2 * r * do + 2 * rp16 * do))),
         "pack_bt": (0.0, float(np.sum(2 * r * do + 2 * rp16 * do))),
     }
+    # K7's items share K5's launch
+    w["shrink_dy+wgrad_b"] = (w["shrink_dy"][0] + w["wgrad_b"][0], w["shrink_dy"][1] + w["wgrad_b"][1])
     return w
 
 

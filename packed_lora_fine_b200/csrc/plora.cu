@@ -148,10 +148,10 @@ __global__ void timeout_probe_kernel(int* err_flag, uint64_t limit_ns) {
 
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
-            kSimt, kAdamw, kPackB, kKinds };
+            kSimt, kAdamw, kPackB, kShrinkDyWgradB, kKinds };
 const char* const kKindNames[kKinds] = {"pack_a", "pack_bt", "base_fwd", "shrink_x", "expand_y", "base_dx",
                                         "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw",
-                                        "pack_b"};
+                                        "pack_b", "shrink_dy+wgrad_b"};
 
 cudaEvent_t take_event(plora_ctx* h) {
     if (!h->pool.empty()) {
@@ -466,7 +466,17 @@ void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const C
     constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : OP == Op::BaseDx ? kBaseDx : OP == Op::ShrinkX ? kShrinkX
                        : OP == Op::ShrinkDy ? kShrinkDy : OP == Op::ExpandY ? kExpandY : OP == Op::ExpandDx ? kExpandDx
                        : OP == Op::WgradB ? kWgradB : kWgradA;
-    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p); });
+    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p, p); });
+}
+
+// Two independent ops in one persistent launch: OP's items (operands a, b) then OP2's (a2, b2).
+template <Op OP, Op OP2>
+void launch_tc2(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                const CUtensorMap& b2, const TcParams& p, const TcParams& p2, int kind, cudaStream_t st) {
+    const int total = p.num_tiles + p2.num_tiles;
+    if (total <= 0) return;
+    const int grid = std::min(total, h->num_sms);
+    tracked(h, kind, st, [&] { tc_kernel<OP, OP2><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p, p2); });
 }
 
 // Base GEMMs on SM pairs: a cluster of two CTAs per 256x256 tile, persistent over the pairs that
@@ -529,9 +539,9 @@ void narrow_ring(TcParams& p, int RP) {
     p.stages = std::min(kMaxStages, kRingBytes / p.stage_bytes);
 }
 
-template <Op OP>
+template <Op OP, Op OP2 = OP>
 cudaError_t set_tc_attr() {
-    return cudaFuncSetAttribute(tc_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+    return cudaFuncSetAttribute(tc_kernel<OP, OP2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
 }
 
 TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
@@ -683,6 +693,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
         if (e == cudaSuccess) e = set_tc_attr<Op::ExpandDx>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradB>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradA>();
+        if (e == cudaSuccess) e = (set_tc_attr<Op::ShrinkDy, Op::WgradB>());
         if (e == cudaSuccess) e = pair_setup<Op::BaseFwd>(h->pairs_fwd);
         if (e == cudaSuccess) e = pair_setup<Op::BaseDx>(h->pairs_dx);
         if (e == cudaSuccess)
@@ -944,7 +955,14 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     q.b_box_rows = P.RP;
     q.out = G; q.out_ld = P.RP;
     narrow_ring(q, P.RP);
-    launch_tc<Op::ShrinkDy>(h, mdY_k, mPB_k, mdY_k, mPB_k, q, st);
+    // K7: dB_i = H'_i^T dY_i (a sum over each adapter's tokens) needs neither G nor dX, so its
+    // items share K5's launch and fill the last wave of K5's equal-cost token tiles.
+    TcParams wb = base_params(h, P, D);
+    wb.M_total = (int32_t)d_out;
+    wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
+    wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
+    narrow_ring(wb, P.RP);
+    launch_tc2<Op::ShrinkDy, Op::WgradB>(h, mdY_k, mPB_k, mdY_mn, mH_mn, q, wb, kShrinkDyWgradB, st);
     if (dX) {
         // K4 (+K6): dX = dY W^T; fused, each tile also accumulates G_j A_j^T of every adapter j
         // overlapping it, so dX is written once.
@@ -970,13 +988,7 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
             launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, mG_k, mPA_mn, r, st);
         }
     }
-    // K7: dB_i = H'_i^T dY_i; K8: dA_i = X_i^T G_i (sums over each adapter's tokens).
-    TcParams wb = base_params(h, P, D);
-    wb.M_total = (int32_t)d_out;
-    wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
-    wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
-    narrow_ring(wb, P.RP);
-    launch_tc<Op::WgradB>(h, mdY_mn, mH_mn, mdY_mn, mH_mn, wb, st);
+    // K8: dA_i = X_i^T G_i (a sum over each adapter's tokens).
     TcParams wa = base_params(h, P, D);
     wa.M_total = (int32_t)d_in;
     wa.red_dtiles = (int32_t)ceil_div(d_in, kTileM);
@@ -1333,6 +1345,6 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     p.num_tiles = (int32_t)P.red.size() * dtiles;
     narrow_ring(p, P.RP);
     if (p.num_tiles > 0)
-        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, mdY, mH, p);
+        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, mdY, mH, p, p);
     return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
 }

@@ -214,11 +214,356 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
     return __bfloat1622float2(v);
 }
 
+// Operand-ring position of one role thread, carried across the work items of a launch.
+struct RingPos {
+    int stage;
+    uint32_t phase;
+    __device__ __forceinline__ void advance(int nst) {
+        if (++stage == nst) { stage = 0; phase ^= 1u; }
+    }
+};
+
+// Producer (one thread): TMA loads of every k-block of work item ti into the ring.  Returns
+// false when a wait ran out of time (the error flag is then set).
 template <Op OP>
+__device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& ti, const MTileRec& lr,
+                                             const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                             const CUtensorMap* tmA2, const CUtensorMap* tmB2, uint8_t* smem,
+                                             int stb, int nst, uint64_t* full_bar, uint64_t* empty_bar,
+                                             RingPos& rp, uint32_t& armed, uint32_t& armed_par,
+                                             volatile int* abort_flag, uint64_t lim) {
+    using Tr = OpTraits<OP>;
+    const uint32_t b_bytes = Tr::kBmn ? (uint32_t)ti.nb_boxes * 8192u : (uint32_t)p.b_box_rows * 128u;
+    for (int kb = 0; kb < ti.kblocks; ++kb) {
+        if (!ptx::mbar_wait(&empty_bar[rp.stage], rp.phase ^ 1u, abort_flag, lim, p.err_flag)) return false;
+        uint8_t* sA = smem + rp.stage * stb;
+        uint8_t* sB = sA + kABytes;
+        ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], (uint32_t)kABytes + b_bytes);
+        armed |= 1u << rp.stage;
+        armed_par = (armed_par & ~(1u << rp.stage)) | (rp.phase << rp.stage);
+        if constexpr (Tr::kAmn) {
+            ptx::tma_load_2d(sA, tmA, &full_bar[rp.stage], ti.a_x, ti.a_y + kb * kBlockK);
+            ptx::tma_load_2d(sA + 8192, tmA, &full_bar[rp.stage], ti.a_x + 64, ti.a_y + kb * kBlockK);
+        } else {
+            ptx::tma_load_2d(sA, tmA, &full_bar[rp.stage], ti.a_x + kb * kBlockK, ti.a_y);
+        }
+        if constexpr (Tr::kBmn) {
+            for (int h = 0; h < ti.nb_boxes; ++h)
+                ptx::tma_load_2d(sB + h * 8192, tmB, &full_bar[rp.stage], ti.b_x + 64 * h, ti.b_y + kb * kBlockK);
+        } else {
+            ptx::tma_load_2d(sB, tmB, &full_bar[rp.stage], ti.b_x + kb * kBlockK, ti.b_y);
+        }
+        rp.advance(nst);
+    }
+    if constexpr (Tr::kBase) {
+        // Low-rank branch folded into the same accumulator: for every adapter j whose
+        // tokens overlap this m-tile, K-steps over its rank with A = its H' (or G) rows,
+        // read at the tile's row offset inside j's zero-padded block (rows outside j's
+        // segment load as zeros).  B has the base B's major-ness: for Y, rows n0.. of
+        // j's row-padded B (K-major, one 256 x 64 box); for dX, j's packed A
+        // (MN-major, 16-row boxes so that only the rank's rows are staged).
+        for (int q = lr.q0; q < lr.q1; ++q) {
+            const LoraSeg sg = mtile_seg(p, lr, q);
+            for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
+                const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
+                if (!ptx::mbar_wait(&empty_bar[rp.stage], rp.phase ^ 1u, abort_flag, lim, p.err_flag)) return false;
+                uint8_t* sA = smem + rp.stage * stb;
+                uint8_t* sB = sA + kABytes;
+                const uint32_t lb_bytes = Tr::kBmn ? 4u * (uint32_t)R * 128u : (uint32_t)kTileN * 128u;
+                ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], (uint32_t)kABytes + lb_bytes);
+                armed |= 1u << rp.stage;
+                armed_par = (armed_par & ~(1u << rp.stage)) | (rp.phase << rp.stage);
+                ptx::tma_load_2d(sA, tmA2, &full_bar[rp.stage], kb * kBlockK, sg.h_y);
+                if constexpr (Tr::kBmn) {
+                    for (int h = 0; h < 4; ++h)
+                        for (int r16 = 0; r16 < R; r16 += 16)
+                            ptx::tma_load_2d(sB + h * R * 128 + r16 * 128, tmB2, &full_bar[rp.stage],
+                                             ti.n0 + 64 * h, sg.adapter * p.RP + kb * kBlockK + r16);
+                } else {
+                    ptx::tma_load_2d(sB, tmB2, &full_bar[rp.stage], kb * kBlockK, sg.adapter * p.N_total + ti.n0);
+                }
+                rp.advance(nst);
+            }
+        }
+    }
+    return true;
+}
+
+// MMA issuer (one thread): the tcgen05.mma of every k-block of work item ti into the
+// accumulator at d_tmem, releasing each ring stage as its MMAs complete.
+template <Op OP>
+__device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, const MTileRec& lr, uint8_t* smem,
+                                         int stb, int nst, uint64_t* full_bar, uint64_t* empty_bar,
+                                         uint32_t d_tmem, RingPos& rp, volatile int* abort_flag, uint64_t lim) {
+    using Tr = OpTraits<OP>;
+    const uint32_t idesc = ptx::idesc_bf16_f32(kTileM, ti.mma_n, Tr::kAmn, Tr::kBmn);
+    for (int kb = 0; kb < ti.kblocks; ++kb) {
+        if (!ptx::mbar_wait(&full_bar[rp.stage], rp.phase, abort_flag, lim, p.err_flag)) return false;
+        ptx::tc_fence_after();
+        const uint32_t sA = ptx::smem_u32(smem + rp.stage * stb);
+        const uint32_t sB = sA + kABytes;
+        const int steps = (kb == ti.kblocks - 1) ? ti.last_ksteps : 4;
+        for (int ks = 0; ks < steps; ++ks) {
+            const uint64_t adesc = Tr::kAmn ? ptx::smem_desc_sw128(sA + ks * 2048, 8192, 1024)
+                                            : ptx::smem_desc_sw128(sA + ks * 32, 16, 1024);
+            const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, 8192, 1024)
+                                            : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
+            ptx::tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | ks) ? 1u : 0u);
+        }
+        ptx::tc_commit(&empty_bar[rp.stage]);
+        rp.advance(nst);
+    }
+    if constexpr (Tr::kBase) {
+        const uint32_t idesc_lr = ptx::idesc_bf16_f32(kTileM, kTileN, false, Tr::kBmn);
+        for (int q = lr.q0; q < lr.q1; ++q) {
+            const LoraSeg sg = mtile_seg(p, lr, q);
+            for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
+                const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
+                if (!ptx::mbar_wait(&full_bar[rp.stage], rp.phase, abort_flag, lim, p.err_flag)) return false;
+                ptx::tc_fence_after();
+                const uint32_t sA = ptx::smem_u32(smem + rp.stage * stb);
+                const uint32_t sB = sA + kABytes;
+                for (int ks = 0; ks < R / 16; ++ks) {
+                    const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024)
+                                                    : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
+                    ptx::tc_mma_f16(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024), bdesc, idesc_lr, 1u);
+                }
+                ptx::tc_commit(&empty_bar[rp.stage]);
+                rp.advance(nst);
+            }
+        }
+    }
+    return true;
+}
+
+// Epilogue (warps 2..5, one accumulator row per thread): drains work item ti's accumulator
+// rows from TMEM at t_row and runs the op's output step.
+template <Op OP>
+__device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo& ti, uint32_t t_row, int q, int lane,
+                                              float* epi_stage, int* red_flag) {
+    using Tr = OpTraits<OP>;
+    const int row = q * 32 + lane;          // accumulator row handled by this thread
+    const bool row_ok = row < ti.rows_valid;
+    if constexpr (Tr::kBase) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
+        for (int c = 0; c < kTileN; c += 16) {
+            uint32_t r[16];
+            ptx::tmem_ld16(t_row + c, r);
+            ptx::tmem_ld_wait();
+            if (row_ok) {
+                uint4 v0, v1;
+                v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
+                v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
+                v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
+                v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
+                v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
+                v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
+                v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
+                v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
+                if (c + 8 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c) = v0;
+                if (c + 16 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c + 8) = v1;
+            }
+        }
+    } else if constexpr (Tr::kShrink) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld;
+        for (int c = 0; c < ti.cols_valid; c += 16) {
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+            if (c < ti.mma_n) {
+                uint32_t r[16];
+                ptx::tmem_ld16(t_row + c, r);
+                ptx::tmem_ld_wait();
+                if (row_ok) {
+                    const float s = ti.scale;
+                    v0.x = pack_bf16x2(s * __uint_as_float(r[0]), s * __uint_as_float(r[1]));
+                    v0.y = pack_bf16x2(s * __uint_as_float(r[2]), s * __uint_as_float(r[3]));
+                    v0.z = pack_bf16x2(s * __uint_as_float(r[4]), s * __uint_as_float(r[5]));
+                    v0.w = pack_bf16x2(s * __uint_as_float(r[6]), s * __uint_as_float(r[7]));
+                    v1.x = pack_bf16x2(s * __uint_as_float(r[8]), s * __uint_as_float(r[9]));
+                    v1.y = pack_bf16x2(s * __uint_as_float(r[10]), s * __uint_as_float(r[11]));
+                    v1.z = pack_bf16x2(s * __uint_as_float(r[12]), s * __uint_as_float(r[13]));
+                    v1.w = pack_bf16x2(s * __uint_as_float(r[14]), s * __uint_as_float(r[15]));
+                }
+            }
+            *reinterpret_cast<uint4*>(out + c) = v0;
+            *reinterpret_cast<uint4*>(out + c + 8) = v1;
+        }
+        // The adapter's block has kLoraPad zero rows before and after its (128-rounded) rows, so that
+        // a base tile straddling the segment can read it at any row offset; the first and the last
+        // tile of the adapter write them.
+        const AdapterDev ad = p.adapters[ti.adapter];
+        const bool first = ti.out_row == ad.h_row;
+        const bool last = ti.out_row + kTileM >= ad.h_row + ad.n;
+        if (first || last) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.out);
+            const int tail = ad.h_row + ((ad.n + kTileM - 1) / kTileM) * kTileM;
+            for (int pr = row; pr < kLoraPad; pr += kTileM) {
+                if (first) {
+                    uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(ad.h_row - kLoraPad + pr) * p.out_ld);
+                    for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                }
+                if (last) {
+                    uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(tail + pr) * p.out_ld);
+                    for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
+                }
+            }
+        }
+    } else if constexpr (Tr::kExpand) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
+        const float s = ti.scale;
+        for (int h = 0; h < kTileN; h += 128) {
+            uint4 y[16];
+            if (row_ok) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    if (h + 8 * u + 8 <= ti.cols_valid) y[u] = *reinterpret_cast<const uint4*>(out + h + 8 * u);
+            }
+#pragma unroll
+            for (int u = 0; u < 16; u += 2) {
+                uint32_t r[16];
+                ptx::tmem_ld16(t_row + h + 8 * u, r);
+                ptx::tmem_ld_wait();
+                if (row_ok) {
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        if (h + 8 * (u + w) + 8 > ti.cols_valid) continue;
+                        uint4 o = y[u + w];
+                        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float2 f = unpack_bf16x2(ow[e]);
+                            f.x += s * __uint_as_float(r[8 * w + 2 * e]);
+                            f.y += s * __uint_as_float(r[8 * w + 2 * e + 1]);
+                            ow[e] = pack_bf16x2(f.x, f.y);
+                        }
+                        *reinterpret_cast<uint4*>(out + h + 8 * (u + w)) = o;
+                    }
+                }
+            }
+        }
+    } else {
+        // Weight gradients: row = hidden index (d_out for dB, d_in for dA), column = rank index.
+        const RedEntry re = p.red[ti.red_idx];
+        const AdapterDev ad = p.adapters[ti.adapter];
+        const int rank = ad.rank;
+        const int hid = ti.out_row + row;
+        const float s = ti.scale;
+        if (re.nsplit == 1 && OP == Op::WgradB) {
+            // dB_i's 128-row tile is one contiguous block ([row][rank]); stage 32 x 32 chunks of
+            // this warp's rows in shared memory and store them with consecutive lanes on
+            // consecutive addresses.
+            float* stg = epi_stage + q * kEpiStageFloats;
+            const int row0 = ti.out_row + q * 32;                 // first hidden row of this warp
+            const int nrows = min(32, p.M_total - row0);
+            float* blk = ad.dB + (int64_t)row0 * rank;
+            for (int c0 = 0; c0 < ti.mma_n && c0 < rank; c0 += 32) {
+                uint32_t r[16];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    ptx::tmem_ld16(t_row + c0 + 16 * hh, r);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) stg[lane * 33 + 16 * hh + e] = s * __uint_as_float(r[e]);
+                }
+                __syncwarp();
+                const int ncols = min(32, rank - c0);
+                if (rank <= 32) {
+                    // the whole [nrows][rank] block is contiguous: linear stores
+                    for (int idx = lane; idx < nrows * rank; idx += 32) {
+                        const int rr = idx / rank, cc = idx - rr * rank;
+                        blk[idx] = stg[rr * 33 + cc];
+                    }
+                } else {
+                    for (int rr = 0; rr < nrows; ++rr)
+                        if (lane < ncols) blk[(int64_t)rr * rank + c0 + lane] = stg[rr * 33 + lane];
+                }
+                __syncwarp();
+            }
+        } else if (re.nsplit == 1) {
+            for (int c = 0; c < ti.mma_n; c += 16) {
+                uint32_t r[16];
+                ptx::tmem_ld16(t_row + c, r);
+                ptx::tmem_ld_wait();
+                if (row_ok) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int k = c + e;
+                        if (k < rank) ad.dA[(int64_t)k * p.M_total + hid] = s * __uint_as_float(r[e]);
+                    }
+                }
+            }
+        } else {
+            // Split along the tokens: write this split's partial, the last split of the
+            // tile to arrive sums all partials in split order (deterministic) and stores.
+            const int64_t slot_elems = (int64_t)kTileM * p.RP;
+            // partial layout [slot][d-tile][rank column][128 rows]: a warp's lanes touch
+            // consecutive rows, so both the writes here and the reduction below coalesce.
+            float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems + row;
+            for (int c = 0; c < ti.mma_n; c += 16) {
+                uint32_t r[16];
+                ptx::tmem_ld16(t_row + c, r);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (c + e < rank) mine[(int64_t)(c + e) * kTileM] = __uint_as_float(r[e]);
+            }
+            __threadfence();
+            ptx::named_bar_sync(1, 128);
+            if (threadIdx.x == 64) {
+                const int old = atomicAdd(&p.counters[re.counter + ti.n0], 1);
+                *red_flag = (old == re.nsplit - 1) ? 1 : 0;
+            }
+            ptx::named_bar_sync(1, 128);
+            if (*red_flag) {
+                __threadfence();
+                if (row_ok) {
+                    const float* first = p.partials + ((int64_t)re.slot * p.red_dtiles + ti.n0) * slot_elems + row;
+                    const int64_t split_stride = (int64_t)p.red_dtiles * slot_elems;
+                    for (int k0 = 0; k0 < rank; k0 += 8) {
+                        // 8 ranks at a time: all of a split's loads are in flight together,
+                        // the sum still runs over the splits in order.
+                        float acc[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+                        for (int sp = 0; sp < re.nsplit; ++sp) {
+                            float v[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                v[u] = (k0 + u < rank) ? __ldcg(first + sp * split_stride + (int64_t)(k0 + u) * kTileM) : 0.f;
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) acc[u] += v[u];
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int k = k0 + u;
+                            if (k < rank) {
+                                if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = s * acc[u];
+                                else ad.dA[(int64_t)k * p.M_total + hid] = s * acc[u];
+                            }
+                        }
+                    }
+                }
+                if (threadIdx.x == 64) p.counters[re.counter + ti.n0] = 0;
+            }
+            ptx::named_bar_sync(1, 128);
+        }
+    }
+}
+
+// One persistent launch runs the work items of OP (p.num_tiles of them) followed, when OP2
+// differs from OP, by those of OP2 (p2.num_tiles, with operands from tmA2 / tmB2).  Both ops
+// use the ring layout of p (stages, stage_bytes).  Items are dealt round-robin over the CTAs,
+// so the second op's items fill the last, partial wave of the first op's.
+template <Op OP, Op OP2 = OP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const TcParams p,
+          const TcParams p2) {
     using Tr = OpTraits<OP>;
+    constexpr bool kDual = OP2 != OP;
+    static_assert(!kDual || (!Tr::kBase && !OpTraits<OP2>::kBase),
+                  "a base GEMM reads its low-rank branch through tmA2 / tmB2");
+    const int total = p.num_tiles + (kDual ? p2.num_tiles : 0);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
@@ -253,7 +598,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     if (warp == 0 && lane == 0) {
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
-        if (Tr::kBase && p.fuse) {
+        if ((Tr::kBase && p.fuse) || kDual) {
             ptx::tma_prefetch_desc(&tmA2);
             ptx::tma_prefetch_desc(&tmB2);
         }
@@ -271,72 +616,20 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
+            RingPos rp{0, 0u};
             uint32_t armed = 0, armed_par = 0;
             bool ok = true;
+            // The folded low-rank record of a base tile is fetched one tile ahead.
             MTileRec lr_next = load_mtile<OP>(p, blockIdx.x);
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = decode_tile<OP>(p, t);
-                const uint32_t b_bytes = Tr::kBmn ? (uint32_t)ti.nb_boxes * 8192u
-                                                  : (uint32_t)p.b_box_rows * 128u;
-                // Folded low-rank branch: this tile's record was fetched one tile ahead.
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const MTileRec lr = lr_next;
                 lr_next = load_mtile<OP>(p, t + gridDim.x);
-                for (int kb = 0; kb < ti.kblocks; ++kb) {
-                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
-                    uint8_t* sA = smem + stage * stb;
-                    uint8_t* sB = sA + kABytes;
-                    ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + b_bytes);
-                    armed |= 1u << stage;
-                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                    if constexpr (Tr::kAmn) {
-                        ptx::tma_load_2d(sA, &tmA, &full_bar[stage], ti.a_x, ti.a_y + kb * kBlockK);
-                        ptx::tma_load_2d(sA + 8192, &tmA, &full_bar[stage], ti.a_x + 64, ti.a_y + kb * kBlockK);
-                    } else {
-                        ptx::tma_load_2d(sA, &tmA, &full_bar[stage], ti.a_x + kb * kBlockK, ti.a_y);
-                    }
-                    if constexpr (Tr::kBmn) {
-                        for (int h = 0; h < ti.nb_boxes; ++h)
-                            ptx::tma_load_2d(sB + h * 8192, &tmB, &full_bar[stage], ti.b_x + 64 * h,
-                                             ti.b_y + kb * kBlockK);
-                    } else {
-                        ptx::tma_load_2d(sB, &tmB, &full_bar[stage], ti.b_x + kb * kBlockK, ti.b_y);
-                    }
-                    if (++stage == nst) { stage = 0; phase ^= 1u; }
-                }
-                if constexpr (Tr::kBase) {
-                    // Low-rank branch folded into the same accumulator: for every adapter j whose
-                    // tokens overlap this m-tile, K-steps over its rank with A = its H' (or G) rows,
-                    // read at the tile's row offset inside j's zero-padded block (rows outside j's
-                    // segment load as zeros).  B has the base B's major-ness: for Y, rows n0.. of
-                    // j's row-padded B (K-major, one 256 x 64 box); for dX, j's packed A
-                    // (MN-major, 16-row boxes so that only the rank's rows are staged).
-                    for (int q = lr.q0; q < lr.q1 && ok; ++q) {
-                        const LoraSeg sg = mtile_seg(p, lr, q);
-                        for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
-                            const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
-                            if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
-                            uint8_t* sA = smem + stage * stb;
-                            uint8_t* sB = sA + kABytes;
-                            const uint32_t lb_bytes = Tr::kBmn ? 4u * (uint32_t)R * 128u : (uint32_t)kTileN * 128u;
-                            ptx::mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)kABytes + lb_bytes);
-                            armed |= 1u << stage;
-                            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                            ptx::tma_load_2d(sA, &tmA2, &full_bar[stage], kb * kBlockK, sg.h_y);
-                            if constexpr (Tr::kBmn) {
-                                for (int h = 0; h < 4; ++h)
-                                    for (int r16 = 0; r16 < R; r16 += 16)
-                                        ptx::tma_load_2d(sB + h * R * 128 + r16 * 128, &tmB2, &full_bar[stage],
-                                                         ti.n0 + 64 * h, sg.adapter * p.RP + kb * kBlockK + r16);
-                            } else {
-                                ptx::tma_load_2d(sB, &tmB2, &full_bar[stage], kb * kBlockK,
-                                                 sg.adapter * p.N_total + ti.n0);
-                            }
-                            if (++stage == nst) { stage = 0; phase ^= 1u; }
-                        }
-                    }
-                }
+                if (kDual && t >= p.num_tiles)
+                    ok = produce_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), lr, &tmA2, &tmB2, &tmA2, &tmB2,
+                                           smem, stb, nst, full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
+                else
+                    ok = produce_item<OP>(p, decode_tile<OP>(p, t), lr, &tmA, &tmB, &tmA2, &tmB2, smem, stb, nst,
+                                          full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
             }
             // Drain: every load this thread issued must have landed before the CTA exits.
             for (int s = 0; s < nst; ++s)
@@ -348,58 +641,21 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
+            RingPos rp{0, 0u};
             int abuf = 0;
             uint32_t aphase = 0;
-            bool ok = true;
             MTileRec lr_next = load_mtile<OP>(p, blockIdx.x);
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-                const TileInfo ti = decode_tile<OP>(p, t);
-                const uint32_t idesc = ptx::idesc_bf16_f32(kTileM, ti.mma_n, Tr::kAmn, Tr::kBmn);
+            for (int t = blockIdx.x; t < total; t += gridDim.x) {
                 const MTileRec lr = lr_next;
                 lr_next = load_mtile<OP>(p, t + gridDim.x);
-                if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p.err_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p.err_flag)) break;
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
-                for (int kb = 0; kb < ti.kblocks; ++kb) {
-                    if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, lim, p.err_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t sA = ptx::smem_u32(smem + stage * stb);
-                    const uint32_t sB = sA + kABytes;
-                    const int steps = (kb == ti.kblocks - 1) ? ti.last_ksteps : 4;
-                    for (int ks = 0; ks < steps; ++ks) {
-                        const uint64_t adesc = Tr::kAmn ? ptx::smem_desc_sw128(sA + ks * 2048, 8192, 1024)
-                                                        : ptx::smem_desc_sw128(sA + ks * 32, 16, 1024);
-                        const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, 8192, 1024)
-                                                        : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
-                        ptx::tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | ks) ? 1u : 0u);
-                    }
-                    ptx::tc_commit(&empty_bar[stage]);
-                    if (++stage == nst) { stage = 0; phase ^= 1u; }
-                }
-                if constexpr (Tr::kBase) {
-                    const uint32_t idesc_lr = ptx::idesc_bf16_f32(kTileM, kTileN, false, Tr::kBmn);
-                    for (int q = lr.q0; q < (ok ? lr.q1 : lr.q0); ++q) {
-                        const LoraSeg sg = mtile_seg(p, lr, q);
-                        for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
-                            const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
-                            if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag, lim, p.err_flag)) { ok = false; break; }
-                            ptx::tc_fence_after();
-                            const uint32_t sA = ptx::smem_u32(smem + stage * stb);
-                            const uint32_t sB = sA + kABytes;
-                            for (int ks = 0; ks < R / 16; ++ks) {
-                                const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024)
-                                                                : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
-                                ptx::tc_mma_f16(d_tmem, ptx::smem_desc_sw128(sA + ks * 32, 16, 1024), bdesc,
-                                                idesc_lr, 1u);
-                            }
-                            ptx::tc_commit(&empty_bar[stage]);
-                            if (++stage == nst) { stage = 0; phase ^= 1u; }
-                        }
-                        if (!ok) break;
-                    }
-                }
+                const bool ok = (kDual && t >= p.num_tiles)
+                    ? mma_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), lr, smem, stb, nst, full_bar,
+                                    empty_bar, d_tmem, rp, abort_flag, lim)
+                    : mma_item<OP>(p, decode_tile<OP>(p, t), lr, smem, stb, nst, full_bar, empty_bar, d_tmem, rp,
+                                   abort_flag, lim);
                 if (!ok) break;
                 ptx::tc_commit(&accf_bar[abuf]);
                 if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
@@ -412,220 +668,16 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
-        const int row = q * 32 + lane;          // accumulator row handled by this thread
         int abuf = 0;
         uint32_t aphase = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-            const TileInfo ti = decode_tile<OP>(p, t);
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
             if (!ptx::mbar_wait(&accf_bar[abuf], aphase, abort_flag, lim, p.err_flag)) break;
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
-            const bool row_ok = row < ti.rows_valid;
-
-            if constexpr (Tr::kBase) {
-                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
-                for (int c = 0; c < kTileN; c += 16) {
-                    uint32_t r[16];
-                    ptx::tmem_ld16(t_row + c, r);
-                    ptx::tmem_ld_wait();
-                    if (row_ok) {
-                        uint4 v0, v1;
-                        v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                        v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                        v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                        v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                        v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                        v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                        v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                        v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                        if (c + 8 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c) = v0;
-                        if (c + 16 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c + 8) = v1;
-                    }
-                }
-            } else if constexpr (Tr::kShrink) {
-                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld;
-                for (int c = 0; c < ti.cols_valid; c += 16) {
-                    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-                    if (c < ti.mma_n) {
-                        uint32_t r[16];
-                        ptx::tmem_ld16(t_row + c, r);
-                        ptx::tmem_ld_wait();
-                        if (row_ok) {
-                            const float s = ti.scale;
-                            v0.x = pack_bf16x2(s * __uint_as_float(r[0]), s * __uint_as_float(r[1]));
-                            v0.y = pack_bf16x2(s * __uint_as_float(r[2]), s * __uint_as_float(r[3]));
-                            v0.z = pack_bf16x2(s * __uint_as_float(r[4]), s * __uint_as_float(r[5]));
-                            v0.w = pack_bf16x2(s * __uint_as_float(r[6]), s * __uint_as_float(r[7]));
-                            v1.x = pack_bf16x2(s * __uint_as_float(r[8]), s * __uint_as_float(r[9]));
-                            v1.y = pack_bf16x2(s * __uint_as_float(r[10]), s * __uint_as_float(r[11]));
-                            v1.z = pack_bf16x2(s * __uint_as_float(r[12]), s * __uint_as_float(r[13]));
-                            v1.w = pack_bf16x2(s * __uint_as_float(r[14]), s * __uint_as_float(r[15]));
-                        }
-                    }
-                    *reinterpret_cast<uint4*>(out + c) = v0;
-                    *reinterpret_cast<uint4*>(out + c + 8) = v1;
-                }
-                // The adapter's block has kLoraPad zero rows before and after its (128-rounded) rows, so that
-                // a base tile straddling the segment can read it at any row offset; the first and the last
-                // tile of the adapter write them.
-                const AdapterDev ad = p.adapters[ti.adapter];
-                const bool first = ti.out_row == ad.h_row;
-                const bool last = ti.out_row + kTileM >= ad.h_row + ad.n;
-                if (first || last) {
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.out);
-                    const int tail = ad.h_row + ((ad.n + kTileM - 1) / kTileM) * kTileM;
-                    for (int pr = row; pr < kLoraPad; pr += kTileM) {
-                        if (first) {
-                            uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(ad.h_row - kLoraPad + pr) * p.out_ld);
-                            for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
-                        }
-                        if (last) {
-                            uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(tail + pr) * p.out_ld);
-                            for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
-                        }
-                    }
-                }
-            } else if constexpr (Tr::kExpand) {
-                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
-                const float s = ti.scale;
-                for (int h = 0; h < kTileN; h += 128) {
-                    uint4 y[16];
-                    if (row_ok) {
-#pragma unroll
-                        for (int u = 0; u < 16; ++u)
-                            if (h + 8 * u + 8 <= ti.cols_valid) y[u] = *reinterpret_cast<const uint4*>(out + h + 8 * u);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        uint32_t r[16];
-                        ptx::tmem_ld16(t_row + h + 8 * u, r);
-                        ptx::tmem_ld_wait();
-                        if (row_ok) {
-#pragma unroll
-                            for (int w = 0; w < 2; ++w) {
-                                if (h + 8 * (u + w) + 8 > ti.cols_valid) continue;
-                                uint4 o = y[u + w];
-                                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    float2 f = unpack_bf16x2(ow[e]);
-                                    f.x += s * __uint_as_float(r[8 * w + 2 * e]);
-                                    f.y += s * __uint_as_float(r[8 * w + 2 * e + 1]);
-                                    ow[e] = pack_bf16x2(f.x, f.y);
-                                }
-                                *reinterpret_cast<uint4*>(out + h + 8 * (u + w)) = o;
-                            }
-                        }
-                    }
-                }
-            } else {
-                // Weight gradients: row = hidden index (d_out for dB, d_in for dA), column = rank index.
-                const RedEntry re = p.red[ti.red_idx];
-                const AdapterDev ad = p.adapters[ti.adapter];
-                const int rank = ad.rank;
-                const int hid = ti.out_row + row;
-                const float s = ti.scale;
-                if (re.nsplit == 1 && OP == Op::WgradB) {
-                    // dB_i's 128-row tile is one contiguous block ([row][rank]); stage 32 x 32 chunks of
-                    // this warp's rows in shared memory and store them with consecutive lanes on
-                    // consecutive addresses.
-                    float* stg = epi_stage + q * kEpiStageFloats;
-                    const int row0 = ti.out_row + q * 32;                 // first hidden row of this warp
-                    const int nrows = min(32, p.M_total - row0);
-                    float* blk = ad.dB + (int64_t)row0 * rank;
-                    for (int c0 = 0; c0 < ti.mma_n && c0 < rank; c0 += 32) {
-                        uint32_t r[16];
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            ptx::tmem_ld16(t_row + c0 + 16 * hh, r);
-                            ptx::tmem_ld_wait();
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) stg[lane * 33 + 16 * hh + e] = s * __uint_as_float(r[e]);
-                        }
-                        __syncwarp();
-                        const int ncols = min(32, rank - c0);
-                        if (rank <= 32) {
-                            // the whole [nrows][rank] block is contiguous: linear stores
-                            for (int idx = lane; idx < nrows * rank; idx += 32) {
-                                const int rr = idx / rank, cc = idx - rr * rank;
-                                blk[idx] = stg[rr * 33 + cc];
-                            }
-                        } else {
-                            for (int rr = 0; rr < nrows; ++rr)
-                                if (lane < ncols) blk[(int64_t)rr * rank + c0 + lane] = stg[rr * 33 + lane];
-                        }
-                        __syncwarp();
-                    }
-                } else if (re.nsplit == 1) {
-                    for (int c = 0; c < ti.mma_n; c += 16) {
-                        uint32_t r[16];
-                        ptx::tmem_ld16(t_row + c, r);
-                        ptx::tmem_ld_wait();
-                        if (row_ok) {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const int k = c + e;
-                                if (k < rank) ad.dA[(int64_t)k * p.M_total + hid] = s * __uint_as_float(r[e]);
-                            }
-                        }
-                    }
-                } else {
-                    // Split along the tokens: write this split's partial, the last split of the
-                    // tile to arrive sums all partials in split order (deterministic) and stores.
-                    const int64_t slot_elems = (int64_t)kTileM * p.RP;
-                    // partial layout [slot][d-tile][rank column][128 rows]: a warp's lanes touch
-                    // consecutive rows, so both the writes here and the reduction below coalesce.
-                    float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems + row;
-                    for (int c = 0; c < ti.mma_n; c += 16) {
-                        uint32_t r[16];
-                        ptx::tmem_ld16(t_row + c, r);
-                        ptx::tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (c + e < rank) mine[(int64_t)(c + e) * kTileM] = __uint_as_float(r[e]);
-                    }
-                    __threadfence();
-                    ptx::named_bar_sync(1, 128);
-                    if (threadIdx.x == 64) {
-                        const int old = atomicAdd(&p.counters[re.counter + ti.n0], 1);
-                        *red_flag = (old == re.nsplit - 1) ? 1 : 0;
-                    }
-                    ptx::named_bar_sync(1, 128);
-                    if (*red_flag) {
-                        __threadfence();
-                        if (row_ok) {
-                            const float* first = p.partials + ((int64_t)re.slot * p.red_dtiles + ti.n0) * slot_elems + row;
-                            const int64_t split_stride = (int64_t)p.red_dtiles * slot_elems;
-                            for (int k0 = 0; k0 < rank; k0 += 8) {
-                                // 8 ranks at a time: all of a split's loads are in flight together,
-                                // the sum still runs over the splits in order.
-                                float acc[8];
-#pragma unroll
-                                for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-                                for (int sp = 0; sp < re.nsplit; ++sp) {
-                                    float v[8];
-#pragma unroll
-                                    for (int u = 0; u < 8; ++u)
-                                        v[u] = (k0 + u < rank) ? __ldcg(first + sp * split_stride + (int64_t)(k0 + u) * kTileM) : 0.f;
-#pragma unroll
-                                    for (int u = 0; u < 8; ++u) acc[u] += v[u];
-                                }
-#pragma unroll
-                                for (int u = 0; u < 8; ++u) {
-                                    const int k = k0 + u;
-                                    if (k < rank) {
-                                        if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = s * acc[u];
-                                        else ad.dA[(int64_t)k * p.M_total + hid] = s * acc[u];
-                                    }
-                                }
-                            }
-                        }
-                        if (threadIdx.x == 64) p.counters[re.counter + ti.n0] = 0;
-                    }
-                    ptx::named_bar_sync(1, 128);
-                }
-            }
+            if (kDual && t >= p.num_tiles)
+                epilogue_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), t_row, q, lane, epi_stage, red_flag);
+            else
+                epilogue_item<OP>(p, decode_tile<OP>(p, t), t_row, q, lane, epi_stage, red_flag);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
