@@ -100,6 +100,38 @@ def algorithmic_work(p):
     return w
 
 
+class EnergyMeter:
+    """The GPU's cumulative energy counter (NVML, millijoules), read around the timed region."""
+
+    def __init__(self, gpu_uuid: str):
+        self.h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+        except Exception:
+            self.h = None
+
+    def read_mj(self):
+        if self.h is None:
+            return None
+        try:
+            return float(self.nvml.nvmlDeviceGetTotalEnergyConsumption(self.h))
+        except Exception:
+            return None
+
+    def start(self):
+        self.e0, self.t0 = self.read_mj(), time.time()
+
+    def stop(self):
+        e1, t1 = self.read_mj(), time.time()
+        if self.e0 is None or e1 is None:
+            return None, None
+        joules = (e1 - self.e0) / 1e3
+        return joules, joules / max(t1 - self.t0, 1e-9)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason sampling during the timed region."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -285,6 +317,9 @@ def main(argv=None):
     dB = [torch.empty(b.shape, dtype=torch.float32, device=dev) for b in B]
     eng = pl.PackedLoRA(p.d_in, p.d_out, "bf16", max_adapters=p.n_adapters, max_rank=int(max(p.ranks)),
                         max_tokens=T, unfused=args.unfused, base_pair=args.base_pair)
+    dev_info = pl.plora_device_info(eng.h)
+    base_gemm = ("SM-pair 256x256 tiles, %d co-resident pairs of %d SMs" % (dev_info["pairs_fwd"], dev_info["sms"])
+                 if args.base_pair else "1-SM 128x256 tiles on %d SMs" % dev_info["sms"])
     tab_f = eng.table(p.scales, A, B)
     tab_b = eng.table(p.scales, A, B, dA, dB)
     saved = torch.empty(eng.saved_bytes(p.off, tab_f), dtype=torch.uint8, device=dev)
@@ -316,13 +351,16 @@ def main(argv=None):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    energy = EnergyMeter(gpu_uuid)
     clocks.start()
     time.sleep(0.3)
+    energy.start()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
+    joules, watts = energy.stop()
     barrier()
     clk = clocks.stop()
     ms_local = ev0.elapsed_time(ev1) / args.steps
@@ -331,6 +369,12 @@ def main(argv=None):
     assert pl.plora_check(eng.h, st) == pl.PLORA_OK
     ms = reduce_max(ms_local, dist)
     tokens_all = reduce_sum(T, dist)
+    # every rank takes part in both sums; a rank without an energy counter turns them into NaN
+    j_all = reduce_sum(joules if joules is not None else float("nan"), dist)
+    w_all = reduce_sum(watts if watts is not None else float("nan"), dist)
+    energy_line = None if math.isnan(j_all) else {
+        "joules_per_step": j_all / args.steps, "watts_per_gpu": w_all / world,
+        "source": "NVML total-energy counter read around the timed region, summed over ranks"}
     value = tokens_all / (ms / 1000.0)
 
     # Per-kernel roofline (device time from events bracketing each launch on its stream).
@@ -445,10 +489,11 @@ def main(argv=None):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": WORKLOAD, "adapters": n, "tokens_per_gpu": T, "global_tokens": int(tokens_all),
                            "d_in": p.d_in, "d_out": p.d_out, "parallelism": f"adapter-sharded x{world}",
-                           "l2": "inputs larger than L2 (X 452 MB, dY 1.6 GB); no flush"},
+                           "l2": "inputs larger than L2 (X 452 MB, dY 1.6 GB); no flush",
+                           "base_gemm": base_gemm},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
                 "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
-                "kernels": kernels}
+                "energy": energy_line, "kernels": kernels}
         print(json.dumps(line), flush=True)
     eng.close()
     if dist is not None:

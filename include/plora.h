@@ -261,6 +261,14 @@ PLORA_API plora_status plora_adamw_step(plora_handle h, int32_t n_adapters, cons
                                         const plora_adamw_state* st, void* stream);
 
 /*
+ * Launch geometry of the handle's device (a diagnostic; the method itself has no such
+ * call): out[0] = SMs, out[1] / out[2] = the 2-SM clusters that can be resident at once
+ * for the SM-pair Y / dX base GEMMs (PLORA_FLAG_BASE_PAIR), each <= SMs / 2.  At most
+ * `capacity` values are written; *count receives 3.
+ */
+PLORA_API plora_status plora_device_info(plora_handle h, int32_t* out, int32_t capacity, int32_t* count);
+
+/*
  * Profiling.  The handle always counts its kernel launches per kernel kind.
  * With profiling enabled, it also brackets every launch with CUDA events on
  * the launching stream and sums each kernel's device time.

@@ -40,7 +40,7 @@ PLORA_STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
-            "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe")
+            "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe", "plora_device_info")
 
 
 class plora_config(ctypes.Structure):
@@ -98,6 +98,8 @@ def load(path: str = LIB_PATH):
     lib.plora_profile_enable.restype = ctypes.c_int
     lib.plora_profile_read.argtypes = [H, I32, ctypes.POINTER(I32), P, P, P]
     lib.plora_profile_read.restype = ctypes.c_int
+    lib.plora_device_info.argtypes = [H, P, I32, ctypes.POINTER(I32)]
+    lib.plora_device_info.restype = ctypes.c_int
     lib.plora_debug_timeout_probe.argtypes = [H, I64, P]
     lib.plora_debug_timeout_probe.restype = ctypes.c_int
     lib.plora_adamw_step.argtypes = [H, I32, P, P, P]
@@ -234,6 +236,14 @@ def plora_profile_read(h: int) -> dict:
     ms = (ctypes.c_double * cap)()
     _raise(h, lib.plora_profile_read(h, cap, ctypes.byref(n), names, launches, ms))
     return {names[k].decode(): (int(launches[k]), float(ms[k])) for k in range(min(n.value, cap))}
+
+
+def plora_device_info(h: int) -> dict:
+    """SMs of the handle's device and the co-resident 2-SM clusters of the pair base GEMMs."""
+    out = (ctypes.c_int32 * 3)()
+    cnt = ctypes.c_int32(0)
+    _raise(h, load().plora_device_info(h, ctypes.cast(out, ctypes.c_void_p), 3, ctypes.byref(cnt)))
+    return {"sms": int(out[0]), "pairs_fwd": int(out[1]), "pairs_dx": int(out[2])}
 
 
 def plora_grad_B_static(cfg: plora_config, dY: int, n: int, off, tab, saved: int, stream: int = 0) -> int:

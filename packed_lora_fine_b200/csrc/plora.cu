@@ -998,6 +998,14 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     return finish(h, D, st);
 }
 
+plora_status plora_device_info(plora_handle h, int32_t* out, int32_t capacity, int32_t* count) {
+    if (!h || !count || capacity < 0 || (capacity > 0 && !out)) return PLORA_ERR_INVALID_ARG;
+    const int32_t v[3] = {h->num_sms, h->pairs_fwd, h->pairs_dx};
+    for (int32_t i = 0; i < 3 && i < capacity; ++i) out[i] = v[i];
+    *count = 3;
+    return PLORA_OK;
+}
+
 plora_status plora_check(plora_handle h, void* stream) {
     if (!h) return PLORA_ERR_INVALID_ARG;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -69,6 +69,17 @@ def test_create_without_gpu_fails_loudly():
     assert s == pl.PLORA_ERR_CUDA and not h
 
 
+def test_null_handle_calls_are_rejected():
+    import ctypes
+    lib = pl.load()
+    out = (ctypes.c_int32 * 3)()
+    cnt = ctypes.c_int32(-1)
+    assert lib.plora_device_info(None, ctypes.cast(out, ctypes.c_void_p), 3, ctypes.byref(cnt)) == pl.PLORA_ERR_INVALID_ARG
+    assert cnt.value == -1
+    assert lib.plora_profile_enable(None, 1) == pl.PLORA_ERR_INVALID_ARG
+    assert lib.plora_check(None, None) == pl.PLORA_ERR_INVALID_ARG
+
+
 def fake_table(ranks, aligned=True, grads=True):
     base = 0x7f0000000000
     n = len(ranks)

@@ -30,7 +30,10 @@ def _worker(rank, world, port, q):
     got_max = bench.reduce_max(ms, dist)
     got_sum = bench.reduce_sum(tokens, dist)
     ranks, counts, _ = wl.config3_shape(1003 + 1000 * rank)
-    q.put((rank, got_max, got_sum, int(counts.sum())))
+    # energy: a rank without a counter reports NaN and the whole-job sum is then NaN on every rank
+    e_ok = bench.reduce_sum([4.0, 6.0][rank], dist)
+    e_missing = bench.reduce_sum([float("nan"), 6.0][rank], dist)
+    q.put((rank, got_max, got_sum, int(counts.sum()), e_ok, e_missing != e_missing))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -47,8 +50,9 @@ def test_two_rank_reductions_gloo():
         p.join(timeout=120)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
-    for rank, mx, sm, _ in res:
+    for rank, mx, sm, _, e_ok, e_nan in res:
         assert mx == 17.25 and sm == 4000.0
+        assert e_ok == 10.0 and e_nan
     assert res[0][3] != res[1][3]   # each rank draws its own adapter mix
 
 
