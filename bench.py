@@ -38,6 +38,12 @@ import plora_workloads as wl  # noqa: E402
 METRIC = "packed LoRA fwd+bwd tokens/sec on 1 B200 (32 adapters); % HBM / tensor roofline"
 UNIT = "tokens/s"
 WORKLOAD = "llama3-8b up_proj 4096->14336 bf16, 32 adapters r~U{8,16,32,64,128}, tokens~logU[512,4096]"
+WORKLOADS = {
+    "llama_up32": WORKLOAD,
+    "small": "llama3-8b up_proj 4096->14336 bf16, the first 8 adapters of the 32-adapter mix x 2048 tokens",
+    "layer_q": "llama3-8b q_proj 4096->4096 bf16, 16 adapters r~U{16,32,64} x 8192 tokens",
+    "llama_up_r16x1": "llama3-8b up_proj 4096->14336 bf16, one rank-16 adapter over the 32-adapter mix's tokens",
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TC_KINDS = ("base_fwd", "base_dx")
 
@@ -57,9 +63,15 @@ def parse_args(argv=None):
                     help="base GEMMs on SM pairs (cta_group::2) instead of single SMs")
     ap.add_argument("--suite", action="store_true",
                     help="measure every workload (packed vs per-adapter sequential loop); one JSON line each")
-    ap.add_argument("--workload", choices=["llama_up32", "small", "layer_q"], default="llama_up32",
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="llama_up32",
                     help="small: 8 adapters of the same mix cut to 2048 tokens each; layer_q: the 4096x4096 q_proj "
-                         "of the one-layer workload, 16 adapters x 8192 tokens (both for profiler captures)")
+                         "of the one-layer workload, 16 adapters x 8192 tokens (both for profiler captures); "
+                         "llama_up_r16x1: one rank-16 adapter over the same tokens (base GEMMs with negligible "
+                         "low-rank work)")
+    ap.add_argument("--base-gemm-reference", action="store_true",
+                    help="time the workload's two base GEMMs (Y = X W^T, dX = dY W) through torch.matmul "
+                         "(cuBLAS) with the same timing, clock and energy records; a context line, not a "
+                         "product path")
     return ap.parse_args(argv)
 
 
@@ -277,6 +289,8 @@ def main(argv=None):
         return run_reference(args)
     if args.suite:
         return run_suite(args)
+    if args.base_gemm_reference:
+        return run_base_gemm_reference(args)
 
     import torch
     import torch.distributed as dist
@@ -301,6 +315,10 @@ def main(argv=None):
                             wl.init_llm(4096), args.seed + 1000 * rank)
     elif args.workload == "layer_q":
         p = wl.config4(seed=1004)[0]
+    elif args.workload == "llama_up_r16x1":
+        _, counts, _ = wl.config3_shape(args.seed + 1000 * rank)
+        p = wl.make_problem("cfg3_r16x1", "bf16", 4096, 14336, np.array([16]), [int(np.sum(counts))], [32.0],
+                            wl.init_llm(4096), args.seed + 1000 * rank)
     else:
         p = wl.config3(seed=args.seed + 1000 * rank)
     T = p.T
@@ -487,9 +505,11 @@ def main(argv=None):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "adapters": n, "tokens_per_gpu": T, "global_tokens": int(tokens_all),
+                "config": {"workload": WORKLOADS[args.workload], "adapters": n, "tokens_per_gpu": T,
+                           "global_tokens": int(tokens_all),
                            "d_in": p.d_in, "d_out": p.d_out, "parallelism": f"adapter-sharded x{world}",
-                           "l2": "inputs larger than L2 (X 452 MB, dY 1.6 GB); no flush",
+                           "l2": "inputs larger than L2 (X %.0f MB, dY %.0f MB); no flush" % (
+                               X.numel() * 2 / 1e6, dY.numel() * 2 / 1e6),
                            "base_gemm": base_gemm},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
                 "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
@@ -498,6 +518,58 @@ def main(argv=None):
     eng.close()
     if dist is not None:
         dist.destroy_process_group()
+    return 0
+
+
+def run_base_gemm_reference(args):
+    """The benchmark workload's two frozen-base GEMMs, Y = X W^T and dX = dY W, through torch.matmul
+    (cuBLAS), timed like a step of our arm: warm-up, CUDA events around `steps` back-to-back pairs,
+    clocks and energy sampled during the timed region.  It measures what the library GEMMs reach on
+    the same shapes under the same power limit; it runs no low-rank work."""
+    import torch
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    _, counts, _ = wl.config3_shape(args.seed)
+    T, di, do = int(np.sum(counts)), 4096, 14336
+    g = torch.Generator(device=dev)
+    g.manual_seed(args.seed)
+    X = torch.randn((T, di), generator=g, device=dev).to(torch.bfloat16)
+    dY = torch.randn((T, do), generator=g, device=dev).to(torch.bfloat16)
+    W = (torch.randn((do, di), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    Y = torch.empty((T, do), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((T, di), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        torch.matmul(X, W.t(), out=Y)
+        torch.matmul(dY, W, out=dX)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    clocks, energy = ClockSampler(uuid), EnergyMeter(uuid)
+    clocks.start()
+    time.sleep(0.3)
+    energy.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    joules, watts = energy.stop()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2 * 2.0 * T * di * do
+    print(json.dumps({"impl": "cublas-base-gemms", "what": "torch.matmul Y = X W^T and dX = dY W only (no low-rank work)",
+                      "config": {"workload": WORKLOAD, "tokens": T, "d_in": di, "d_out": do},
+                      "steps": args.steps, "ms_per_step": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                      "energy": None if joules is None else {"joules_per_step": joules / args.steps, "watts": watts},
+                      "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]}}),
+          flush=True)
     return 0
 
 

@@ -53,7 +53,8 @@ struct plora_ctx {
     size_t ws_bytes = 0;
     Region r_G, r_packA, r_packBT, r_part, r_cnt, r_err, r_blob[kSlots];
 
-    uint8_t* h_blob[kSlots] = {};
+    uint8_t* h_blob[kSlots] = {};       // mapped pinned staging of each slot (host view)
+    uint8_t* h_blob_dev[kSlots] = {};   // the same buffers as the device addresses them
     cudaEvent_t ev[kSlots] = {};
     int next_slot = 0;
 
@@ -148,10 +149,10 @@ __global__ void timeout_probe_kernel(int* err_flag, uint64_t limit_ns) {
 
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
-            kSimt, kAdamw, kPackB, kShrinkDyWgradB, kKinds };
+            kSimt, kAdamw, kPackB, kShrinkDyWgradB, kStage, kKinds };
 const char* const kKindNames[kKinds] = {"pack_a", "pack_bt", "base_fwd", "shrink_x", "expand_y", "base_dx",
                                         "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw",
-                                        "pack_b", "shrink_dy+wgrad_b"};
+                                        "pack_b", "shrink_dy+wgrad_b", "stage_copy"};
 
 cudaEvent_t take_event(plora_ctx* h) {
     if (!h->pool.empty()) {
@@ -367,6 +368,27 @@ struct DevPlan {
     int slot = 0;
 };
 
+// Copies a call's schedule from the slot's mapped pinned staging buffer into device memory.  A kernel
+// rather than cudaMemcpyAsync: its reads of host memory do not wait in the copy-engine queue behind
+// bulk host-to-device copies that the caller may have in flight (the next step's inputs, say).
+__global__ void stage_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n16) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = src[i];
+}
+
+// `bytes` of slot `slot`'s staging into device memory at d (rounded up to 16 bytes; the staging and
+// the device region are both whole multiples of 256 bytes).
+cudaError_t stage_copy(plora_ctx* h, int slot, uint8_t* d, size_t bytes, cudaStream_t st) {
+    const int64_t n16 = (int64_t)((bytes + 15) / 16);
+    if (n16 == 0) return cudaSuccess;
+    const int blocks = (int)std::min<int64_t>(ceil_div(n16, 256), 64);
+    tracked(h, kStage, st, [&] {
+        stage_copy_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(h->h_blob_dev[slot]),
+                                                  reinterpret_cast<uint4*>(d), n16);
+    });
+    return cudaGetLastError();
+}
+
 plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& ops, cudaStream_t st,
                     DevPlan& D) {
     const int slot = h->next_slot;
@@ -388,8 +410,8 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     const size_t o_mtl = put(P.mt_seg.data(), P.mt_seg.size() * sizeof(LoraSeg));
     if (o > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "schedule exceeds the handle's staging size");
     uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
-    e = cudaMemcpyAsync(d, h->h_blob[slot], o, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync(schedule)");
+    e = stage_copy(h, slot, d, o, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "copying the schedule to the device");
     D.ad = reinterpret_cast<AdapterDev*>(d + o_ad);
     D.tok = reinterpret_cast<TokTile*>(d + o_tok);
     D.red = reinterpret_cast<RedEntry*>(d + o_red);
@@ -413,8 +435,8 @@ plora_status upload_parts(plora_ctx* h, const void* a, size_t na, const void* b,
     if (na) memcpy(h->h_blob[slot], a, na);
     if (nb) memcpy(h->h_blob[slot] + ob, b, nb);
     uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
-    e = cudaMemcpyAsync(d, h->h_blob[slot], total, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync(optimizer tables)");
+    e = stage_copy(h, slot, d, total, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "copying the optimizer tables to the device");
     *da = d;
     *db = d + ob;
     *slot_out = slot;
@@ -681,7 +703,8 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     if (e != cudaSuccess) { cudaGetLastError(); delete h; return PLORA_ERR_OOM; }
     e = cudaMemset(h->ws, 0, h->ws_bytes);
     for (int s = 0; s < kSlots && e == cudaSuccess; ++s) {
-        e = cudaMallocHost(&h->h_blob[s], h->blob_bytes);
+        e = cudaHostAlloc(&h->h_blob[s], h->blob_bytes, cudaHostAllocMapped | cudaHostAllocPortable);
+        if (e == cudaSuccess) e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->h_blob_dev[s]), h->h_blob[s], 0);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev[s], cudaEventDisableTiming);
     }
     if (e == cudaSuccess && h->tc) {
