@@ -250,7 +250,7 @@ def config5_mix(which: str, seed: int = 1005) -> Problem:
     i:   8 adapters alternating rank 1 and rank 256, 2048 tokens each
     ii:  8 adapters with 1 and 8192 tokens alternating, rank 16
     iii: 16 equal segments of 2048 tokens, rank ~ U{1,16,256}
-    iv:  mix iii with a 0-token adapter inserted (an extra case of this build)"""
+    iv:  mix iii with a 0-token adapter inserted (an added edge case: an adapter with no tokens)"""
     if which == "i":
         r = [1, 256] * 4
         c = [2048] * 8
