@@ -404,7 +404,12 @@ def main(argv=None):
         if cnt == 0:
             continue
         avg_ms = tot / cnt
-        fl, by = work.get(kind, (0.0, 0.0))
+        if kind not in work:
+            # no algorithmic work of its own (the schedule staging copy): latency, not a roofline
+            kernels[kind] = {"launches": cnt, "avg_ms": avg_ms, "bound": "latency", "achieved": None,
+                             "unit": None, "frac": None}
+            continue
+        fl, by = work[kind]
         if kind in TC_KINDS:
             ach = fl / (avg_ms / 1e3) / 1e12
             kernels[kind] = {"launches": cnt, "avg_ms": avg_ms, "bound": "tensor", "achieved": ach,
