@@ -748,7 +748,102 @@ def run_suite(args):
             L["eng"].close()
         del layers
         torch.cuda.empty_cache()
+    layer_shared_inputs(args)
     return 0
+
+
+def layer_shared_inputs(args):
+    """One LLaMA-3-8B layer whose LoRA targets read their inputs as in the model: q, k and v share
+    one input, gate and up another, o and down have their own.  Timed as seven single-projection
+    calls and as four calls with q|k|v and gate|up stacked as output blocks (one base GEMM each).
+    16 adapters x 8192 tokens, r ~ U{16,32,64}, alpha = 2r.  One JSON line."""
+    import torch
+    import packed_lora_fine_b200 as pl
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(args.seed + 7)
+    ranks = [int(x) for x in wl.rng_for(1004, 1).choice(np.array([16, 32, 64]), size=16)]
+    n = len(ranks)
+    off = np.arange(n + 1, dtype=np.int64) * 8192
+    T = int(off[-1])
+    scales = [2.0] * n
+    shape = {nm: (di, do) for nm, di, do in wl.LLAMA3_LAYER}
+    groups = [("q", "k", "v"), ("o",), ("gate", "up"), ("down",)]
+    proj = {}
+    for grp in groups:
+        X = torch.randn((T, shape[grp[0]][0]), generator=g, device=dev).to(torch.bfloat16)
+        for nm in grp:
+            di, do = shape[nm]
+            bound = math.sqrt(6.0 / di)
+            proj[nm] = dict(X=X, dY=torch.randn((T, do), generator=g, device=dev).to(torch.bfloat16),
+                            W=(torch.randn((do, di), generator=g, device=dev) * 0.02).to(torch.bfloat16),
+                            A=[((torch.rand((r, di), generator=g, device=dev) * 2 - 1) * bound).to(torch.bfloat16)
+                               for r in ranks],
+                            B=[(torch.randn((do, r), generator=g, device=dev) * 0.01).to(torch.bfloat16)
+                               for r in ranks])
+
+    def call(nms):
+        """A handle and its buffers for the projections `nms` (stacked as output blocks if several)."""
+        di = shape[nms[0]][0]
+        widths = [shape[nm][1] for nm in nms]
+        cat = lambda ts, dim=0: ts[0] if len(ts) == 1 else torch.cat(ts, dim=dim).contiguous()
+        W = cat([proj[nm]["W"] for nm in nms])
+        dY = cat([proj[nm]["dY"] for nm in nms], 1)
+        A = [cat([proj[nm]["A"][i] for nm in nms]) for i in range(n)]
+        B = [cat([proj[nm]["B"][i] for nm in nms]) for i in range(n)]
+        eng = pl.PackedLoRA(di, sum(widths), "bf16", max_adapters=n, max_rank=max(ranks), max_tokens=T,
+                            out_blocks=widths if len(nms) > 1 else None)
+        dA = [torch.empty(a.shape, dtype=torch.float32, device=dev) for a in A]
+        dB = [torch.empty(b.shape, dtype=torch.float32, device=dev) for b in B]
+        tf, tb = eng.table(scales, A, B), eng.table(scales, A, B, dA, dB)
+        return dict(eng=eng, X=proj[nms[0]]["X"], W=W, dY=dY, A=A, B=B, dA=dA, dB=dB, tf=tf, tb=tb,
+                    Y=torch.empty((T, sum(widths)), dtype=torch.bfloat16, device=dev),
+                    dX=torch.empty((T, di), dtype=torch.bfloat16, device=dev),
+                    saved=torch.empty(max(256, eng.saved_bytes(off, tf)), dtype=torch.uint8, device=dev))
+
+    def step(calls):
+        for c in calls:
+            e = c["eng"]
+            pl.plora_forward(e.h, c["X"].data_ptr(), c["W"].data_ptr(), c["Y"].data_ptr(), n, off, c["tf"],
+                             c["saved"].data_ptr(), st.cuda_stream)
+            pl.plora_backward(e.h, c["X"].data_ptr(), c["W"].data_ptr(), c["dY"].data_ptr(), c["dX"].data_ptr(),
+                              n, off, c["tb"], c["saved"].data_ptr(), st.cuda_stream)
+
+    def timed(calls, steps):
+        for _ in range(3):
+            step(calls)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            step(calls)
+        e1.record(st)
+        torch.cuda.synchronize()
+        for c in calls:
+            assert pl.plora_check(c["eng"].h, 0) == pl.PLORA_OK
+        return e0.elapsed_time(e1) / steps
+
+    steps = max(5, min(args.steps, 20))
+    sep = [call((nm,)) for grp in groups for nm in grp]
+    ms_sep = timed(sep, steps)
+    q_sep = sep[0]["Y"].clone()
+    for c in sep:
+        c["eng"].close()
+    del sep
+    torch.cuda.empty_cache()
+    fused = [call(grp) for grp in groups]
+    ms_fused = timed(fused, steps)
+    same_q = bool(torch.equal(fused[0]["Y"][:, :shape["q"][1]], q_sep))
+    for c in fused:
+        c["eng"].close()
+    print(json.dumps({"suite": "llama3-8b layer, shared inputs: q|k|v and gate|up as output blocks",
+                      "tokens": T, "adapters": n, "projections": 7,
+                      "separate_calls": 7, "separate_ms_per_step": ms_sep, "separate_tokens_per_s": T / (ms_sep / 1e3),
+                      "fused_calls": len(groups), "fused_ms_per_step": ms_fused,
+                      "fused_tokens_per_s": T / (ms_fused / 1e3), "fused_over_separate": ms_sep / ms_fused,
+                      "q_output_bit_identical": same_q}), flush=True)
+    torch.cuda.empty_cache()
 
 
 if __name__ == "__main__":

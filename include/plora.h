@@ -102,12 +102,28 @@ enum {
 /* Limits. */
 #define PLORA_MAX_RANK 256
 #define PLORA_MAX_ADAPTERS 4096
+#define PLORA_MAX_OUT_BLOCKS 8
 
 /*
  * Handle configuration.  d_in, d_out: projection sizes, multiples of 8 in
  * [8, 65536].  dtype: a plora_dtype.  max_adapters in [1, PLORA_MAX_ADAPTERS],
  * max_rank in [1, PLORA_MAX_RANK], max_tokens >= 1: upper bounds of every
  * later call, used to size the workspace.
+ *
+ * Output blocks (shared-input projections in one base GEMM).  LoRA is usually
+ * applied to the attention's query, key and value projections, which read the
+ * same input ("LoRA加速集成方案", cloud.baidu.com, 七 › 2. 层的选择), and PEFT
+ * configures them as one fused query_key_value module ("LLM+LoRA微调加速技术原理解析",
+ * m.youleyou.com, 深入理解LoRA：基本原理与PEFT实现).  With n_out_blocks = P in
+ * [2, PLORA_MAX_OUT_BLOCKS], W is P such projections stacked along d_out: block p
+ * holds output columns [out_block_end[p-1], out_block_end[p]) (out_block_end[-1] = 0),
+ * each end a multiple of 256, out_block_end[P-1] = d_out.  Every adapter then has its
+ * own low-rank pair per block, all of rank r: Y[:, block p] = X W_p^T + s X A_p^T B_p^T.
+ * The layouts stack the blocks (see plora_adapter).  P * roundup(max_rank, 16) must not
+ * exceed 256.  Output blocks need the default tensor-core path (bf16, no
+ * PLORA_FLAG_SIMT / UNFUSED / BASE_PAIR); other combinations return
+ * PLORA_ERR_UNSUPPORTED.  n_out_blocks = 0 or 1 means one projection (the ends are
+ * then ignored).
  */
 typedef struct {
     int64_t d_in;
@@ -117,13 +133,18 @@ typedef struct {
     int32_t max_rank;
     uint32_t flags;
     int64_t max_tokens;
+    int32_t n_out_blocks;
+    int32_t reserved;                               /* 0 */
+    int64_t out_block_end[PLORA_MAX_OUT_BLOCKS];
 } plora_config;
 
 /*
  * One adapter.  rank r in [1, max_rank]; scale = alpha / r as the caller
  * computed it (finite); A: [r][d_in], B: [d_out][r] in the handle's dtype;
  * dA: [r][d_in], dB: [d_out][r] in fp32 (written by plora_backward, ignored
- * by plora_forward).  Every pointer 16-byte aligned.
+ * by plora_forward).  Every pointer 16-byte aligned.  With P output blocks,
+ * A and dA are [P r][d_in] (rows p r .. p r + r - 1 are block p's A_p) and B, dB
+ * stay [d_out][r] (the rows of block p's columns are its B_p).
  */
 typedef struct {
     int32_t rank;
@@ -194,7 +215,8 @@ PLORA_API const char* plora_last_error(plora_handle h);
 /*
  * Debug: copy adapter i's saved activation H'_i = s_i X_i A_i (the scaled
  * shrink, which both the expand and dB consume) out of `saved` as fp32
- * [n_i][r_i] into the device buffer H_out (16-byte aligned).
+ * [n_i][r_i] into the device buffer H_out (16-byte aligned); with P output blocks,
+ * [n_i][P r_i], block p in columns p r_i .. p r_i + r_i - 1.
  */
 PLORA_API plora_status plora_debug_unpack_saved(plora_handle h, int32_t n_adapters, const int64_t* off,
                                       const plora_adapter* tab, const void* saved, int32_t i,
@@ -300,8 +322,8 @@ PLORA_API plora_status plora_profile_read(plora_handle h, int32_t capacity, int3
  * loading this library holds until the process exits.  The call allocates
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *
- * cfg: as for plora_create (bf16, no PLORA_FLAG_SIMT; the max_* fields bound
- * the call).  dY: [T][d_out] bf16 device; saved: the buffer a plora_forward
+ * cfg: as for plora_create (bf16, no PLORA_FLAG_SIMT, one output block; the max_*
+ * fields bound the call).  dY: [T][d_out] bf16 device; saved: the buffer a plora_forward
  * with the same off and adapter ranks filled; off, tab: host arrays as for
  * plora_backward (only rank, scale and dB are read; dB must be non-NULL and
  * 16-byte aligned, A and B must still be valid pointers).  Writes every dB_i.

@@ -35,6 +35,7 @@ PLORA_FLAG_UNFUSED = 2
 PLORA_FLAG_BASE_PAIR = 4
 PLORA_MAX_RANK = 256
 PLORA_MAX_ADAPTERS = 4096
+PLORA_MAX_OUT_BLOCKS = 8
 PLORA_STATIC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
@@ -46,7 +47,21 @@ EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward
 class plora_config(ctypes.Structure):
     _fields_ = [("d_in", ctypes.c_int64), ("d_out", ctypes.c_int64), ("dtype", ctypes.c_int32),
                 ("max_adapters", ctypes.c_int32), ("max_rank", ctypes.c_int32), ("flags", ctypes.c_uint32),
-                ("max_tokens", ctypes.c_int64)]
+                ("max_tokens", ctypes.c_int64), ("n_out_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("out_block_end", ctypes.c_int64 * PLORA_MAX_OUT_BLOCKS)]
+
+
+def make_config(d_in, d_out, dtype, max_adapters, max_rank, max_tokens, flags=0, out_blocks=None):
+    """plora_config; out_blocks: the output widths of P >= 2 shared-input projections stacked in W
+    (their sum is d_out), or None for one projection."""
+    cfg = plora_config(d_in, d_out, dtype, max_adapters, max_rank, flags, max_tokens)
+    if out_blocks is not None and len(out_blocks) > 1:
+        cfg.n_out_blocks = len(out_blocks)
+        end = 0
+        for b, w in enumerate(out_blocks):
+            end += int(w)
+            cfg.out_block_end[b] = end
+    return cfg
 
 
 class plora_adapter(ctypes.Structure):
@@ -146,9 +161,9 @@ def make_table(ranks: Sequence[int], scales: Sequence[float], A: Sequence[int], 
 
 # ---------------------------------------------------------------- C names
 def plora_create(d_in: int, d_out: int, dtype: int, max_adapters: int, max_rank: int, max_tokens: int,
-                 flags: int = 0) -> int:
+                 flags: int = 0, out_blocks=None) -> int:
     lib = load()
-    cfg = plora_config(d_in, d_out, dtype, max_adapters, max_rank, flags, max_tokens)
+    cfg = make_config(d_in, d_out, dtype, max_adapters, max_rank, max_tokens, flags, out_blocks)
     h = ctypes.c_void_p()
     s = lib.plora_create(ctypes.byref(h), ctypes.byref(cfg))
     if s != PLORA_OK:
@@ -293,16 +308,20 @@ class PackedLoRA:
     ``A[i]`` is ``[r_i][d_in]`` (lora_A.weight), ``B[i]`` is ``[d_out][r_i]``
     (lora_B.weight), ``W`` is ``[d_out][d_in]`` (nn.Linear.weight), ``X`` is
     the packed ``[T][d_in]`` token buffer, ``off`` the host segment offsets.
+    With ``out_blocks`` (the widths of P shared-input projections stacked in W, e.g.
+    q, k, v), ``A[i]`` is the P projections' lora_A weights stacked, ``[P r_i][d_in]``,
+    and ``B[i]`` their lora_B weights stacked, ``[d_out][r_i]``.
     """
 
     def __init__(self, d_in, d_out, dtype="bf16", max_adapters=64, max_rank=PLORA_MAX_RANK,
-                 max_tokens=1 << 16, simt=False, unfused=False, base_pair=False):
+                 max_tokens=1 << 16, simt=False, unfused=False, base_pair=False, out_blocks=None):
         self.d_in, self.d_out = int(d_in), int(d_out)
         self.dtype = dtype
+        self.out_blocks = list(out_blocks) if out_blocks is not None else None
         self.h = plora_create(self.d_in, self.d_out, PLORA_BF16 if dtype == "bf16" else PLORA_FP32,
                               max_adapters, max_rank, max_tokens,
                               (PLORA_FLAG_SIMT if simt else 0) | (PLORA_FLAG_UNFUSED if unfused else 0)
-                              | (PLORA_FLAG_BASE_PAIR if base_pair else 0))
+                              | (PLORA_FLAG_BASE_PAIR if base_pair else 0), out_blocks)
 
     def close(self):
         if self.h:
@@ -316,7 +335,7 @@ class PackedLoRA:
             pass
 
     def table(self, scales, A, B, dA=None, dB=None):
-        ranks = [a.shape[0] for a in A]
+        ranks = [b.shape[1] for b in B]
         return make_table(ranks, scales, [a.data_ptr() for a in A], [b.data_ptr() for b in B],
                           None if dA is None else [x.data_ptr() for x in dA],
                           None if dB is None else [x.data_ptr() for x in dB])

@@ -1,8 +1,8 @@
 // plan.cuh -- per-call schedule structures shared by the host code and the kernels.
 //
 // A call's schedule is built on the host from the segment offsets and the
-// adapter table, copied once to the device (one cudaMemcpyAsync from pinned
-// staging), and read by every kernel of the call.
+// adapter table, copied once to the device (by a small kernel, from mapped
+// pinned staging), and read by every kernel of the call.
 #pragma once
 #include <cstdint>
 
@@ -15,20 +15,29 @@ constexpr int kSplitTokens = 16384; // weight-gradient split size along the toke
 constexpr int kLoraPad = 256;       // zero rows before and after each adapter's H' / G block
 constexpr int kLoraTileM = 256;     // base-GEMM rows per overlap record (one CTA-pair tile)
 
-// One adapter, as the kernels see it.
+constexpr int kMaxOutBlocks = 8;    // output blocks (shared-input projections stacked along d_out)
+
+// The output blocks of a handle: block b holds output columns [end[b-1], end[b]).
+struct OutBlocks {
+    int32_t n;
+    int32_t end[kMaxOutBlocks];
+};
+
+// One adapter, as the kernels see it.  With P output blocks an adapter has one rank-r pair
+// per block; H' and G hold block p in columns [p rblk, p rblk + r) (zeros up to (p+1) rblk).
 struct AdapterDev {
-    const void* A;     // A_store [rank][d_in]
+    const void* A;     // A_store [P rank][d_in] (block p = rows p rank ..)
     const void* B;     // B_store [d_out][rank]
-    float* dA;         // [rank][d_in]
+    float* dA;         // [P rank][d_in]
     float* dB;         // [d_out][rank]
     int32_t x_row;     // first token row in X / Y / dY / dX (= off[i])
     int32_t n;         // tokens of this adapter
     int32_t h_row;     // first row of this adapter's block in the saved H / workspace G buffers
     int32_t rank;
     float scale;
-    int32_t rp16;      // rank rounded up to 16 (the MMA N or K extent)
-    int32_t rp64;      // rank rounded up to 64 (the MN-major tile width)
-    int32_t pad_;
+    int32_t rp16;      // width of its H' / G columns, P rblk (the shrink's N, the dX fold's K)
+    int32_t rp64;      // rp16 rounded up to 64 (the MN-major tile width of dA)
+    int32_t rblk;      // rank rounded up to 16 (one block's pitch: the Y fold's and dB's extent)
 };
 static_assert(sizeof(AdapterDev) == 64, "AdapterDev layout");
 
@@ -58,8 +67,8 @@ static_assert(sizeof(RedEntry) == 32, "RedEntry layout");
 struct LoraSeg {
     int32_t adapter;
     int32_t h_y;       // H' / G row holding the tile's first token, inside the adapter's zero-padded block
-    int32_t rp16;      // rank rounded up to 16 (the K extent of the folded product)
-    int32_t pad_;
+    int32_t rp16;      // K extent of the folded dX product (the adapter's P rblk)
+    int32_t rblk;      // K extent of the folded Y product (one output block's rank, rounded up to 16)
 };
 static_assert(sizeof(LoraSeg) == 16, "LoraSeg layout");
 

@@ -47,6 +47,8 @@ struct plora_ctx {
     int64_t max_slots = 0, max_counters = 0;
     size_t blob_bytes = 0;
     bool tc = false;           // tensor-core path (bf16 without PLORA_FLAG_SIMT)
+    int nblk = 1;              // output blocks (shared-input projections stacked along d_out)
+    int32_t blk_end[kMaxOutBlocks] = {};   // cumulative output-column ends of the blocks
     int pairs_fwd = 0, pairs_dx = 0;   // co-resident SM pairs for the pair-tile base GEMMs
 
     uint8_t* ws = nullptr;     // one device allocation, carved into regions
@@ -246,7 +248,7 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
     P.T = off[n];
     int maxr = 1;
     for (int32_t i = 0; i < n; ++i) maxr = std::max(maxr, tab[i].rank);
-    P.RP = (int32_t)round_up(maxr, kRankAlign);
+    P.RP = (int32_t)round_up(h->nblk * round_up(maxr, 16), kRankAlign);   // the widest adapter's P rblk
     P.ad.resize(n);
     int64_t hrow = 0;
     const int64_t dtiles = std::max(ceil_div(h->cfg.d_in, kTileM), ceil_div(h->cfg.d_out, kTileM));
@@ -261,9 +263,9 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
         a.h_row = (int32_t)hrow;
         a.rank = tab[i].rank;
         a.scale = tab[i].scale;
-        a.rp16 = (int32_t)round_up(a.rank, 16);
-        a.rp64 = (int32_t)round_up(a.rank, 64);
-        a.pad_ = 0;
+        a.rblk = (int32_t)round_up(a.rank, 16);
+        a.rp16 = h->nblk * a.rblk;
+        a.rp64 = (int32_t)round_up(a.rp16, 64);
         if (a.n == 0) {
             P.empty.push_back(i);
             continue;
@@ -300,7 +302,7 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
         while (first < n && off[first + 1] <= m0) ++first;
         for (int32_t j = first; j < n && off[j] < m1; ++j)
             if (off[j + 1] > off[j])
-                P.mt_seg.push_back(LoraSeg{j, (int32_t)(P.ad[j].h_row + (m0 - off[j])), P.ad[j].rp16, 0});
+                P.mt_seg.push_back(LoraSeg{j, (int32_t)(P.ad[j].h_row + (m0 - off[j])), P.ad[j].rp16, P.ad[j].rblk});
     }
     P.mt_off[tiles_m] = (int32_t)P.mt_seg.size();
     P.mt_rec.assign(tiles_m, MTileRec{});
@@ -346,10 +348,11 @@ plora_status check_extents(plora_ctx* h, const HostPlan& P, const plora_adapter*
             return fail(h, PLORA_ERR_INVALID_ARG, "%s is not a device buffer of %zu bytes", it.name, it.bytes);
     for (int32_t i = 0; i < P.n; ++i) {
         const size_t r = (size_t)tab[i].rank;
-        if (a.adapters_AB && (!in_device_allocation(tab[i].A, r * di * es) ||
+        const size_t ra = r * (size_t)h->nblk;   // rows of A and dA: one rank-r block per output block
+        if (a.adapters_AB && (!in_device_allocation(tab[i].A, ra * di * es) ||
                               !in_device_allocation(tab[i].B, dout * r * es)))
             return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: A or B is not a device buffer of its size", i);
-        if (a.adapters_dA && !in_device_allocation(tab[i].dA, r * di * sizeof(float)))
+        if (a.adapters_dA && !in_device_allocation(tab[i].dA, ra * di * sizeof(float)))
             return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: dA is not a device buffer of its size", i);
         if (a.adapters_dB && !in_device_allocation(tab[i].dB, dout * r * sizeof(float)))
             return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: dB is not a device buffer of its size", i);
@@ -582,6 +585,8 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     p.fuse = 0;
     p.stages = kStages;
     p.stage_bytes = kStageBytes;
+    p.nblk = h->nblk;
+    for (int b = 0; b < kMaxOutBlocks; ++b) p.blk_end[b] = h->blk_end[b];
     return p;
 }
 
@@ -599,7 +604,7 @@ plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, BPa
     const int grid_a = (int)std::min<int64_t>(ceil_div(vecs, 256), grid_cap);
     tracked(h, kPackA, st, [&] { pack_a_kernel<<<grid_a, 256, 0, st>>>(D.ad, P.n, P.RP, h->cfg.d_in, pa); });
     if (bp == BPack::RowPadded) {
-        int maxr16 = 16; for (const AdapterDev& a : P.ad) maxr16 = std::max(maxr16, a.rp16);
+        int maxr16 = 16; for (const AdapterDev& a : P.ad) maxr16 = std::max(maxr16, a.rblk);
         const int64_t per_adapter = h->cfg.d_out * (maxr16 / 8);
         dim3 grid_b((unsigned)std::min<int64_t>(ceil_div(per_adapter, 256), 65535), (unsigned)P.n);
         tracked(h, kPackB, st, [&] { pack_b_kernel<<<grid_b, 256, 0, st>>>(D.ad, P.RP, (int)h->cfg.d_out, pb); });
@@ -608,7 +613,10 @@ plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, BPa
     dim3 gb((unsigned)ceil_div(h->cfg.d_out, 128), (unsigned)P.n);
     int maxr = 1; for (const AdapterDev& a : P.ad) maxr = std::max(maxr, a.rank);
     const size_t smem_bt = (size_t)128 * (maxr + 2) * sizeof(__nv_bfloat16);
-    tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, smem_bt, st>>>(D.ad, P.RP, h->cfg.d_out, pb); });
+    OutBlocks blocks{};
+    blocks.n = h->nblk;
+    for (int b = 0; b < kMaxOutBlocks; ++b) blocks.end[b] = h->blk_end[b];
+    tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, smem_bt, st>>>(D.ad, P.RP, h->cfg.d_out, blocks, pb); });
     return PLORA_OK;
 }
 
@@ -633,7 +641,27 @@ const char* plora_status_string(plora_status s) {
 
 const char* plora_last_error(plora_handle h) { return h ? h->last_error.c_str() : ""; }
 
-int32_t plora_version(void) { return 100; }
+int32_t plora_version(void) { return 101; }
+
+// Output blocks of a config: 1 (one projection) or n_out_blocks, with the checks the header lists.
+plora_status check_out_blocks(const plora_config* cfg, int* nblk) {
+    *nblk = 1;
+    if (cfg->n_out_blocks < 0 || cfg->n_out_blocks > PLORA_MAX_OUT_BLOCKS || cfg->reserved != 0)
+        return PLORA_ERR_INVALID_ARG;
+    if (cfg->n_out_blocks <= 1) return PLORA_OK;
+    if (cfg->dtype != PLORA_BF16 || (cfg->flags & (PLORA_FLAG_SIMT | PLORA_FLAG_UNFUSED | PLORA_FLAG_BASE_PAIR)))
+        return PLORA_ERR_UNSUPPORTED;
+    int64_t prev = 0;
+    for (int b = 0; b < cfg->n_out_blocks; ++b) {
+        const int64_t e = cfg->out_block_end[b];
+        if (e <= prev || e % 256) return PLORA_ERR_INVALID_ARG;
+        prev = e;
+    }
+    if (prev != cfg->d_out) return PLORA_ERR_INVALID_ARG;
+    if (cfg->n_out_blocks * round_up(cfg->max_rank, 16) > PLORA_MAX_RANK) return PLORA_ERR_INVALID_ARG;
+    *nblk = cfg->n_out_blocks;
+    return PLORA_OK;
+}
 
 plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     if (!out) return PLORA_ERR_INVALID_ARG;
@@ -646,10 +674,15 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     if (cfg->max_rank < 1 || cfg->max_rank > PLORA_MAX_RANK) return PLORA_ERR_INVALID_ARG;
     if (cfg->max_tokens < 1 || cfg->max_tokens > ((int64_t)1 << 30)) return PLORA_ERR_INVALID_ARG;
     if (cfg->flags & ~(uint32_t)(PLORA_FLAG_SIMT | PLORA_FLAG_UNFUSED | PLORA_FLAG_BASE_PAIR)) return PLORA_ERR_INVALID_ARG;
+    int nblk = 1;
+    const plora_status sb = check_out_blocks(cfg, &nblk);
+    if (sb != PLORA_OK) return sb;
 
     plora_ctx* h = new (std::nothrow) plora_ctx();
     if (!h) return PLORA_ERR_OOM;
     h->cfg = *cfg;
+    h->nblk = nblk;
+    for (int b = 0; b < nblk; ++b) h->blk_end[b] = (int32_t)(nblk > 1 ? cfg->out_block_end[b] : cfg->d_out);
     h->esize = cfg->dtype == PLORA_BF16 ? 2 : 4;
     h->tc = cfg->dtype == PLORA_BF16 && !(cfg->flags & PLORA_FLAG_SIMT);
 
@@ -663,7 +696,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
 
     // Workspace sizing (all bounds follow from the config).
     const int64_t na = cfg->max_adapters;
-    h->RPmax = (int)round_up(cfg->max_rank, kRankAlign);
+    h->RPmax = (int)round_up(nblk * round_up(cfg->max_rank, 16), kRankAlign);
     h->max_h_rows = cfg->max_tokens + (int64_t)(kTileM - 1 + 2 * kLoraPad) * na;
     const int64_t dtiles = std::max(ceil_div(cfg->d_in, kTileM), ceil_div(cfg->d_out, kTileM));
     h->max_slots = 2 * (cfg->max_tokens / kSplitTokens) + 1;
@@ -678,7 +711,8 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
                     (size_t)round_up((tok_max + 1) * (int64_t)sizeof(MTileRec), 256) +
                     (size_t)round_up((tok_max + na) * (int64_t)sizeof(LoraSeg), 256) + 1024;
     // The AdamW step's tables (segments and chunks) travel through the same staging ring.
-    const int64_t adamw_chunks = 2 * na + na * (int64_t)cfg->max_rank * (cfg->d_in + cfg->d_out) / kAdamwChunk;
+    const int64_t adamw_chunks =
+        2 * na + na * (int64_t)cfg->max_rank * (nblk * cfg->d_in + cfg->d_out) / kAdamwChunk;
     h->blob_bytes = std::max(h->blob_bytes, (size_t)round_up(2 * na * (int64_t)sizeof(AdamwSeg), 256) +
                                                 (size_t)round_up(adamw_chunks * (int64_t)sizeof(AdamwChunk), 256) +
                                                 1024);
@@ -907,7 +941,7 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
     // Adapters without tokens: their weight gradients are zero.
     for (int32_t i : P.empty) {
-        ce = cudaMemsetAsync(tab[i].dA, 0, (size_t)tab[i].rank * d_in * sizeof(float), st);
+        ce = cudaMemsetAsync(tab[i].dA, 0, (size_t)tab[i].rank * h->nblk * d_in * sizeof(float), st);
         if (ce == cudaSuccess) ce = cudaMemsetAsync(tab[i].dB, 0, (size_t)tab[i].rank * d_out * sizeof(float), st);
         if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaMemsetAsync(dA/dB of an empty adapter)");
     }
@@ -1061,18 +1095,19 @@ plora_status plora_debug_unpack_saved(plora_handle h, int32_t n, const int64_t* 
         ta.saved = saved;
         ta.adapters_AB = false;
         s = check_extents(h, P, tab, ta);
-        if (s == PLORA_OK && !in_device_allocation(H_out, (size_t)a.n * a.rank * sizeof(float)))
-            s = fail(h, PLORA_ERR_INVALID_ARG, "H_out is not a device buffer of %zu bytes",
-                     (size_t)a.n * a.rank * sizeof(float));
+        const size_t out_bytes = (size_t)a.n * a.rank * h->nblk * sizeof(float);
+        if (s == PLORA_OK && !in_device_allocation(H_out, out_bytes))
+            s = fail(h, PLORA_ERR_INVALID_ARG, "H_out is not a device buffer of %zu bytes", out_bytes);
         if (s != PLORA_OK) return s;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int grid = (int)std::min<int64_t>(ceil_div((int64_t)a.n * a.rank, 256), 1024);
+    const int grid = (int)std::min<int64_t>(ceil_div((int64_t)a.n * a.rank * h->nblk, 256), 1024);
     if (h->cfg.dtype == PLORA_FP32)
-        unpack_saved_kernel<float><<<grid, 256, 0, st>>>((const float*)saved, a.h_row, P.RP, a.n, a.rank, H_out);
+        unpack_saved_kernel<float><<<grid, 256, 0, st>>>((const float*)saved, a.h_row, P.RP, a.n, a.rank, h->nblk,
+                                                         a.rblk, H_out);
     else
         unpack_saved_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)saved, a.h_row, P.RP, a.n,
-                                                                 a.rank, H_out);
+                                                                 a.rank, h->nblk, a.rblk, H_out);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PLORA_OK : cuda_fail(h, e, "unpack launch");
 }
@@ -1104,12 +1139,13 @@ plora_status plora_adamw_step(plora_handle h, int32_t n, const plora_adapter* ta
         if (!bf16 && (o.A_master || o.B_master))
             return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: an fp32 handle updates A and B in place", i);
         const size_t r = (size_t)a.rank;
+        const size_t ra = r * (size_t)h->nblk;   // rows of A: one rank-r block per output block
         const size_t es = h->esize;
         float* pA = bf16 ? o.A_master : const_cast<float*>(static_cast<const float*>(a.A));
         float* pB = bf16 ? o.B_master : const_cast<float*>(static_cast<const float*>(a.B));
         const void* ptrs[] = {a.A, a.B, a.dA, a.dB, pA, pB, o.mA, o.vA, o.mB, o.vB};
-        const size_t bytes[] = {r * di * es, dout * r * es, r * di * 4, dout * r * 4, r * di * 4, dout * r * 4,
-                                r * di * 4, r * di * 4, dout * r * 4, dout * r * 4};
+        const size_t bytes[] = {ra * di * es, dout * r * es, ra * di * 4, dout * r * 4, ra * di * 4, dout * r * 4,
+                                ra * di * 4, ra * di * 4, dout * r * 4, dout * r * 4};
         for (int k = 0; k < 10; ++k) {
             if (!ptrs[k] || !aligned16(ptrs[k]))
                 return fail(h, PLORA_ERR_INVALID_ARG, "adapter %d: a parameter, gradient or state pointer is NULL "
@@ -1130,7 +1166,7 @@ plora_status plora_adamw_step(plora_handle h, int32_t n, const plora_adapter* ta
         sg.eps = o.eps;
         AdamwSeg sa = sg, sb = sg;
         sa.p = pA; sa.m = o.mA; sa.v = o.vA; sa.g = a.dA; sa.out = bf16 ? const_cast<void*>(a.A) : nullptr;
-        sa.n = (int64_t)(r * di);
+        sa.n = (int64_t)(ra * di);
         sb.p = pB; sb.m = o.mB; sb.v = o.vB; sb.g = a.dB; sb.out = bf16 ? const_cast<void*>(a.B) : nullptr;
         sb.n = (int64_t)(dout * r);
         for (const AdamwSeg& x : {sa, sb}) {
@@ -1206,7 +1242,9 @@ plora_status plora_debug_schedule(const plora_config* cfg, int32_t n, const int6
     plora_ctx tmp;
     tmp.cfg = *cfg;
     tmp.esize = cfg->dtype == PLORA_FP32 ? 4 : 2;
-    plora_status s = check_table(&tmp, n, off, tab, grads != 0);
+    plora_status s = check_out_blocks(cfg, &tmp.nblk);
+    if (s != PLORA_OK) return s;
+    s = check_table(&tmp, n, off, tab, grads != 0);
     if (s != PLORA_OK) return s;
     HostPlan P;
     build_plan(&tmp, n, off, tab, P);
@@ -1294,7 +1332,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void* dY, int32_t n, const int64_t* off,
                                             const plora_adapter* tab, const void* saved, void* stream) {
     if (!cfg) return PLORA_ERR_INVALID_ARG;
-    if (cfg->dtype != PLORA_BF16 || (cfg->flags & PLORA_FLAG_SIMT)) return PLORA_ERR_UNSUPPORTED;
+    if (cfg->dtype != PLORA_BF16 || (cfg->flags & PLORA_FLAG_SIMT) || cfg->n_out_blocks > 1)
+        return PLORA_ERR_UNSUPPORTED;
     if (cfg->d_in < 8 || cfg->d_out < 8 || cfg->d_in > 65536 || cfg->d_out > 65536 || cfg->d_in % 8 ||
         cfg->d_out % 8)
         return PLORA_ERR_UNSUPPORTED;
@@ -1364,6 +1403,7 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
         return PLORA_ERR_CUDA;
     TcParams p{};
     p.RP = P.RP;
+    p.nblk = 1;
     p.adapters = reinterpret_cast<const AdapterDev*>(base + o_ad);
     p.red = reinterpret_cast<const RedEntry*>(base + o_red);
     p.err_flag = reinterpret_cast<int*>(base);

@@ -89,13 +89,17 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtOp* __restrict
 
 // Copy adapter i's saved H block ([n][rp] rows of the saved buffer, pitch RP) to fp32 [n][rank].
 template <typename T>
+// out[t][p rank + k] = saved row h_row + t, column p rblk + k (block p of nblk output blocks).
 __global__ void unpack_saved_kernel(const T* __restrict__ saved, int64_t h_row, int RP, int n, int rank,
-                                    float* __restrict__ out) {
-    const int64_t total = (int64_t)n * rank;
+                                    int nblk, int rblk, float* __restrict__ out) {
+    const int width = nblk * rank;
+    const int64_t total = (int64_t)n * width;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = e / rank;
-        const int k = (int)(e % rank);
-        out[e] = to_f<T>(saved[(h_row + t) * RP + k]);
+        const int64_t t = e / width;
+        const int j = (int)(e - t * width);
+        const int pb = j / rank;
+        const int k = j - pb * rank;
+        out[e] = to_f<T>(saved[(h_row + t) * RP + pb * rblk + k]);
     }
 }
 

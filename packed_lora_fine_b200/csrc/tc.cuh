@@ -85,7 +85,18 @@ struct TcParams {
     int32_t fuse;
     int32_t stages;         // operand ring depth (<= kMaxStages)
     int32_t stage_bytes;    // bytes per ring stage: A tile + this op's largest B tile
+    // Output blocks (shared-input projections stacked along d_out): block b holds the output
+    // columns [blk_end[b-1], blk_end[b]); nblk = 1 for a single projection.
+    int32_t nblk;
+    int32_t blk_end[kMaxOutBlocks];
 };
+
+// The output block holding output column `col`.
+__device__ __forceinline__ int out_block(const TcParams& p, int col) {
+    int b = 0;
+    while (b + 1 < p.nblk && col >= p.blk_end[b]) ++b;
+    return b;
+}
 
 struct TileInfo {
     int32_t a_x, a_y, b_x, b_y;
@@ -168,11 +179,17 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         ti.red_idx = e;
         ti.a_x = db * kTileM;
         ti.a_y = re.x_row;
-        ti.b_x = 0;
         ti.b_y = re.h_row;
-        ti.nb_boxes = ad.rp64 / 64;
+        if constexpr (OP == Op::WgradB) {
+            // dB rows of output block b pair with block b's columns of H' only
+            ti.b_x = out_block(p, db * kTileM) * ad.rblk;
+            ti.mma_n = (ad.rblk + 63) / 64 * 64;
+        } else {
+            ti.b_x = 0;
+            ti.mma_n = ad.rp64;
+        }
+        ti.nb_boxes = ti.mma_n / 64;
         ti.kblocks = re.kblocks;
-        ti.mma_n = ad.rp64;
         ti.out_row = db * kTileM;
         ti.rows_valid = min(kTileM, p.M_total - ti.out_row);
         ti.n0 = db;  // the d-tile index (for partial slots)
@@ -261,11 +278,15 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
         // read at the tile's row offset inside j's zero-padded block (rows outside j's
         // segment load as zeros).  B has the base B's major-ness: for Y, rows n0.. of
         // j's row-padded B (K-major, one 256 x 64 box); for dX, j's packed A
-        // (MN-major, 16-row boxes so that only the rank's rows are staged).
+        // (MN-major, 16-row boxes so that only the rank's rows are staged).  With output
+        // blocks, Y's tile reads only its block's columns of H' (K = rblk from b rblk); dX's
+        // sums over every block (K = P rblk).
         for (int q = lr.q0; q < lr.q1; ++q) {
             const LoraSeg sg = mtile_seg(p, lr, q);
-            for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
-                const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
+            const int kext = Tr::kBmn ? sg.rp16 : sg.rblk;
+            const int hx0 = Tr::kBmn ? 0 : out_block(p, ti.n0) * sg.rblk;
+            for (int kb = 0; kb * kBlockK < kext; ++kb) {
+                const int R = min(kBlockK, kext - kb * kBlockK);
                 if (!ptx::mbar_wait(&empty_bar[rp.stage], rp.phase ^ 1u, abort_flag, lim, p.err_flag)) return false;
                 uint8_t* sA = smem + rp.stage * stb;
                 uint8_t* sB = sA + kABytes;
@@ -273,7 +294,7 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
                 ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], (uint32_t)kABytes + lb_bytes);
                 armed |= 1u << rp.stage;
                 armed_par = (armed_par & ~(1u << rp.stage)) | (rp.phase << rp.stage);
-                ptx::tma_load_2d(sA, tmA2, &full_bar[rp.stage], kb * kBlockK, sg.h_y);
+                ptx::tma_load_2d(sA, tmA2, &full_bar[rp.stage], hx0 + kb * kBlockK, sg.h_y);
                 if constexpr (Tr::kBmn) {
                     for (int h = 0; h < 4; ++h)
                         for (int r16 = 0; r16 < R; r16 += 16)
@@ -317,8 +338,9 @@ __device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, 
         const uint32_t idesc_lr = ptx::idesc_bf16_f32(kTileM, kTileN, false, Tr::kBmn);
         for (int q = lr.q0; q < lr.q1; ++q) {
             const LoraSeg sg = mtile_seg(p, lr, q);
-            for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
-                const int R = min(kBlockK, sg.rp16 - kb * kBlockK);
+            const int kext = Tr::kBmn ? sg.rp16 : sg.rblk;   // as the producer staged it
+            for (int kb = 0; kb * kBlockK < kext; ++kb) {
+                const int R = min(kBlockK, kext - kb * kBlockK);
                 if (!ptx::mbar_wait(&full_bar[rp.stage], rp.phase, abort_flag, lim, p.err_flag)) return false;
                 ptx::tc_fence_after();
                 const uint32_t sA = ptx::smem_u32(smem + rp.stage * stb);
@@ -487,8 +509,11 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
                 if (row_ok) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
+                        // column k of X^T G is block pb's rank row kk (rows pb rank + kk of dA)
                         const int k = c + e;
-                        if (k < rank) ad.dA[(int64_t)k * p.M_total + hid] = s * __uint_as_float(r[e]);
+                        const int pb = k / ad.rblk, kk = k - pb * ad.rblk;
+                        if (pb < p.nblk && kk < rank)
+                            ad.dA[(int64_t)(pb * rank + kk) * p.M_total + hid] = s * __uint_as_float(r[e]);
                     }
                 }
             }
@@ -496,6 +521,8 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
             // Split along the tokens: write this split's partial, the last split of the
             // tile to arrive sums all partials in split order (deterministic) and stores.
             const int64_t slot_elems = (int64_t)kTileM * p.RP;
+            // accumulator columns that reach an output: dB's rank, or every block's columns of dA
+            const int ncols = (OP == Op::WgradB || p.nblk == 1) ? rank : ad.rp16;
             // partial layout [slot][d-tile][rank column][128 rows]: a warp's lanes touch
             // consecutive rows, so both the writes here and the reduction below coalesce.
             float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems + row;
@@ -505,7 +532,7 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
                 ptx::tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    if (c + e < rank) mine[(int64_t)(c + e) * kTileM] = __uint_as_float(r[e]);
+                    if (c + e < ncols) mine[(int64_t)(c + e) * kTileM] = __uint_as_float(r[e]);
             }
             __threadfence();
             ptx::named_bar_sync(1, 128);
@@ -519,7 +546,7 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
                 if (row_ok) {
                     const float* first = p.partials + ((int64_t)re.slot * p.red_dtiles + ti.n0) * slot_elems + row;
                     const int64_t split_stride = (int64_t)p.red_dtiles * slot_elems;
-                    for (int k0 = 0; k0 < rank; k0 += 8) {
+                    for (int k0 = 0; k0 < ncols; k0 += 8) {
                         // 8 ranks at a time: all of a split's loads are in flight together,
                         // the sum still runs over the splits in order.
                         float acc[8];
@@ -529,16 +556,19 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
                             float v[8];
 #pragma unroll
                             for (int u = 0; u < 8; ++u)
-                                v[u] = (k0 + u < rank) ? __ldcg(first + sp * split_stride + (int64_t)(k0 + u) * kTileM) : 0.f;
+                                v[u] = (k0 + u < ncols) ? __ldcg(first + sp * split_stride + (int64_t)(k0 + u) * kTileM) : 0.f;
 #pragma unroll
                             for (int u = 0; u < 8; ++u) acc[u] += v[u];
                         }
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
                             const int k = k0 + u;
-                            if (k < rank) {
-                                if constexpr (OP == Op::WgradB) ad.dB[(int64_t)hid * rank + k] = s * acc[u];
-                                else ad.dA[(int64_t)k * p.M_total + hid] = s * acc[u];
+                            if constexpr (OP == Op::WgradB) {
+                                if (k < rank) ad.dB[(int64_t)hid * rank + k] = s * acc[u];
+                            } else {
+                                const int pb = k / ad.rblk, kk = k - pb * ad.rblk;
+                                if (pb < p.nblk && kk < rank)
+                                    ad.dA[(int64_t)(pb * rank + kk) * p.M_total + hid] = s * acc[u];
                             }
                         }
                     }
@@ -693,8 +723,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
 // ---------------------------------------------------------------------------
 // Packing of the small per-adapter factors into the MMA-ready padded layouts.
-//   packA [n*RP][d_in]:  row i*RP + k = A_i[k][:]       (k < r_i), zero for r_i <= k < rp16_i
-//   packBT[n*RP][d_out]: row i*RP + k = B_i[:][k]       (k < r_i), zero for r_i <= k < rp16_i
+//   packA [n*RP][d_in]:  row i*RP + b*rblk_i + k = A_i[b*r_i + k][:] (k < r_i), zero up to rblk_i
+//   packBT[n*RP][d_out]: row i*RP + b*rblk_i + k = B_i[:][k] on block b's columns (k < r_i), else zero
+// (b = output block, rblk_i = r_i rounded up to 16; one block: b = 0 and rblk_i = rp16_i).
 // Rows rp16_i <= k < RP are never read by an MMA and are left unwritten.
 // ---------------------------------------------------------------------------
 __global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, int64_t d_in,
@@ -705,24 +736,27 @@ __global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, 
         const int64_t rowi = e / vec_per_row;
         const int64_t v = e - rowi * vec_per_row;
         const int i = (int)(rowi / RP);
-        const int k = (int)(rowi - (int64_t)i * RP);
-        if (k >= ad[i].rp16) continue;   // rows past the MMA extent are never read
+        const int j = (int)(rowi - (int64_t)i * RP);
+        if (j >= ad[i].rp16) continue;   // rows past the MMA extent are never read
+        // row j is output block pb's rank row k (A_store row pb rank + k)
+        const int pb = j / ad[i].rblk, k = j - pb * ad[i].rblk;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (k < ad[i].rank)
-            val = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ad[i].A) + (int64_t)k * d_in)[v];
+            val = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ad[i].A) +
+                                                 (int64_t)(pb * ad[i].rank + k) * d_in)[v];
         reinterpret_cast<uint4*>(packA + rowi * d_in)[v] = val;
     }
 }
 
 // Row-padded copy of every B for the fused forward (the expand's B operand, K-major like W):
-// packB[(i d_out + c) RP + k] = B_i[c][k] for k < r_i, 0 for r_i <= k < rp16_i; columns at or
-// past rp16_i are never multiplied and stay unwritten.  grid.y = adapter; one thread per 16-byte
+// packB[(i d_out + c) RP + k] = B_i[c][k] for k < r_i, 0 for r_i <= k < rblk_i (r_i rounded up to
+// 16); columns at or past rblk_i are never multiplied and stay unwritten.  grid.y = adapter; one thread per 16-byte
 // chunk of the rp16_i columns, so consecutive threads read consecutive bytes of B_i.
 __global__ void __launch_bounds__(256) pack_b_kernel(const AdapterDev* __restrict__ ad, int RP, int d_out,
                                                      __nv_bfloat16* __restrict__ packB) {
     const int i = blockIdx.y;
     const int r = ad[i].rank;
-    const unsigned vc = (unsigned)ad[i].rp16 / 8u;          // chunks per row
+    const unsigned vc = (unsigned)ad[i].rblk / 8u;          // chunks per row
     const unsigned total = (unsigned)d_out * vc;
     const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(ad[i].B);
     __nv_bfloat16* dst = packB + (int64_t)i * d_out * RP;
@@ -749,7 +783,7 @@ __global__ void __launch_bounds__(256) pack_b_kernel(const AdapterDev* __restric
 // grid: (ceil(d_out/128), n); block 256.  Stages B_i[c0..c0+127][0..r) in shared memory (dynamic,
 // 128 x (r + 2) bf16), then writes rows k < rp16 of packBT, 128 columns each.
 __global__ void __launch_bounds__(256) pack_bt_kernel(const AdapterDev* __restrict__ ad, int RP, int64_t d_out,
-                                                      __nv_bfloat16* __restrict__ packBT) {
+                                                      OutBlocks blocks, __nv_bfloat16* __restrict__ packBT) {
     extern __shared__ __nv_bfloat16 tile[];
     const int i = blockIdx.y;
     const int64_t c0 = (int64_t)blockIdx.x * 128;
@@ -775,14 +809,22 @@ __global__ void __launch_bounds__(256) pack_bt_kernel(const AdapterDev* __restri
         }
     }
     __syncthreads();
+    // With output blocks the pack is block-diagonal: row pb rblk + k holds B's column k on block
+    // pb's output columns and zeros elsewhere, so block pb of G sums over block pb's columns only.
+    // A 128-column tile lies in one block (block ends are multiples of 256).
+    int cb = 0;
+    while (cb + 1 < blocks.n && c0 >= blocks.end[cb]) ++cb;
+    const int rblk = ad[i].rblk;
     const int rows = ad[i].rp16;   // rows past the MMA extent are never read
     for (int e = threadIdx.x; e < rows * 64; e += blockDim.x) {
-        const int k = e >> 6, cc = (e & 63) * 2;
+        const int j = e >> 6, cc = (e & 63) * 2;
+        const int pb = j / rblk, k = j - pb * rblk;
+        const bool live = pb == cb && k < r;
         if (cc < cols) {
             __nv_bfloat162 v;
-            v.x = (k < r) ? tile[cc * ld + k] : __float2bfloat16_rn(0.f);
-            v.y = (k < r) ? tile[(cc + 1) * ld + k] : __float2bfloat16_rn(0.f);
-            *reinterpret_cast<__nv_bfloat162*>(packBT + ((int64_t)i * RP + k) * d_out + c0 + cc) = v;
+            v.x = live ? tile[cc * ld + k] : __float2bfloat16_rn(0.f);
+            v.y = live ? tile[(cc + 1) * ld + k] : __float2bfloat16_rn(0.f);
+            *reinterpret_cast<__nv_bfloat162*>(packBT + ((int64_t)i * RP + j) * d_out + c0 + cc) = v;
         }
     }
 }

@@ -61,6 +61,43 @@ def test_create_rejects_bad_config(c, want):
     assert s == want and not h
 
 
+def blocked_cfg(widths, d_out=None, **kw):
+    c = cfg(d_out=d_out if d_out is not None else sum(widths), **kw)
+    end = 0
+    c.n_out_blocks = len(widths)
+    for b, w in enumerate(widths[:pl.PLORA_MAX_OUT_BLOCKS]):
+        end += w
+        c.out_block_end[b] = end
+    return c
+
+
+@pytest.mark.parametrize("c, want", [
+    (blocked_cfg([200, 312]), pl.PLORA_ERR_INVALID_ARG),                 # a block end not a multiple of 256
+    (blocked_cfg([256, 512], d_out=512), pl.PLORA_ERR_INVALID_ARG),      # ends past d_out
+    (blocked_cfg([256, 256, 256], max_rank=96), pl.PLORA_ERR_INVALID_ARG),  # 3 x 96 padded ranks > 256
+    (blocked_cfg([256] * 9), pl.PLORA_ERR_INVALID_ARG),                  # more than 8 blocks
+    (blocked_cfg([256, 256], dtype=pl.PLORA_FP32), pl.PLORA_ERR_UNSUPPORTED),
+    (blocked_cfg([256, 256], flags=pl.PLORA_FLAG_SIMT), pl.PLORA_ERR_UNSUPPORTED),
+    (blocked_cfg([256, 256], flags=pl.PLORA_FLAG_UNFUSED), pl.PLORA_ERR_UNSUPPORTED),
+    (blocked_cfg([256, 256], flags=pl.PLORA_FLAG_BASE_PAIR), pl.PLORA_ERR_UNSUPPORTED),
+])
+def test_create_rejects_bad_output_blocks(c, want):
+    s, h = pl.plora_create_status(c)
+    assert s == want and not h
+
+
+def test_output_blocks_widen_the_padded_rank():
+    # rank 24 per block: each block's columns of H' are 32 wide (24 rounded up to 16), so three
+    # blocks need 96 columns and the saved / G pitch RP rounds that up to 128
+    off = np.array([0, 100], np.int64)
+    c1, c3 = cfg(d_out=768, max_rank=64), blocked_cfg([256, 256, 256], max_rank=64)
+    for c, want in ((c1, 64), (c3, 128)):
+        s, v = pl.plora_debug_schedule(c, 1, off, fake_table([24]), False, 3)
+        assert s == pl.PLORA_OK and v[0] == want
+    s, v = pl.plora_debug_schedule(c3, 1, off, fake_table([24]), False, 2)
+    assert s == pl.PLORA_OK
+
+
 def test_create_without_gpu_fails_loudly():
     import torch
     if torch.cuda.is_available():
