@@ -701,8 +701,11 @@ def run_suite(args):
             return e0.elapsed_time(e1) / steps, prof
 
         steps = max(5, min(args.steps, 30))
-        ms_p, prof = timed(packed_step, steps, profile=True)
+        # both loops timed without the per-launch profiling events (they cost microseconds per
+        # launch, which shows on the small workloads); the kernel breakdown comes from its own pass
+        ms_p, _ = timed(packed_step, steps)
         ms_s, _ = timed(seq_step, max(3, steps // 3))
+        _, prof = timed(packed_step, steps, profile=True)
         kern = {}
         for k, (c, tot) in prof.items():
             if c:

@@ -96,3 +96,40 @@ def test_adamw_rejects_bad_state():
     torch.cuda.synchronize()
     assert not torch.any(Am) and not torch.any(A)       # nothing written
     eng.close()
+
+
+def test_adamw_step_with_output_blocks():
+    # with P output blocks A (and its master, moments, gradient) is [P r][d_in]; the update is
+    # elementwise, so it matches the oracle step on the whole stacked tensor
+    d_in, widths, ranks = 136, [256, 256], [8, 16]
+    rng = np.random.default_rng(12)
+    eng = pl.PackedLoRA(d_in, sum(widths), "bf16", max_adapters=2, max_rank=16, max_tokens=16, out_blocks=widths)
+    t = lambda a: torch.from_numpy(a).to("cuda")
+    hp = [HP[0], HP[1]]
+    A16, B16, Am, Bm, mA, vA, mB, vB, dA, dB, host = ([] for _ in range(11))
+    for r in ranks:
+        h = dict(A=_draw(rng, (2 * r, d_in), 0.05), B=_draw(rng, (sum(widths), r), 0.05),
+                 mA=_draw(rng, (2 * r, d_in), 1e-3), vA=np.abs(_draw(rng, (2 * r, d_in), 1e-4)),
+                 mB=_draw(rng, (sum(widths), r), 1e-3), vB=np.abs(_draw(rng, (sum(widths), r), 1e-4)),
+                 gA=_draw(rng, (2 * r, d_in), 1e-2), gB=_draw(rng, (sum(widths), r), 1e-2))
+        host.append(h)
+        A16.append(torch.empty((2 * r, d_in), dtype=torch.bfloat16, device="cuda"))
+        B16.append(torch.empty((sum(widths), r), dtype=torch.bfloat16, device="cuda"))
+        Am.append(t(h["A"])); Bm.append(t(h["B"]))
+        mA.append(t(h["mA"])); vA.append(t(h["vA"])); mB.append(t(h["mB"])); vB.append(t(h["vB"]))
+        dA.append(t(h["gA"])); dB.append(t(h["gB"]))
+    tab = eng.table([1.0, 1.0], A16, B16, dA, dB)
+    st = pl.make_adamw_states(hp, [x.data_ptr() for x in Am], [x.data_ptr() for x in Bm],
+                              [x.data_ptr() for x in mA], [x.data_ptr() for x in vA],
+                              [x.data_ptr() for x in mB], [x.data_ptr() for x in vB])
+    pl.plora_adamw_step(eng.h, 2, tab, st, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert pl.plora_check(eng.h, 0) == pl.PLORA_OK
+    for i, h in enumerate(host):
+        for name, g, m, v, pdev, copy in (("A", h["gA"], mA[i], vA[i], Am[i], A16[i]),
+                                          ("B", h["gB"], mB[i], vB[i], Bm[i], B16[i])):
+            p_ref, m_ref, v_ref = oracle.adamw(h[name], h["m" + name], h["v" + name], g, **hp[i])
+            assert rel_err(pdev.cpu().numpy(), p_ref) <= TOL, (i, name)
+            assert rel_err(m.cpu().numpy(), m_ref) <= TOL and rel_err(v.cpu().numpy(), v_ref) <= TOL, (i, name)
+            assert np.array_equal(copy.view(torch.uint16).cpu().numpy(), wl.f32_to_bf16_bits(pdev.cpu().numpy()))
+    eng.close()
