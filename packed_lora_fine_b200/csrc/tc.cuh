@@ -12,7 +12,7 @@
 //   ShrinkX    H_i = X_i A_i       (per 128-token tile)   X      K-major          A pack     K-major
 //   ShrinkDy   G_i = s_i dY_i B_i^T                       dY     K-major          B^T pack   K-major
 //   ExpandY    Y_i += s_i H_i B_i                         H      K-major          B^T pack   MN-major
-//              (folded into BaseFwd instead: B row-padded pack, K-major)
+//              (by default folded into BaseFwd instead: B row-padded pack, K-major)
 //   ExpandDx   dX_i += G_i A_i^T                          G      K-major          A pack     MN-major
 //   WgradB     dB_i = s_i dY_i^T H_i (sum over tokens)    dY     MN-major         H          MN-major
 //   WgradA     dA_i = X_i^T G_i      (sum over tokens)    X      MN-major         G          MN-major
@@ -28,6 +28,16 @@
 // warp 1 owns TMEM and issues tcgen05.mma into one of two 128x256 fp32
 // accumulators, warps 2-5 drain an accumulator (tcgen05.ld) and run the
 // op's epilogue while the next tile is being multiplied.
+//
+// A launch may carry a second, independent op (tc_kernel<OP, OP2>): its work
+// items follow OP's in the same persistent grid (the backward runs dB's items
+// after G's, filling the last wave of G's equal-cost token tiles).
+//
+// Output blocks: W may stack P projections that read the same X (q|k|v).  Each
+// adapter then has one rank-r pair per block; H' and G hold block b in columns
+// [b rblk, b rblk + r).  Y's folded product and dB read only their block's
+// columns; G (through a block-diagonal B^T pack) and the folded dX product
+// span all of them.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
