@@ -233,6 +233,17 @@ def time_oracle(p, nthreads: int) -> float:
     return time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(seed: int) -> dict:
     import oracle
     oracle.build()
@@ -241,7 +252,7 @@ def cpu_baseline(seed: int) -> dict:
     p = oracle_sample_problem(seed, 8, 4)
     time_oracle(oracle_sample_problem(seed, 1, 1), nt)  # load / page in
     dt = time_oracle(p, nt)
-    return {"value": p.T / dt, "unit": UNIT, "cores": nt, "kind": "oracle",
+    return {"value": p.T / dt, "unit": UNIT, "cores": nt, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"fp64 oracle fwd+bwd (Y, dX, dA, dB) of {p.T} tokens: the first 8 adapters of the "
                       f"32-adapter LLaMA-3-8B up_proj mix cut to 4 tokens each; {dt:.2f} s"}
 
@@ -385,6 +396,22 @@ def main(argv=None):
     prof = pl.plora_profile_read(eng.h)
     pl.plora_profile_enable(eng.h, False)
     assert pl.plora_check(eng.h, st) == pl.PLORA_OK
+
+    # The same steps with L2 flushed before each one (a 256 MB write, twice the L2): each step is
+    # timed on its own between events, so the flush stays outside the timed time.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    k_fl = max(3, min(args.steps, 10))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k_fl)]
+    barrier()
+    for a_, b_ in evs:
+        flush.fill_(1)
+        a_.record(stream)
+        step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms_flushed = reduce_max(sum(a_.elapsed_time(b_) for a_, b_ in evs) / k_fl, dist)
+    del flush
+    assert pl.plora_check(eng.h, st) == pl.PLORA_OK
     ms = reduce_max(ms_local, dist)
     tokens_all = reduce_sum(T, dist)
     # every rank takes part in both sums; a rank without an energy counter turns them into NaN
@@ -518,7 +545,10 @@ def main(argv=None):
                            "base_gemm": base_gemm},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
                 "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
-                "energy": energy_line, "kernels": kernels}
+                "energy": energy_line,
+                "l2_flushed": {"value": tokens_all / (ms_flushed / 1000.0), "unit": UNIT, "ms_per_step": ms_flushed,
+                               "steps": k_fl, "how": "256 MB written before each step, outside its timed region"},
+                "kernels": kernels}
         print(json.dumps(line), flush=True)
     eng.close()
     if dist is not None:

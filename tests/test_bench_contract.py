@@ -50,4 +50,6 @@ def test_library_arm_line():
     assert d["gpu_launches"] == 3 * 11     # 11 launches per fwd+bwd step
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1 and cb["cpu_model"]
+    fl = d["l2_flushed"]                   # the same steps with L2 flushed before each one
+    assert fl["value"] > 0 and fl["ms_per_step"] > 0 and fl["unit"] == d["unit"]
