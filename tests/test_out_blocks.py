@@ -112,3 +112,41 @@ def test_output_blocks_equal_separate_calls_bit_for_bit():
             assert np.array_equal(g["dB"][i][cols], h["dB"][i]), (b, i)
         dX_sum = dX_sum + h["dX"]
     assert rel_err(g["dX"], dX_sum) <= BF16_TOL
+
+
+def test_output_blocks_llama_qkv_sampled():
+    # LLaMA-3-8B q|k|v (4096 -> 4096 + 1024 + 1024), 16 adapters, r ~ U{16,32,64}, long-tail segment
+    # lengths; each block against the oracle on sampled rows of Y / dX and sampled columns of dA / dB
+    d_in, widths = 4096, [4096, 1024, 1024]
+    rng = np.random.default_rng(31)
+    ranks = rng.choice(np.array([16, 32, 64]), size=16)
+    counts = np.round(np.exp(rng.uniform(np.log(256), np.log(2048), size=16))).astype(np.int64)
+    r = np.asarray(ranks)
+    d_out = sum(widths)
+    base = wl.make_problem("qkv", "bf16", d_in, d_out, r, counts, 2.0 * r, wl.init_llm(d_in), 1201)
+    # the k and v blocks' A factors (A depends on d_in and the ranks only; a 1-token draw suffices)
+    extra = [wl.make_problem(f"qkv{b}", "bf16", d_in, 8, r, [1] * 16, 2.0 * r, wl.init_llm(d_in), 1201 + 100 * b).A
+             for b in (1, 2)]
+    A_blocks = [base.A] + extra
+    stacked = dataclasses.replace(base, A=[np.concatenate([A_blocks[b][i] for b in range(3)]) for i in range(16)])
+    eng = pl.PackedLoRA(d_in, d_out, "bf16", max_adapters=16, max_rank=64, max_tokens=stacked.T, out_blocks=widths)
+    g = run(stacked, engine=eng)
+    eng.close()
+    rows = wl.sample_rows(stacked, per_segment=2)
+    cols_a = np.unique(rng.integers(0, d_in, 48))
+    nt = oracle.num_procs()
+    dX_ref, c0 = 0.0, 0
+    for b, w in enumerate(widths):
+        cols = slice(c0, c0 + w)
+        pb = dataclasses.replace(base, d_out=w, W=base.W[cols], dY=base.dY[:, cols], A=A_blocks[b],
+                                 B=[x[cols] for x in base.B])
+        cols_b = np.unique(rng.integers(0, w, 48))
+        assert rel_err(g["Y"][rows][:, cols], oracle.forward(pb, rows=rows, nthreads=nt)["Y"]) <= BF16_TOL, b
+        dX_ref = dX_ref + oracle.input_grad(pb, rows=rows, nthreads=nt)["dX"]
+        o = oracle.weight_grads(pb, nthreads=nt, cols_a=cols_a, cols_b=cols_b)
+        for i, ri in enumerate(r):
+            ri = int(ri)
+            assert rel_err(g["dA"][i][b * ri:(b + 1) * ri][:, cols_a], o["dA"][i][:, cols_a]) <= BF16_TOL, (b, i)
+            assert rel_err(g["dB"][i][cols][cols_b], o["dB"][i][cols_b]) <= BF16_TOL, (b, i)
+        c0 += w
+    assert rel_err(g["dX"][rows], dX_ref) <= BF16_TOL

@@ -222,10 +222,12 @@ def test_config2_qwen_q_proj():
     assert not bad, (bad, errs)
 
 
-def test_config3_llama_up_proj_32_adapters():
-    """The benchmark workload (LLaMA-3-8B up_proj, 32 long-tail adapters) on sampled outputs."""
+@pytest.mark.parametrize("path", ["tc", "tc_pair"])
+def test_config3_llama_up_proj_32_adapters(path):
+    """The benchmark workload (LLaMA-3-8B up_proj, 32 long-tail adapters) on sampled outputs, with the
+    base GEMMs on single SMs (the default) and on SM pairs."""
     p = wl.config3()
-    g = run(p)
+    g = run(p, base_pair=(path == "tc_pair"))
     rows = wl.sample_rows(p, per_segment=2)
     rng = np.random.default_rng(6)
     cols_a = np.unique(rng.integers(0, p.d_in, 64))
