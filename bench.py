@@ -513,7 +513,7 @@ def main(argv=None):
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        k2 = max(5, min(args.steps, 20))
+        k2 = max(5, min(args.steps, 50))   # the pipeline fill (one uncovered copy) spreads over k2 steps
         e0.record(stream)
         s_in.wait_stream(stream)
         s_out.wait_stream(stream)
