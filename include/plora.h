@@ -283,6 +283,23 @@ PLORA_API plora_status plora_adamw_step(plora_handle h, int32_t n_adapters, cons
                                         const plora_adamw_state* st, void* stream);
 
 /*
+ * CUDA graph capture (a runtime facility; the pages describe no API).  A plora_forward,
+ * plora_backward or plora_adamw_step called while its stream is being captured
+ * (cudaStreamBeginCapture, torch.cuda.graph) takes one schedule slot reserved here instead
+ * of the handle's ring, and keeps it: every replay of the graph re-copies that call's
+ * schedule from the slot, which no later call overwrites.  Reserve before the capture begins
+ * (these calls allocate: n pinned host buffers and n device buffers, each as large as one
+ * call's schedule staging); a call captured with no reserved slot left returns
+ * PLORA_ERR_INVALID_ARG and enqueues nothing.  Captured calls record no profiling events.
+ * Replays and eager calls share the handle's workspace, so as for eager calls only one runs at
+ * a time per handle.  plora_capture_release synchronises the device and frees every capture
+ * slot: call it only once no graph that holds captured calls of this handle will replay again.
+ * plora_destroy frees them too.
+ */
+PLORA_API plora_status plora_capture_reserve(plora_handle h, int32_t n);
+PLORA_API plora_status plora_capture_release(plora_handle h);
+
+/*
  * Launch geometry of the handle's device (a diagnostic; the method itself has no such
  * call): out[0] = SMs, out[1] / out[2] = the 2-SM clusters that can be resident at once
  * for the SM-pair Y / dX base GEMMs (PLORA_FLAG_BASE_PAIR), each <= SMs / 2.  At most

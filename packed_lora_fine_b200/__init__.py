@@ -41,7 +41,8 @@ PLORA_STATIC_SCRATCH_BYTES = 16 << 20
 EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
-            "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe", "plora_device_info")
+            "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe", "plora_device_info",
+            "plora_capture_reserve", "plora_capture_release")
 
 
 class plora_config(ctypes.Structure):
@@ -113,6 +114,10 @@ def load(path: str = LIB_PATH):
     lib.plora_profile_enable.restype = ctypes.c_int
     lib.plora_profile_read.argtypes = [H, I32, ctypes.POINTER(I32), P, P, P]
     lib.plora_profile_read.restype = ctypes.c_int
+    lib.plora_capture_reserve.argtypes = [H, I32]
+    lib.plora_capture_reserve.restype = ctypes.c_int
+    lib.plora_capture_release.argtypes = [H]
+    lib.plora_capture_release.restype = ctypes.c_int
     lib.plora_device_info.argtypes = [H, P, I32, ctypes.POINTER(I32)]
     lib.plora_device_info.restype = ctypes.c_int
     lib.plora_debug_timeout_probe.argtypes = [H, I64, P]
@@ -251,6 +256,16 @@ def plora_profile_read(h: int) -> dict:
     ms = (ctypes.c_double * cap)()
     _raise(h, lib.plora_profile_read(h, cap, ctypes.byref(n), names, launches, ms))
     return {names[k].decode(): (int(launches[k]), float(ms[k])) for k in range(min(n.value, cap))}
+
+
+def plora_capture_reserve(h: int, n: int) -> None:
+    """Reserve n schedule slots for calls captured into CUDA graphs (one per captured call)."""
+    _raise(h, load().plora_capture_reserve(h, int(n)))
+
+
+def plora_capture_release(h: int) -> None:
+    """Free the capture slots (only once no graph holding this handle's captured calls replays)."""
+    _raise(h, load().plora_capture_release(h))
 
 
 def plora_device_info(h: int) -> dict:

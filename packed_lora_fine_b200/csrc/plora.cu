@@ -57,6 +57,17 @@ struct plora_ctx {
 
     uint8_t* h_blob[kSlots] = {};       // mapped pinned staging of each slot (host view)
     uint8_t* h_blob_dev[kSlots] = {};   // the same buffers as the device addresses them
+    // Schedule slots for calls made while their stream is being captured into a CUDA graph: each
+    // captured call keeps its slot (staging and device copy) until plora_capture_release, so every
+    // replay of the graph re-runs its staging copy from buffers no later call overwrites.
+    struct CaptureSlot {
+        uint8_t* host = nullptr;
+        uint8_t* host_dev = nullptr;
+        uint8_t* dev = nullptr;
+    };
+    std::vector<CaptureSlot> cap;
+    size_t cap_next = 0;
+    bool in_capture = false;   // the current call's stream is capturing (no profiling events then)
     cudaEvent_t ev[kSlots] = {};
     int next_slot = 0;
 
@@ -171,7 +182,7 @@ cudaEvent_t take_event(plora_ctx* h) {
 template <typename F>
 void tracked(plora_ctx* h, int kind, cudaStream_t st, F&& launch) {
     h->launches[kind] += 1;
-    if (!h->profiling) {
+    if (!h->profiling || h->in_capture) {
         launch();
         return;
     }
@@ -379,29 +390,67 @@ __global__ void stage_copy_kernel(const uint4* __restrict__ src, uint4* __restri
         dst[i] = src[i];
 }
 
-// `bytes` of slot `slot`'s staging into device memory at d (rounded up to 16 bytes; the staging and
-// the device region are both whole multiples of 256 bytes).
-cudaError_t stage_copy(plora_ctx* h, int slot, uint8_t* d, size_t bytes, cudaStream_t st) {
+// `bytes` of staging (device view `src`) into device memory at d (rounded up to 16 bytes; the
+// staging and the device region are both whole multiples of 256 bytes).
+cudaError_t stage_copy(plora_ctx* h, const uint8_t* src, uint8_t* d, size_t bytes, cudaStream_t st) {
     const int64_t n16 = (int64_t)((bytes + 15) / 16);
     if (n16 == 0) return cudaSuccess;
     const int blocks = (int)std::min<int64_t>(ceil_div(n16, 256), 64);
     tracked(h, kStage, st, [&] {
-        stage_copy_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(h->h_blob_dev[slot]),
-                                                  reinterpret_cast<uint4*>(d), n16);
+        stage_copy_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(d),
+                                                  n16);
     });
     return cudaGetLastError();
 }
 
-plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& ops, cudaStream_t st,
-                    DevPlan& D) {
+bool stream_capturing(cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    return cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive;
+}
+
+// The schedule slot of the current call: the next ring slot once its previous use has finished, or,
+// while the stream is being captured, the next reserved capture slot (slot index -1 - k).
+struct Slot {
+    int index = 0;
+    uint8_t* host = nullptr;
+    const uint8_t* host_dev = nullptr;
+    uint8_t* dev = nullptr;
+};
+
+plora_status take_slot(plora_ctx* h, cudaStream_t st, Slot& sl) {
+    h->in_capture = stream_capturing(st);
+    if (h->in_capture) {
+        if (h->cap_next >= h->cap.size())
+            return fail(h, PLORA_ERR_INVALID_ARG, "the stream is being captured and no reserved schedule slot is "
+                        "left (plora_capture_reserve before the capture)");
+        const plora_ctx::CaptureSlot& c = h->cap[h->cap_next];
+        sl.index = -1 - (int)h->cap_next;
+        ++h->cap_next;
+        sl.host = c.host;
+        sl.host_dev = c.host_dev;
+        sl.dev = c.dev;
+        return PLORA_OK;
+    }
     const int slot = h->next_slot;
     h->next_slot = (h->next_slot + 1) % kSlots;
     cudaError_t e = cudaEventSynchronize(h->ev[slot]);
     if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize(staging slot)");
+    sl.index = slot;
+    sl.host = h->h_blob[slot];
+    sl.host_dev = h->h_blob_dev[slot];
+    sl.dev = h->at<uint8_t>(h->r_blob[slot]);
+    return PLORA_OK;
+}
+
+plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& ops, cudaStream_t st,
+                    DevPlan& D) {
+    Slot sl;
+    plora_status ps = take_slot(h, st, sl);
+    if (ps != PLORA_OK) return ps;
     size_t o = 0;
     auto put = [&](const void* src, size_t bytes) {
         const size_t at = o;
-        if (bytes) memcpy(h->h_blob[slot] + at, src, bytes);
+        if (bytes) memcpy(sl.host + at, src, bytes);
         o = round_up((int64_t)(o + bytes), 256);
         return at;
     };
@@ -412,8 +461,8 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     const size_t o_mto = put(P.mt_rec.data(), P.mt_rec.size() * sizeof(MTileRec));
     const size_t o_mtl = put(P.mt_seg.data(), P.mt_seg.size() * sizeof(LoraSeg));
     if (o > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "schedule exceeds the handle's staging size");
-    uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
-    e = stage_copy(h, slot, d, o, st);
+    uint8_t* d = sl.dev;
+    cudaError_t e = stage_copy(h, sl.host_dev, d, o, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "copying the schedule to the device");
     D.ad = reinterpret_cast<AdapterDev*>(d + o_ad);
     D.tok = reinterpret_cast<TokTile*>(d + o_tok);
@@ -421,36 +470,37 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     D.ops = reinterpret_cast<SimtOp*>(d + o_ops);
     D.mt_rec = reinterpret_cast<MTileRec*>(d + o_mto);
     D.mt_seg = reinterpret_cast<LoraSeg*>(d + o_mtl);
-    D.slot = slot;
+    D.slot = sl.index;
     return PLORA_OK;
 }
 
 // Copy two host arrays to the device through the staging ring (same slot discipline as upload()).
 plora_status upload_parts(plora_ctx* h, const void* a, size_t na, const void* b, size_t nb, cudaStream_t st,
                           uint8_t** da, uint8_t** db, int* slot_out) {
-    const int slot = h->next_slot;
-    h->next_slot = (h->next_slot + 1) % kSlots;
-    cudaError_t e = cudaEventSynchronize(h->ev[slot]);
-    if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize(staging slot)");
     const size_t ob = (size_t)round_up((int64_t)na, 256);
     const size_t total = ob + nb;
     if (total > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "optimizer tables exceed the staging size");
-    if (na) memcpy(h->h_blob[slot], a, na);
-    if (nb) memcpy(h->h_blob[slot] + ob, b, nb);
-    uint8_t* d = h->at<uint8_t>(h->r_blob[slot]);
-    e = stage_copy(h, slot, d, total, st);
+    Slot sl;
+    plora_status ps = take_slot(h, st, sl);
+    if (ps != PLORA_OK) return ps;
+    if (na) memcpy(sl.host, a, na);
+    if (nb) memcpy(sl.host + ob, b, nb);
+    uint8_t* d = sl.dev;
+    cudaError_t e = stage_copy(h, sl.host_dev, d, total, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "copying the optimizer tables to the device");
     *da = d;
     *db = d + ob;
-    *slot_out = slot;
+    *slot_out = sl.index;
     return PLORA_OK;
 }
 
 plora_status finish(plora_ctx* h, const DevPlan& D, cudaStream_t st) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
-    e = cudaEventRecord(h->ev[D.slot], st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    if (D.slot >= 0) {   // a ring slot: its event guards reuse (a capture slot is never reused)
+        e = cudaEventRecord(h->ev[D.slot], st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+    }
     return PLORA_OK;
 }
 
@@ -779,8 +829,51 @@ plora_status plora_destroy(plora_handle h) {
         cudaEventDestroy(r.b);
     }
     for (cudaEvent_t e : h->pool) cudaEventDestroy(e);
+    for (const plora_ctx::CaptureSlot& c : h->cap) {
+        if (c.host) cudaFreeHost(c.host);
+        if (c.dev) cudaFree(c.dev);
+    }
     if (h->ws) cudaFree(h->ws);
     delete h;
+    return PLORA_OK;
+}
+
+plora_status plora_capture_reserve(plora_handle h, int32_t n) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    if (n < 0 || n > 4096) return fail(h, PLORA_ERR_INVALID_ARG, "n=%d outside [0, 4096]", n);
+    cudaError_t e = cudaSetDevice(h->device);
+    for (int32_t k = 0; k < n && e == cudaSuccess; ++k) {
+        plora_ctx::CaptureSlot c;
+        e = cudaHostAlloc(&c.host, h->blob_bytes, cudaHostAllocMapped | cudaHostAllocPortable);
+        if (e == cudaSuccess) e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&c.host_dev), c.host, 0);
+        if (e == cudaSuccess) e = cudaMalloc(&c.dev, h->blob_bytes);
+        if (e != cudaSuccess) {
+            if (c.host) cudaFreeHost(c.host);
+            if (c.dev) cudaFree(c.dev);
+            cudaGetLastError();
+            break;
+        }
+        h->cap.push_back(c);
+    }
+    if (e != cudaSuccess)
+        return e == cudaErrorMemoryAllocation ? fail(h, PLORA_ERR_OOM, "capture slots: out of memory")
+                                              : cuda_fail(h, e, "reserving capture slots");
+    return PLORA_OK;
+}
+
+plora_status plora_capture_release(plora_handle h) {
+    if (!h) return PLORA_ERR_INVALID_ARG;
+    h->last_error.clear();
+    cudaError_t e = cudaSetDevice(h->device);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(h, e, "synchronising before releasing capture slots");
+    for (const plora_ctx::CaptureSlot& c : h->cap) {
+        if (c.host) cudaFreeHost(c.host);
+        if (c.dev) cudaFree(c.dev);
+    }
+    h->cap.clear();
+    h->cap_next = 0;
     return PLORA_OK;
 }
 

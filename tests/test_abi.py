@@ -114,6 +114,8 @@ def test_null_handle_calls_are_rejected():
     assert lib.plora_device_info(None, ctypes.cast(out, ctypes.c_void_p), 3, ctypes.byref(cnt)) == pl.PLORA_ERR_INVALID_ARG
     assert cnt.value == -1
     assert lib.plora_profile_enable(None, 1) == pl.PLORA_ERR_INVALID_ARG
+    assert lib.plora_capture_reserve(None, 1) == pl.PLORA_ERR_INVALID_ARG
+    assert lib.plora_capture_release(None) == pl.PLORA_ERR_INVALID_ARG
     assert lib.plora_check(None, None) == pl.PLORA_ERR_INVALID_ARG
 
 
