@@ -238,3 +238,42 @@ def test_config3_llama_up_proj_32_adapters(path):
     o.update(oracle.weight_grads(p, nthreads=nt, cols_a=cols_a, cols_b=cols_b))
     errs, bad = compare(p, g, o, BF16_TOL, rows=rows, cols_a=cols_a, cols_b=cols_b)
     assert not bad, (bad, errs)
+
+
+def sampled_check(p, g, per_segment=2, ncols=48, seed=8):
+    rows = wl.sample_rows(p, per_segment=per_segment)
+    rng = np.random.default_rng(seed)
+    cols_a = np.unique(rng.integers(0, p.d_in, ncols))
+    cols_b = np.unique(rng.integers(0, p.d_out, ncols))
+    nt = oracle.num_procs()
+    o = {"Y": oracle.forward(p, rows=rows, nthreads=nt)["Y"],
+         "dX": oracle.input_grad(p, rows=rows, nthreads=nt)["dX"]}
+    o.update(oracle.weight_grads(p, nthreads=nt, cols_a=cols_a, cols_b=cols_b))
+    return compare(p, g, o, BF16_TOL, rows=rows, cols_a=cols_a, cols_b=cols_b)
+
+
+@pytest.mark.parametrize("which", ["i", "ii", "iii", "iv"])
+def test_config5_degenerate_mixes(which):
+    """Full-size degenerate mixes: rank 1 next to rank 256, 1-token next to 8192-token segments,
+    mixed ranks over equal segments, and an adapter with no tokens."""
+    p = wl.config5_mix(which)
+    errs, bad = sampled_check(p, run(p))
+    assert not bad, (which, bad, errs)
+
+
+def test_config5_scaling_32_adapters():
+    p = wl.config5_scaling(32)
+    errs, bad = sampled_check(p, run(p))
+    assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("proj", range(7))
+def test_config4_layer_projection_shapes(proj):
+    """Each of the LLaMA-3-8B layer's seven projection shapes (q, k, v, o, gate, up, down; the down
+    projection reads 14336-wide inputs), 16 adapters r ~ U{16,32,64}, at 512 tokens per adapter."""
+    nm, di, do = wl.LLAMA3_LAYER[proj]
+    ranks = wl.rng_for(1004, 1).choice(np.array([16, 32, 64]), size=16)
+    p = wl.make_problem(f"cfg4s_{nm}", "bf16", di, do, ranks, [512] * 16, 2.0 * ranks, wl.init_llm(di),
+                        1004 * 16 + proj)
+    errs, bad = sampled_check(p, run(p))
+    assert not bad, (nm, bad, errs)
