@@ -307,3 +307,39 @@ def test_adamw_zero_gradient_is_pure_decay():
     p0 = np.random.default_rng(7).standard_normal(40)
     p1, m1, v1 = oracle.adamw(p0, np.zeros(40), np.zeros(40), np.zeros(40), lr=0.1, weight_decay=0.2, step=3)
     assert np.array_equal(p1, p0 * (1 - 0.1 * 0.2)) and not np.any(m1) and not np.any(v1)
+
+
+def test_output_blocks_equal_one_block_diagonal_adapter():
+    """Stacking P projections that read the same input (q|k|v), each adapter holding one rank-r pair
+    per projection, is the same layer as one adapter of rank P r over the stacked W whose B is
+    block-diagonal.  The oracle run on each projection's slice and on that block-diagonal embedding
+    agree: Y and dX, the row blocks of dA and the diagonal blocks of dB (the reading that output
+    blocks implement)."""
+    widths, ranks, counts, d_in = [8, 4, 4], [2, 3], [5, 7], 12
+    P, r = len(widths), np.asarray(ranks)
+    base = wl.make_problem("blk", "fp32", d_in, sum(widths), r, counts, 2.0 * r, wl.init_small(d_in), 41)
+    extra = [wl.make_problem(f"blk{b}", "fp32", d_in, 8, r, [1, 1], 2.0 * r, wl.init_small(d_in), 41 + b).A
+             for b in range(1, P)]
+    A_blocks = [base.A] + extra
+    bounds = np.concatenate([[0], np.cumsum(widths)])
+    A_bd, B_bd = [], []
+    for i, ri in enumerate(ranks):
+        A_bd.append(np.concatenate([A_blocks[b][i] for b in range(P)]))
+        Bi = np.zeros((sum(widths), P * ri), dtype=base.B[i].dtype)
+        for b in range(P):
+            Bi[bounds[b]:bounds[b + 1], b * ri:(b + 1) * ri] = base.B[i][bounds[b]:bounds[b + 1]]
+        B_bd.append(Bi)
+    bd = dataclasses.replace(base, ranks=P * r, A=A_bd, B=B_bd)   # same scales s_i = alpha_i / r_i
+    o_bd = oracle.full(bd)
+    dX = 0.0
+    for b in range(P):
+        cols = slice(bounds[b], bounds[b + 1])
+        pb = dataclasses.replace(base, d_out=widths[b], W=base.W[cols], dY=base.dY[:, cols], A=A_blocks[b],
+                                 B=[x[cols] for x in base.B])
+        o = oracle.full(pb)
+        assert rel(o_bd["Y"][:, cols], o["Y"]) < 1e-12
+        dX = dX + o["dX"]
+        for i, ri in enumerate(ranks):
+            assert rel(o_bd["dA"][i][b * ri:(b + 1) * ri], o["dA"][i]) < 1e-12
+            assert rel(o_bd["dB"][i][cols, b * ri:(b + 1) * ri], o["dB"][i]) < 1e-12
+    assert rel(o_bd["dX"], dX) < 1e-12
