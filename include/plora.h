@@ -43,7 +43,10 @@
  * Semantics.  Y, dX, dA_i and dB_i are overwritten, never accumulated into.
  * An adapter with no tokens (off[i] == off[i+1]) gets dA_i = dB_i = 0.
  * All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
- * stream); calls return once it is enqueued.
+ * stream); calls return once it is enqueued.  A handle stages each call's
+ * schedule in one of four slots, so a call first waits until the work of the
+ * call four before it on the same handle has run (calls captured into a CUDA
+ * graph use reserved slots instead; see plora_capture_reserve).
  *
  * Errors.  Every argument is checked before anything is enqueued; on an
  * error nothing is written and the call returns a non-zero status, with a
@@ -234,8 +237,9 @@ PLORA_API plora_status plora_debug_unpack_saved(plora_handle h, int32_t n_adapte
  *              first partial slot (-1 if unsplit), first counter (-1);
  *   which = 2: adapters, 5 per adapter: first token row, tokens, first H/G
  *              row (each adapter with tokens owns a block of 256 zero rows,
- *              its rows rounded up to 128, then 256 zero rows), rank rounded
- *              up to 16, rank rounded up to 64;
+ *              its rows rounded up to 128, then 256 zero rows), the width of
+ *              its H/G columns (P output blocks x the rank rounded up to 16;
+ *              P = 1 without output blocks), that width rounded up to 64;
  *   which = 3: two values: the padded rank pitch RP and the H/G row count;
  *   which = 4: per global 256-row tile of the base GEMMs, the first index
  *              into the list of which = 5 (plus the end): ceil(T/256) + 1 values;

@@ -95,7 +95,9 @@ def test_output_blocks_widen_the_padded_rank():
         s, v = pl.plora_debug_schedule(c, 1, off, fake_table([24]), False, 3)
         assert s == pl.PLORA_OK and v[0] == want
     s, v = pl.plora_debug_schedule(c3, 1, off, fake_table([24]), False, 2)
-    assert s == pl.PLORA_OK
+    assert s == pl.PLORA_OK and list(v[3:5]) == [96, 128]        # H/G width 3 x 32, rounded to 64
+    s, v = pl.plora_debug_schedule(c1, 1, off, fake_table([24]), False, 2)
+    assert s == pl.PLORA_OK and list(v[3:5]) == [32, 64]
 
 
 def test_create_without_gpu_fails_loudly():
