@@ -53,3 +53,12 @@ def test_library_arm_line():
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1 and cb["cpu_model"]
     fl = d["l2_flushed"]                   # the same steps with L2 flushed before each one
     assert fl["value"] > 0 and fl["ms_per_step"] > 0 and fl["unit"] == d["unit"]
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    # under torchrun only rank 0 runs the oracle and prints; the other ranks exit 0 without work
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert not [l for l in out.stdout.splitlines() if l.startswith("{")]
