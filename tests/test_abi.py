@@ -246,3 +246,12 @@ def test_empty_call_is_valid():
     assert len(v) == 0
     v = schedule(cfg(), [0, 0, 0], [3, 5], 1, grads=True)
     assert len(v) == 0
+
+
+def test_make_config_writes_cumulative_block_ends():
+    c = pl.make_config(4096, 6144, pl.PLORA_BF16, 16, 64, 1 << 16, 0, out_blocks=[4096, 1024, 1024])
+    assert c.n_out_blocks == 3 and list(c.out_block_end[:3]) == [4096, 5120, 6144] and c.reserved == 0
+    assert pl.make_config(64, 64, pl.PLORA_BF16, 1, 8, 8, 0, out_blocks=[64]).n_out_blocks == 0
+    off = np.array([0, 10], np.int64)
+    s, v = pl.plora_debug_schedule(c, 1, off, fake_table([16]), False, 3)
+    assert s == pl.PLORA_OK and v[0] == 3 * 16 + 16        # RP: 3 blocks x 16, rounded up to 64
