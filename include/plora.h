@@ -349,19 +349,29 @@ PLORA_API plora_status plora_profile_read(plora_handle h, int32_t capacity, int3
  * plora_backward (only rank, scale and dB are read; dB must be non-NULL and
  * 16-byte aligned, A and B must still be valid pointers).  Writes every dB_i.
  *
- * Returns PLORA_ERR_UNSUPPORTED if the call's schedule (64 bytes per adapter
- * plus 32 bytes per 16384-token split) exceeds 1 MiB - 256 bytes, or if its
- * split partials exceed the rest of the array: (splits of adapters longer
- * than 16384 tokens) x ceil(d_out/128) x (4 + 128 x RP x 4) bytes must fit
- * in PLORA_STATIC_SCRATCH_BYTES - 1 MiB, RP = max rank rounded up to 64.  Other errors as for
- * plora_backward; a device wait that runs out of time is not reported
- * (there is no handle to report it through).
+ * Returns PLORA_ERR_UNSUPPORTED when the call does not fit the array, whose
+ * first MiB holds the schedule and whose rest holds the split state:
+ *   - the schedule, 256 + 64 x n_adapters + 32 x (token splits) bytes (each
+ *     part rounded up to 256), must fit in 1 MiB; an adapter has
+ *     ceil(n_i / 16384) token splits;
+ *   - the split state of the adapters longer than 16384 tokens must fit in
+ *     PLORA_STATIC_SCRATCH_BYTES - 1 MiB: their arrival counters,
+ *     S x max(ceil(d_in/128), ceil(d_out/128)) x 4 bytes rounded up to 256
+ *     (S = the number of such adapters), then their partials,
+ *     (their token splits) x ceil(d_out/128) x 128 x RP x 4 bytes, with RP the
+ *     largest rank rounded up to 64.
+ * Other errors as for plora_backward; a device wait that runs out of time is
+ * not reported (there is no handle to report it through).
  *
+ * The schedule reaches the array through the parameters of small staging
+ * kernels, which the launch copies when it is enqueued: the call copies
+ * nothing from host memory and does not wait for the stream's earlier work.
  * The first call on each device resolves the array's device address and sets
- * the kernel up; make that first call before any stream capture.  Every call
- * shares the one array and clears what must start at zero; calls whose work
- * overlaps on the GPU (different streams, or different host threads) race on
- * it and must be serialised by the caller.
+ * the kernel up; make that first call before any stream capture begins.
+ * Every call shares the one array and clears what must start at zero (the
+ * error flag and the arrival counters); calls whose work overlaps on the GPU
+ * (different streams, or different host threads) race on it and must be
+ * serialised by the caller.
  */
 #define PLORA_STATIC_SCRATCH_BYTES (16u << 20)
 PLORA_API plora_status plora_grad_B_static(const plora_config* cfg, const void* dY, int32_t n_adapters,

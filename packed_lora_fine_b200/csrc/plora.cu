@@ -1376,18 +1376,47 @@ plora_status plora_debug_schedule(const plora_config* cfg, int32_t n, const int6
 // device address (on the host it only stands for the symbol), so the first
 // call on each device looks the address up with cudaGetSymbolAddress and
 // passes that pointer to the kernel.
+//
+// The schedule reaches the array through kernel parameters: the launch copies
+// them when it is enqueued, so the call needs neither pinned staging (which it
+// would have to allocate) nor a copy from pageable host memory (which may wait
+// for the stream's earlier work).
 // ===========================================================================
 namespace {
 
 constexpr size_t kStaticScratchBytes = PLORA_STATIC_SCRATCH_BYTES;
 constexpr size_t kStaticSchedBytes = (size_t)1 << 20;      // error flag + adapter table + splits
 constexpr int kStaticMaxDevices = 64;
+constexpr int kStaticParam16 = 1536;                       // 24 KB of schedule per staging launch
+
+// One staging launch: `n16` 16-byte words of schedule for [dst, dst + 16 n16) of the array and,
+// on the first launch of a call, the error flag ([0, 256)) and `zero16` words at `zero` (the arrival
+// counters) cleared, since the previous call may have left them set.
+struct StaticStage {
+    uint32_t dst;      // byte offset of the schedule words in the array
+    uint32_t n16;
+    uint32_t zero;     // byte offset of the counters to clear
+    uint32_t zero16;
+    uint32_t clear_flag;
+    uint32_t pad_[3];
+    uint4 words[kStaticParam16];
+};
+static_assert(sizeof(StaticStage) + sizeof(void*) < 32000, "kernel parameters of the staging launch");
 
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_plora_static_scratch[kStaticScratchBytes];
 
 namespace {
+
+__global__ void static_stage_kernel(const __grid_constant__ StaticStage s, uint8_t* scratch) {
+    const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
+    uint4* dst = reinterpret_cast<uint4*>(scratch + s.dst);
+    for (uint32_t i = tid; i < s.n16; i += nth) dst[i] = s.words[i];
+    uint4* z = reinterpret_cast<uint4*>(scratch + s.zero);
+    for (uint32_t i = tid; i < s.zero16; i += nth) z[i] = make_uint4(0, 0, 0, 0);
+    if (s.clear_flag && tid < 256 / 16) reinterpret_cast<uint4*>(scratch)[tid] = make_uint4(0, 0, 0, 0);
+}
 
 struct StaticDevice {
     uint8_t* scratch = nullptr;   // device address of g_plora_static_scratch on this device
@@ -1420,6 +1449,27 @@ plora_status static_setup(int dev, StaticDevice& out) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Byte layout of one call's scratch inside the static array.
+struct StaticLayout {
+    size_t o_ad, o_red, sched_end;   // [0, 256) error flag | adapter table | splits   (< kStaticSchedBytes)
+    size_t o_cnt, cnt_bytes;         // arrival counters: the plan's count, one int each
+    size_t o_part, part_end;         // split partials [slot][d_out tile][rank column][128 rows] fp32
+};
+
+StaticLayout static_layout(const HostPlan& P, int32_t dtiles_out) {
+    StaticLayout L;
+    L.o_ad = 256;
+    L.o_red = align256(L.o_ad + P.ad.size() * sizeof(AdapterDev));
+    L.sched_end = align256(L.o_red + P.red.size() * sizeof(RedEntry));
+    L.o_cnt = kStaticSchedBytes;
+    // build_plan spaces each split adapter's counters by max(d_in, d_out tiles): size the area from
+    // its total, not from the d_out tiles the dB product reads.
+    L.cnt_bytes = align256((size_t)P.counters * sizeof(int32_t));
+    L.o_part = L.o_cnt + L.cnt_bytes;
+    L.part_end = L.o_part + (size_t)P.slots * dtiles_out * kTileM * (size_t)P.RP * sizeof(float);
+    return L;
+}
+
 }  // namespace
 
 extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void* dY, int32_t n, const int64_t* off,
@@ -1448,15 +1498,8 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     build_plan(&tmp, n, off, tab, P);
     const int64_t d_out = cfg->d_out;
     const int32_t dtiles = (int32_t)ceil_div(d_out, kTileM);
-    // Scratch layout: [0,256) error flag | adapter table | splits  (within kStaticSchedBytes)
-    //                 | counters | partials                         (the rest of the array)
-    const size_t o_ad = 256;
-    const size_t o_red = align256(o_ad + P.ad.size() * sizeof(AdapterDev));
-    const size_t sched_end = align256(o_red + P.red.size() * sizeof(RedEntry));
-    const size_t o_cnt = kStaticSchedBytes;
-    const size_t o_part = align256(o_cnt + (size_t)P.slots * dtiles * sizeof(int32_t));
-    const size_t part_end = o_part + (size_t)P.slots * dtiles * kTileM * (size_t)P.RP * sizeof(float);
-    if (sched_end > kStaticSchedBytes || part_end > kStaticScratchBytes) return PLORA_ERR_UNSUPPORTED;
+    const StaticLayout L = static_layout(P, dtiles);
+    if (L.sched_end > kStaticSchedBytes || L.part_end > kStaticScratchBytes) return PLORA_ERR_UNSUPPORTED;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStaticMaxDevices) return PLORA_ERR_CUDA;
@@ -1479,17 +1522,28 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
             return PLORA_ERR_CUDA;
     if (P.T == 0) return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
 
-    // The array keeps the previous call's contents: clear the error flag and the arrival
-    // counters, then copy this call's schedule in.
+    // The array keeps the previous call's contents.  The schedule words ([256, sched_end): adapter
+    // table, then splits) travel in the parameters of one or more staging launches; the first also
+    // clears the error flag and this call's arrival counters.
+    std::vector<uint8_t> blob(L.sched_end - L.o_ad, 0);
+    memcpy(blob.data(), P.ad.data(), P.ad.size() * sizeof(AdapterDev));
+    if (!P.red.empty()) memcpy(blob.data() + (L.o_red - L.o_ad), P.red.data(), P.red.size() * sizeof(RedEntry));
     uint8_t* base = sd.scratch;
-    if (cudaMemsetAsync(base, 0, 256, st) != cudaSuccess) return PLORA_ERR_CUDA;
-    if (P.slots > 0 && cudaMemsetAsync(base + o_cnt, 0, (size_t)P.slots * dtiles * sizeof(int32_t), st) != cudaSuccess)
-        return PLORA_ERR_CUDA;
-    if (cudaMemcpyAsync(base + o_ad, P.ad.data(), P.ad.size() * sizeof(AdapterDev), cudaMemcpyHostToDevice, st) !=
-            cudaSuccess ||
-        cudaMemcpyAsync(base + o_red, P.red.data(), P.red.size() * sizeof(RedEntry), cudaMemcpyHostToDevice, st) !=
-            cudaSuccess)
-        return PLORA_ERR_CUDA;
+    StaticStage stg{};
+    const size_t chunk = sizeof(stg.words);
+    size_t at = 0;
+    do {   // blob.size() is a positive multiple of 256 (every call here has an adapter with tokens)
+        const size_t bytes = std::min(chunk, blob.size() - at);
+        const bool first = at == 0;
+        stg.dst = (uint32_t)(L.o_ad + at);
+        stg.n16 = (uint32_t)(bytes / 16);
+        memcpy(stg.words, blob.data() + at, bytes);
+        stg.zero = first ? (uint32_t)L.o_cnt : 0u;
+        stg.zero16 = first ? (uint32_t)(L.cnt_bytes / 16) : 0u;
+        stg.clear_flag = first ? 1u : 0u;
+        static_stage_kernel<<<8, 256, 0, st>>>(stg, base);
+        at += chunk;
+    } while (at < blob.size());
 
     CUtensorMap mdY, mH;
     if (!make_map(&mdY, dY, d_out, P.T, d_out, 64, 64) || !make_map(&mH, saved, P.RP, P.h_rows, P.RP, 64, 64))
@@ -1497,12 +1551,12 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     TcParams p{};
     p.RP = P.RP;
     p.nblk = 1;
-    p.adapters = reinterpret_cast<const AdapterDev*>(base + o_ad);
-    p.red = reinterpret_cast<const RedEntry*>(base + o_red);
+    p.adapters = reinterpret_cast<const AdapterDev*>(base + L.o_ad);
+    p.red = reinterpret_cast<const RedEntry*>(base + L.o_red);
     p.err_flag = reinterpret_cast<int*>(base);
     p.timeout_ns = kTimeoutNs;
-    p.partials = reinterpret_cast<float*>(base + o_part);
-    p.counters = reinterpret_cast<int32_t*>(base + o_cnt);
+    p.partials = reinterpret_cast<float*>(base + L.o_part);
+    p.counters = reinterpret_cast<int32_t*>(base + L.o_cnt);
     p.group_m = 16;
     p.M_total = (int32_t)d_out;
     p.red_dtiles = dtiles;

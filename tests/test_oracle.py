@@ -249,6 +249,28 @@ def test_rows_api_matches_full_rows():
         oracle.forward(p, rows=np.array([p.T], np.int64))
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_column_subset_api_matches_full_columns(dtype):
+    """The column-subset mode of the weight gradients (the full-size parity tests check sampled
+    hidden columns of dA and rows of dB) gives exactly the full call's values on the requested
+    columns, for every adapter including the empty one, and leaves every other column untouched.
+    The requested columns come unsorted and include both ends."""
+    p = small(62, dtype)
+    full = oracle.weight_grads(p)
+    cols_a = np.array([p.d_in - 1, 3, 0, 11], np.int64)
+    cols_b = np.array([7, p.d_out - 1, 0, 2, 15], np.int64)
+    sub = oracle.weight_grads(p, cols_a=cols_a, cols_b=cols_b)
+    for i in range(p.n_adapters):
+        assert np.array_equal(sub["dA"][i][:, cols_a], full["dA"][i][:, cols_a]), i
+        assert np.array_equal(sub["dB"][i][cols_b], full["dB"][i][cols_b]), i
+        rest_a = np.setdiff1d(np.arange(p.d_in), cols_a)
+        rest_b = np.setdiff1d(np.arange(p.d_out), cols_b)
+        assert not np.any(sub["dA"][i][:, rest_a]) and not np.any(sub["dB"][i][rest_b]), i
+    # the subsets are not all zero: the comparison above has something to see
+    assert any(np.any(sub["dA"][i][:, cols_a]) for i in range(p.n_adapters))
+    assert any(np.any(sub["dB"][i][cols_b]) for i in range(p.n_adapters))
+
+
 def test_threads_do_not_change_results():
     p = small(71, "bf16")
     a, b = oracle.full(p, nthreads=1), oracle.full(p, nthreads=4)

@@ -23,6 +23,12 @@ MUTANTS = {
     "H_uses_wrong_factor_row": ("ld(Ai, dtype, (int64_t)k * d_in + j);", "ld(Ai, dtype, j);"),
     "adamw_bias_correction_dropped": ("p[e] = p[e] - (lr / bc1) * m[e] / denom;", "p[e] = p[e] - lr * m[e] / denom;"),
     "adamw_decay_coupled": ("p[e] = p[e] * (1.0 - lr * weight_decay);", "p[e] = p[e] * (1.0 - weight_decay);"),
+    # column-subset mode: the q-th requested column stored at position q instead of its own index
+    "dB_column_subset_stored_by_position": ("dB[i][c * r + k] = s * acc;", "dB[i][q * r + k] = s * acc;"),
+    "dA_column_subset_stored_by_position": ("dA[i][(int64_t)k * d_in + j] = acc;",
+                                            "dA[i][(int64_t)k * d_in + q] = acc;"),
+    "dA_column_subset_reads_position": ("acc += ld(X, dtype, (t0 + u) * d_in + j) * G[u * r + k];",
+                                        "acc += ld(X, dtype, (t0 + u) * d_in + q) * G[u * r + k];"),
 }
 
 PINS = [
@@ -33,6 +39,8 @@ PINS = [
     ("linear_in_scale", T.test_linear_in_scale),
     ("finite_differences", T.test_gradients_match_central_finite_differences),
     ("segment_signature", T.test_segment_signature_exact),
+    ("column_subset_fp32", lambda: T.test_column_subset_api_matches_full_columns("fp32")),
+    ("column_subset_bf16", lambda: T.test_column_subset_api_matches_full_columns("bf16")),
     ("adamw_torch", lambda: T.test_adamw_matches_torch_adamw_in_float64(T.ADAMW_CASES[0])),
     ("adamw_first_step", T.test_adamw_first_step_closed_form),
     ("adamw_zero_grad", T.test_adamw_zero_gradient_is_pure_decay),
