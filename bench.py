@@ -9,9 +9,11 @@ shape, resident in HBM before the timed region (larger than L2, so no flush).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 runs under torch.distributed.run, one process per GPU; each rank packs
-its own 32 adapters (adapters are independent, so the work shards with no
-data-path collective: weak scaling); the step time is the max over ranks.
+N > 1 runs under torch.distributed.run, one process per GPU.  By default the
+32 adapters are split across the GPUs by plora_partition (longest processing
+time first over the per-adapter cost): adapters are independent, so the work
+shards with no data-path collective (strong scaling); `--scaling weak` gives
+every rank its own 32-adapter set instead.  The step time is the max over ranks.
 `--impl reference` times the fp64 CPU oracle on the host cores instead.
 Rank 0 prints one JSON line.
 """
@@ -68,6 +70,9 @@ def parse_args(argv=None):
                          "of the one-layer workload, 16 adapters x 8192 tokens (both for profiler captures); "
                          "llama_up_r16x1: one rank-16 adapter over the same tokens (base GEMMs with negligible "
                          "low-rank work)")
+    ap.add_argument("--scaling", choices=["strong", "weak"], default="strong",
+                    help="N > 1: strong = one 32-adapter set split across the GPUs by plora_partition (LPT over "
+                         "the per-adapter cost); weak = every GPU runs its own 32-adapter set")
     ap.add_argument("--base-gemm-reference", action="store_true",
                     help="time the workload's two base GEMMs (Y = X W^T, dX = dY W) through torch.matmul "
                          "(cuBLAS) with the same timing, clock and energy records; a context line, not a "
@@ -210,6 +215,18 @@ def reduce_sum(x: float, dist) -> float:
     return float(t.item())
 
 
+def shard_for_rank(p, world: int, rank: int):
+    """This rank's share of one adapter set split across `world` GPUs (plora_partition: longest
+    processing time first over the per-adapter cost); adapters are independent, so no rank needs
+    another's data."""
+    import packed_lora_fine_b200 as pl
+    owner, _ = pl.plora_partition(p.counts, p.ranks, p.d_in, p.d_out, world)
+    ids, _, _ = pl.shard(owner, p.off, rank)
+    if len(ids) == 0:
+        raise SystemExit(f"rank {rank}: no adapter left for this GPU ({p.n_adapters} adapters over {world} GPUs)")
+    return wl.take_adapters(p, ids)
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -283,7 +300,8 @@ def run_reference(args):
     sample = (f"fp64 oracle fwd+bwd of {p.T} tokens per step (first 8 adapters of the 32-adapter mix, "
               f"{tokens_each} tokens each) on {nt} host threads")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if (args.gpus > 1 and args.scaling == "strong") else "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD, "adapters": 8, "tokens_per_step": p.T, "d_in": 4096,
                        "d_out": 14336},
@@ -330,6 +348,8 @@ def main(argv=None):
         _, counts, _ = wl.config3_shape(args.seed + 1000 * rank)
         p = wl.make_problem("cfg3_r16x1", "bf16", 4096, 14336, np.array([16]), [int(np.sum(counts))], [32.0],
                             wl.init_llm(4096), args.seed + 1000 * rank)
+    elif world > 1 and args.scaling == "strong":
+        p = shard_for_rank(wl.config3(seed=args.seed), world, rank)
     else:
         p = wl.config3(seed=args.seed + 1000 * rank)
     T = p.T
@@ -535,11 +555,14 @@ def main(argv=None):
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong" if (world > 1 and args.scaling == "strong" and args.workload == "llama_up32") else "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": WORKLOADS[args.workload], "adapters": n, "tokens_per_gpu": T,
                            "global_tokens": int(tokens_all),
-                           "d_in": p.d_in, "d_out": p.d_out, "parallelism": f"adapter-sharded x{world}",
+                           "d_in": p.d_in, "d_out": p.d_out,
+                           "parallelism": (f"one adapter set split over {world} GPUs (LPT, plora_partition)"
+                                           if world > 1 and args.scaling == "strong" else f"adapter-sharded x{world}"),
                            "l2": "inputs larger than L2 (X %.0f MB, dY %.0f MB); no flush" % (
                                X.numel() * 2 / 1e6, dY.numel() * 2 / 1e6),
                            "base_gemm": base_gemm},

@@ -379,6 +379,29 @@ PLORA_API plora_status plora_grad_B_static(const plora_config* cfg, const void* 
                                            void* stream);
 
 /*
+ * Multi-GPU sharding of one adapter set: assign each adapter to one of n_parts GPUs (one process
+ * per GPU, each running its own handle over its share), balancing the parts' costs.  PLoRA runs
+ * each packed job on a chosen number of GPUs (PLoRA summary, gist.science, arXiv 2508.02932,
+ * 技术摘要 › 方法论 › 1. LoRA 打包规划器 (parallelism degree per job)); adapters are independent, so a
+ * part needs no data from another and no collective follows.  Host logic only: no device, no handle.
+ *
+ * counts: host int64[n] tokens per adapter (>= 0); ranks: host int32[n] in [1, PLORA_MAX_RANK];
+ * d_in, d_out: the projection; flops_per_s, bytes_per_s (> 0): the tensor and memory peaks the cost
+ * model divides by.  Adapter i costs
+ *     n_i ( (4 d_in d_out + 6 r_i (d_in + d_out)) / flops_per_s + (8 (d_in + d_out) + 12 r_i) / bytes_per_s )
+ * (its tokens' share of the two base GEMMs and the low-rank products, and the low-rank kernels' bytes).
+ * Longest processing time first: adapters by decreasing cost (ties: lower index first) each go to the
+ * part with the least cost so far (ties: lower part index), so the result is deterministic and the
+ * largest part's cost is at most (4/3 - 1/(3 n_parts)) times the best possible.
+ * owner (out): host int32[n], the part of each adapter; part_cost (out, may be NULL): host
+ * double[n_parts], each part's summed cost.  n in [0, PLORA_MAX_ADAPTERS], n_parts in
+ * [1, PLORA_MAX_ADAPTERS]; anything else returns PLORA_ERR_INVALID_ARG and writes nothing.
+ */
+PLORA_API plora_status plora_partition(int32_t n_adapters, const int64_t* counts, const int32_t* ranks,
+                                       int64_t d_in, int64_t d_out, double flops_per_s, double bytes_per_s,
+                                       int32_t n_parts, int32_t* owner, double* part_cost);
+
+/*
  * Debug / failure detection: launch one CTA whose bounded wait is on a barrier that
  * nothing ever arrives at, through the same bounded-wait code the kernels use, with a
  * limit of timeout_ns (1 ms .. 10 s).  The wait runs out, the kernel records

@@ -42,7 +42,7 @@ EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
             "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe", "plora_device_info",
-            "plora_capture_reserve", "plora_capture_release")
+            "plora_capture_reserve", "plora_capture_release", "plora_partition")
 
 
 class plora_config(ctypes.Structure):
@@ -128,6 +128,8 @@ def load(path: str = LIB_PATH):
     lib.plora_grad_B_static.restype = ctypes.c_int
     lib.plora_version.argtypes = []
     lib.plora_version.restype = ctypes.c_int32
+    lib.plora_partition.argtypes = [I32, P, P, I64, I64, ctypes.c_double, ctypes.c_double, I32, P, P]
+    lib.plora_partition.restype = ctypes.c_int
     for fn in ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
                "plora_check", "plora_debug_unpack_saved"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -274,6 +276,41 @@ def plora_device_info(h: int) -> dict:
     cnt = ctypes.c_int32(0)
     _raise(h, load().plora_device_info(h, ctypes.cast(out, ctypes.c_void_p), 3, ctypes.byref(cnt)))
     return {"sms": int(out[0]), "pairs_fwd": int(out[1]), "pairs_dx": int(out[2])}
+
+
+# Nominal B200 peaks for the partition cost model (dense bf16 tensor FLOP/s, HBM bytes/s); only their
+# ratio matters for the balance.
+PARTITION_FLOPS = 2.25e15
+PARTITION_BYTES = 8.0e12
+
+
+def plora_partition(counts, ranks, d_in: int, d_out: int, n_parts: int, flops_per_s: float = PARTITION_FLOPS,
+                    bytes_per_s: float = PARTITION_BYTES):
+    """Assign each adapter to one of n_parts GPUs (longest processing time first over the per-adapter
+    cost of include/plora.h).  Returns (owner int32[n], part_cost float64[n_parts]); raises PloraError."""
+    counts = np.ascontiguousarray(counts, dtype=np.int64)
+    ranks = np.ascontiguousarray(ranks, dtype=np.int32)
+    n = len(counts)
+    owner = np.full(n, -1, np.int32)
+    cost = np.zeros(max(1, int(n_parts)), np.float64)
+    st = load().plora_partition(n, counts.ctypes.data, ranks.ctypes.data, int(d_in), int(d_out), float(flops_per_s),
+                                float(bytes_per_s), int(n_parts), owner.ctypes.data, cost.ctypes.data)
+    if st != PLORA_OK:
+        raise PloraError(st, "plora_partition")
+    return owner, cost[:n_parts]
+
+
+def shard(owner, off, part: int):
+    """Part `part`'s share of a packed adapter set: (adapter ids in increasing order, their local
+    offsets int64[k+1] into the part's own packed token buffer, and the global row ranges
+    [(off[i], off[i+1])] to gather that buffer from).  Index bookkeeping only."""
+    owner = np.asarray(owner)
+    off = np.asarray(off, dtype=np.int64)
+    ids = np.nonzero(owner == part)[0].astype(np.int64)
+    counts = off[ids + 1] - off[ids]
+    local = np.zeros(len(ids) + 1, np.int64)
+    local[1:] = np.cumsum(counts)
+    return ids, local, [(int(off[i]), int(off[i + 1])) for i in ids]
 
 
 def plora_grad_B_static(cfg: plora_config, dY: int, n: int, off, tab, saved: int, stream: int = 0) -> int:

@@ -1363,6 +1363,45 @@ plora_status plora_debug_schedule(const plora_config* cfg, int32_t n, const int6
     return PLORA_OK;
 }
 
+plora_status plora_partition(int32_t n, const int64_t* counts, const int32_t* ranks, int64_t d_in, int64_t d_out,
+                             double flops_per_s, double bytes_per_s, int32_t n_parts, int32_t* owner,
+                             double* part_cost) {
+    if (n < 0 || n > PLORA_MAX_ADAPTERS || n_parts < 1 || n_parts > PLORA_MAX_ADAPTERS) return PLORA_ERR_INVALID_ARG;
+    if (d_in < 1 || d_out < 1 || !(flops_per_s > 0.0) || !(bytes_per_s > 0.0) || !std::isfinite(flops_per_s) ||
+        !std::isfinite(bytes_per_s))
+        return PLORA_ERR_INVALID_ARG;
+    if (n > 0 && (!counts || !ranks || !owner)) return PLORA_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i)
+        if (counts[i] < 0 || ranks[i] < 1 || ranks[i] > PLORA_MAX_RANK) return PLORA_ERR_INVALID_ARG;
+    // An adapter's cost is the ideal time of its share of one packed step at the given peaks: its tokens'
+    // share of the two base GEMMs and its low-rank products (4 d_in d_out + 6 r (d_in + d_out) flop per
+    // token) plus the low-rank kernels' memory traffic (8 (d_in + d_out) + 12 r bytes per token).
+    const double di = (double)d_in, dout = (double)d_out;
+    std::vector<double> cost(n);
+    for (int32_t i = 0; i < n; ++i) {
+        const double r = (double)ranks[i];
+        const double per_token = (4.0 * di * dout + 6.0 * r * (di + dout)) / flops_per_s +
+                                 (8.0 * (di + dout) + 12.0 * r) / bytes_per_s;
+        cost[i] = (double)counts[i] * per_token;
+    }
+    // Longest processing time first: adapters by decreasing cost (ties: lower index first), each to the
+    // part with the least cost so far (ties: lower part index).  Deterministic.
+    std::vector<int32_t> order(n);
+    for (int32_t i = 0; i < n; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return cost[a] > cost[b]; });
+    std::vector<double> load(n_parts, 0.0);
+    for (int32_t i : order) {
+        int32_t best = 0;
+        for (int32_t q = 1; q < n_parts; ++q)
+            if (load[q] < load[best]) best = q;
+        owner[i] = best;
+        load[best] += cost[i];
+    }
+    if (part_cost)
+        for (int32_t q = 0; q < n_parts; ++q) part_cost[q] = load[q];
+    return PLORA_OK;
+}
+
 }  // extern "C"
 
 // ===========================================================================

@@ -228,15 +228,23 @@ LLAMA3_LAYER = [("q", 4096, 4096), ("k", 4096, 1024), ("v", 4096, 1024), ("o", 4
                 ("gate", 4096, 14336), ("up", 4096, 14336), ("down", 14336, 4096)]
 
 
+def config4_ranks(seed: int = 1004) -> np.ndarray:
+    """The 16 adapter ranks of the one-layer workload, U{16,32,64}."""
+    return rng_for(seed, _S_RANK).choice(np.array([16, 32, 64]), size=16)
+
+
+def config4_projection(index: int, seed: int = 1004, draw_tokens: bool = True) -> Problem:
+    """Projection `index` of LLAMA3_LAYER in the one-layer workload: 16 adapters r ~ U{16,32,64},
+    4x2048 tokens each, with its own W, X, dY and per-adapter A, B (independent streams)."""
+    nm, di, do = LLAMA3_LAYER[index]
+    ranks = config4_ranks(seed)
+    return make_problem(f"cfg4_llama_{nm}", "bf16", di, do, ranks, [8192] * 16, 2.0 * ranks, init_llm(di),
+                        seed * 16 + index, draw_tokens)
+
+
 def config4(seed: int = 1004, draw_tokens: bool = True) -> List[Problem]:
-    """One LLaMA-3-8B layer's seven LoRA targets, 16 adapters r ~ U{16,32,64}, 4x2048 tokens each.
-    Each projection has its own W, X, dY and per-adapter A, B (independent streams)."""
-    ranks = rng_for(seed, _S_RANK).choice(np.array([16, 32, 64]), size=16)
-    out = []
-    for p, (nm, di, do) in enumerate(LLAMA3_LAYER):
-        out.append(make_problem(f"cfg4_llama_{nm}", "bf16", di, do, ranks, [8192] * 16,
-                                2.0 * ranks, init_llm(di), seed * 16 + p, draw_tokens))
-    return out
+    """One LLaMA-3-8B layer's seven LoRA targets (config4_projection for each of LLAMA3_LAYER)."""
+    return [config4_projection(k, seed, draw_tokens) for k in range(len(LLAMA3_LAYER))]
 
 
 def config5_scaling(k: int, seed: int = 1005) -> Problem:
@@ -282,6 +290,25 @@ def with_zero_W(p: Problem) -> Problem:
     q = dataclasses.replace(p)
     q.W = np.zeros_like(p.W)
     return q
+
+
+def take_adapters(p: Problem, ids) -> Problem:
+    """The adapters `ids` of p (in that order) as a problem of their own: their rows of X and dY packed
+    contiguously with local offsets, their factors, the same W.  Data selection only (one GPU's share
+    of an adapter set split across GPUs)."""
+    ids = [int(i) for i in ids]
+    counts = np.array([p.off[i + 1] - p.off[i] for i in ids], dtype=np.int64)
+    off = np.zeros(len(ids) + 1, dtype=np.int64)
+    off[1:] = np.cumsum(counts)
+
+    def rows(a):
+        if a is None:
+            return None
+        parts = [a[p.off[i]:p.off[i + 1]] for i in ids]
+        return np.ascontiguousarray(np.concatenate(parts)) if parts else a[:0].copy()
+    return dataclasses.replace(p, name=f"{p.name}_part", off=off, ranks=p.ranks[ids], alphas=p.alphas[ids],
+                               scales=p.scales[ids], X=rows(p.X), dY=rows(p.dY), A=[p.A[i] for i in ids],
+                               B=[p.B[i] for i in ids])
 
 
 def sample_rows(p: Problem, per_segment: int = 6, seed: int = 7) -> np.ndarray:

@@ -94,3 +94,70 @@ def compare(p, g, o, tol, rows=None, cols_a=None, cols_b=None):
         errs[f"dB{i}"] = rel_err(gb, ob)
     bad = {k: v for k, v in errs.items() if not (v <= tol)}
     return errs, bad
+
+
+def row_subproblem(p, rows):
+    """The problem restricted to the given rows (sorted): each adapter keeps only its sampled rows
+    of X and dY, as one contiguous segment.  A row of Y or dX depends only on that row of X or dY
+    and on its adapter, so the oracle run on this small problem gives exactly those rows of the
+    full problem's Y and dX (checked on the CPU by tests/test_oracle.py); full-size tests use it
+    so that the oracle never copies a multi-GB input."""
+    import dataclasses
+    rows = np.asarray(rows, dtype=np.int64)
+    assert np.all(np.diff(rows) > 0)
+    seg = np.searchsorted(p.off, rows, side="right") - 1
+    counts = np.bincount(seg, minlength=p.n_adapters).astype(np.int64)
+    off = np.zeros(p.n_adapters + 1, np.int64)
+    off[1:] = np.cumsum(counts)
+    return dataclasses.replace(p, off=off, X=np.ascontiguousarray(p.X[rows]), dY=np.ascontiguousarray(p.dY[rows]))
+
+
+def adapter_subproblem(p, i, out_cols=None, A_rows=None):
+    """Adapter i alone over its own rows (the packed result equals each adapter run alone; pinned on
+    the CPU).  out_cols / A_rows select one output block's columns of W, dY, B and its rows of A."""
+    import dataclasses
+    a, b = int(p.off[i]), int(p.off[i + 1])
+    cols = slice(None) if out_cols is None else out_cols
+    A = p.A[i] if A_rows is None else p.A[i][A_rows]
+    W = p.W[cols]
+    dY = np.ascontiguousarray(p.dY[a:b, cols])
+    return dataclasses.replace(p, d_out=int(W.shape[0]), off=np.array([0, b - a], np.int64),
+                               ranks=p.ranks[i:i + 1], alphas=p.alphas[i:i + 1], scales=p.scales[i:i + 1],
+                               X=np.ascontiguousarray(p.X[a:b]), W=np.ascontiguousarray(W), dY=dY,
+                               A=[np.ascontiguousarray(A)], B=[np.ascontiguousarray(p.B[i][cols])])
+
+
+def run_sampled(p, rows, engine=None, unfused=False, base_pair=False, out_blocks=None):
+    """One packed forward + backward through the C ABI; returns the sampled rows of Y and dX
+    (gathered on the device) and every dA_i, dB_i, as numpy float64."""
+    import torch
+    import packed_lora_fine_b200 as pl
+    d = DeviceProblem(p)
+    own = engine is None
+    if own:
+        engine = pl.PackedLoRA(p.d_in, p.d_out, p.dtype, max_adapters=max(1, p.n_adapters),
+                               max_rank=int(max(p.ranks)), max_tokens=max(1, p.T), unfused=unfused,
+                               base_pair=base_pair, out_blocks=out_blocks)
+    Y, saved = engine.forward(d.X, d.W, p.off, p.scales, d.A, d.B)
+    dX, dA, dB = engine.backward(d.X, d.W, d.dY, p.off, p.scales, d.A, d.B, saved)
+    torch.cuda.synchronize()
+    st = pl.plora_check(engine.h, 0)
+    assert st == pl.PLORA_OK, pl.status_string(st)
+    idx = torch.from_numpy(np.asarray(rows, np.int64)).to(Y.device)
+    out = {"Y": from_dev(Y.index_select(0, idx)), "dX": from_dev(dX.index_select(0, idx)),
+           "dA": [from_dev(x) for x in dA], "dB": [from_dev(x) for x in dB]}
+    del Y, dX, saved, d
+    if own:
+        engine.close()
+    return out
+
+
+_PROBLEMS = {}
+
+
+def cached_problem(key, factory):
+    """One draw per test session of a large seeded problem (drawing config 3 takes half a minute on one
+    host core); callers must not modify the arrays in place."""
+    if key not in _PROBLEMS:
+        _PROBLEMS[key] = factory()
+    return _PROBLEMS[key]

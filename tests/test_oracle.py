@@ -271,6 +271,29 @@ def test_column_subset_api_matches_full_columns(dtype):
     assert any(np.any(sub["dB"][i][cols_b]) for i in range(p.n_adapters))
 
 
+def test_row_and_adapter_subproblems_give_the_full_problems_rows():
+    """The full-size parity tests run the oracle on small derived problems: the sampled rows
+    (each adapter's sampled rows as its segment), and one adapter alone (optionally one output
+    block's columns).  Both reproduce the full problem's values bit for bit."""
+    from plora_testlib import adapter_subproblem, row_subproblem
+    p = small(63, "bf16", counts=(9, 0, 14, 6))
+    full = oracle.full(p)
+    rows = np.array([0, 4, 8, 9, 15, 22, 23, 28], np.int64)
+    sub = oracle.full(row_subproblem(p, rows))
+    assert np.array_equal(sub["Y"], full["Y"][rows]) and np.array_equal(sub["dX"], full["dX"][rows])
+    for i in range(p.n_adapters):
+        alone = oracle.weight_grads(adapter_subproblem(p, i))
+        assert np.array_equal(alone["dA"][0], full["dA"][i]) and np.array_equal(alone["dB"][0], full["dB"][i])
+    # one output block: columns [8, 20) of W, dY, B; the weight gradients of that block alone
+    cols = slice(8, 20)
+    blk = dataclasses.replace(p, d_out=12, W=p.W[cols], dY=np.ascontiguousarray(p.dY[:, cols]),
+                              B=[np.ascontiguousarray(b[cols]) for b in p.B])
+    fb = oracle.weight_grads(blk)
+    for i in range(p.n_adapters):
+        alone = oracle.weight_grads(adapter_subproblem(p, i, out_cols=cols))
+        assert np.array_equal(alone["dA"][0], fb["dA"][i]) and np.array_equal(alone["dB"][0], fb["dB"][i])
+
+
 def test_threads_do_not_change_results():
     p = small(71, "bf16")
     a, b = oracle.full(p, nthreads=1), oracle.full(p, nthreads=4)

@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import plora_workloads as wl
-from plora_testlib import BF16_TOL, FP32_TOL, DeviceProblem, compare, rel_err, run
+from plora_testlib import BF16_TOL, FP32_TOL, DeviceProblem, cached_problem, compare, rel_err, run
 
 pytestmark = pytest.mark.gpu
 
@@ -226,7 +226,7 @@ def test_config2_qwen_q_proj():
 def test_config3_llama_up_proj_32_adapters(path):
     """The benchmark workload (LLaMA-3-8B up_proj, 32 long-tail adapters) on sampled outputs, with the
     base GEMMs on single SMs (the default) and on SM pairs."""
-    p = wl.config3()
+    p = cached_problem("config3", wl.config3)
     g = run(p, base_pair=(path == "tc_pair"))
     rows = wl.sample_rows(p, per_segment=2)
     rng = np.random.default_rng(6)
