@@ -107,10 +107,8 @@ def algorithmic_work(p):
         "expand_dx": (float(np.sum(2 * n * di * r)), float(np.sum(n * (4 * di + 2 * r) + 2 * r * di))),
         "wgrad_b": (float(np.sum(2 * n * do * r)), float(np.sum(n * (2 * do + 2 * r) + 4 * r * do))),
         "wgrad_a": (float(np.sum(2 * n * di * r)), float(np.sum(n * (2 * di + 2 * r) + 4 * r * di))),
-        # packs read each factor once and write rows (A, B^T) or columns (B) up to rp16
-        "pack_a": (0.0, float(np.sum(2 * r * di + 2 * rp16 * di))),
-        "pack_b": (0.0, float(np.sum(2 * r * do + 2 * rp16 * do))),
-        "pack_bt": (0.0, float(np.sum(2 * r * do + 2 * rp16 * do))),
+        # one pack per step: reads each factor once, writes A's rows and B's columns up to rp16
+        "pack_ab": (0.0, float(np.sum(2 * r * (di + do) + 2 * rp16 * (di + do)))),
     }
     # K7's items share K5's launch
     w["shrink_dy+wgrad_b"] = (w["shrink_dy"][0] + w["wgrad_b"][0], w["shrink_dy"][1] + w["wgrad_b"][1])

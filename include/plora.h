@@ -85,7 +85,8 @@ typedef enum {
     PLORA_ERR_UNSUPPORTED = 2,  /* a shape or dtype the library does not handle */
     PLORA_ERR_OOM = 3,          /* workspace allocation failed in plora_create */
     PLORA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
-    PLORA_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (see plora_check) */
+    PLORA_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out (see plora_check) */
+    PLORA_ERR_BOUNDS = 6        /* PLORA_DEBUG builds: a device-side bounds check failed (see plora_check) */
 } plora_status;
 
 typedef enum {
@@ -174,8 +175,10 @@ PLORA_API plora_status plora_destroy(plora_handle h);
 /*
  * Size in bytes of the `saved` buffer that plora_forward fills and
  * plora_backward reads for this segment map and adapter table.  Its layout
- * is the library's (per-adapter zero-padded blocks of s_i X_i A_i rows); read it
- * only through plora_debug_unpack_saved.
+ * is the library's: per-adapter zero-padded blocks of s_i X_i A_i rows and, on
+ * the tensor-core path, every adapter's A and B packed as the tensor cores read
+ * them (the forward packs them once; the backward reuses them, so A and B must
+ * not change between the two calls).  Read it only through plora_debug_unpack_saved.
  */
 PLORA_API plora_status plora_saved_bytes(plora_handle h, int32_t n_adapters, const int64_t* off,
                                const plora_adapter* tab, size_t* bytes);
@@ -204,8 +207,9 @@ PLORA_API plora_status plora_backward(plora_handle h, const void* X, const void*
 
 /*
  * Synchronise `stream` and report the handle's device error flag: PLORA_OK,
- * PLORA_ERR_TIMEOUT (a bounded device wait ran out; the flag is then
- * cleared) or PLORA_ERR_CUDA.
+ * PLORA_ERR_TIMEOUT (a bounded device wait ran out), PLORA_ERR_BOUNDS (a
+ * PLORA_DEBUG build's bounds check failed) or PLORA_ERR_CUDA.  A reported
+ * flag is cleared.
  */
 PLORA_API plora_status plora_check(plora_handle h, void* stream);
 
@@ -413,6 +417,17 @@ PLORA_API plora_status plora_debug_timeout_probe(plora_handle h, int64_t timeout
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 PLORA_API int32_t plora_version(void);
+
+/*
+ * 1 for the PLORA_DEBUG build of this library (libplora_debug.so), 0 otherwise (a diagnostic; the
+ * method has no such call).  In the debug build every kernel compares each index it forms from a
+ * call's schedule with the extent of the buffer it addresses, as the host allocated it (the output
+ * and the saved activations, the packed factors, the split partials and arrival counters, the
+ * schedule tables); a failed check sets the handle's error flag to PLORA_ERR_BOUNDS and the access
+ * is skipped (an out-of-range schedule entry is replaced by entry 0), so plora_check reports the error
+ * and nothing traps.  The checks cost time; results on valid inputs are those of the release build.
+ */
+PLORA_API int32_t plora_debug_build(void);
 
 #ifdef __cplusplus
 }

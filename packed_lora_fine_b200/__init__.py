@@ -20,7 +20,9 @@ from typing import Iterable, List, Optional, Sequence
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libplora.so")
+# PLORA_LIBRARY may name another build of the library (the PLORA_DEBUG build with device-side bounds
+# checks, libplora_debug.so); a missing file still raises ImportError.
+LIB_PATH = os.environ.get("PLORA_LIBRARY") or os.path.join(_HERE, "libplora.so")
 
 PLORA_OK = 0
 PLORA_ERR_INVALID_ARG = 1
@@ -28,6 +30,7 @@ PLORA_ERR_UNSUPPORTED = 2
 PLORA_ERR_OOM = 3
 PLORA_ERR_CUDA = 4
 PLORA_ERR_TIMEOUT = 5
+PLORA_ERR_BOUNDS = 6
 PLORA_BF16 = 0
 PLORA_FP32 = 1
 PLORA_FLAG_SIMT = 1
@@ -42,7 +45,7 @@ EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
             "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe", "plora_device_info",
-            "plora_capture_reserve", "plora_capture_release", "plora_partition")
+            "plora_capture_reserve", "plora_capture_release", "plora_partition", "plora_debug_build")
 
 
 class plora_config(ctypes.Structure):
@@ -128,6 +131,8 @@ def load(path: str = LIB_PATH):
     lib.plora_grad_B_static.restype = ctypes.c_int
     lib.plora_version.argtypes = []
     lib.plora_version.restype = ctypes.c_int32
+    lib.plora_debug_build.argtypes = []
+    lib.plora_debug_build.restype = ctypes.c_int32
     lib.plora_partition.argtypes = [I32, P, P, I64, I64, ctypes.c_double, ctypes.c_double, I32, P, P]
     lib.plora_partition.restype = ctypes.c_int
     for fn in ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",

@@ -17,6 +17,28 @@ constexpr int kLoraTileM = 256;     // base-GEMM rows per overlap record (one CT
 
 constexpr int kMaxOutBlocks = 8;    // output blocks (shared-input projections stacked along d_out)
 
+// Device-side bounds checks (the PLORA_DEBUG build).  A kernel compares each index it forms from the
+// schedule with the extent of the buffer it addresses, as the host allocated it; a failed check records
+// kErrBounds (PLORA_ERR_BOUNDS) in the handle's error flag and the access is skipped (or the schedule
+// entry replaced by entry 0), so a wrong schedule shows up as an error status, never as a fault.  In
+// release builds the checks compile to nothing.
+#ifdef PLORA_DEBUG
+constexpr bool kDeviceChecks = true;
+#else
+constexpr bool kDeviceChecks = false;
+#endif
+constexpr int kErrBounds = 6;
+
+__device__ __forceinline__ bool dcheck(int* err_flag, bool ok) {
+    if constexpr (kDeviceChecks) {
+        if (!ok) {
+            if (err_flag) atomicCAS(err_flag, 0, kErrBounds);
+            return false;
+        }
+    }
+    return true;
+}
+
 // The output blocks of a handle: block b holds output columns [end[b-1], end[b]).
 struct OutBlocks {
     int32_t n;

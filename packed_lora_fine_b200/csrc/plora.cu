@@ -53,7 +53,7 @@ struct plora_ctx {
 
     uint8_t* ws = nullptr;     // one device allocation, carved into regions
     size_t ws_bytes = 0;
-    Region r_G, r_packA, r_packBT, r_part, r_cnt, r_err, r_blob[kSlots];
+    Region r_G, r_part, r_cnt, r_err, r_blob[kSlots];
 
     uint8_t* h_blob[kSlots] = {};       // mapped pinned staging of each slot (host view)
     uint8_t* h_blob_dev[kSlots] = {};   // the same buffers as the device addresses them
@@ -161,11 +161,11 @@ __global__ void timeout_probe_kernel(int* err_flag, uint64_t limit_ns) {
 }
 
 // Kernel kinds for launch accounting / profiling.
-enum Kind { kPackA = 0, kPackBT, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
-            kSimt, kAdamw, kPackB, kShrinkDyWgradB, kStage, kKinds };
-const char* const kKindNames[kKinds] = {"pack_a", "pack_bt", "base_fwd", "shrink_x", "expand_y", "base_dx",
+enum Kind { kPack = 0, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
+            kSimt, kAdamw, kShrinkDyWgradB, kStage, kKinds };
+const char* const kKindNames[kKinds] = {"pack_ab", "base_fwd", "shrink_x", "expand_y", "base_dx",
                                         "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw",
-                                        "pack_b", "shrink_dy+wgrad_b", "stage_copy"};
+                                        "shrink_dy+wgrad_b", "stage_copy"};
 
 cudaEvent_t take_event(plora_ctx* h) {
     if (!h->pool.empty()) {
@@ -329,9 +329,27 @@ void build_plan(const plora_ctx* h, int32_t n, const int64_t* off, const plora_a
                      [](const RedEntry& a, const RedEntry& b) { return a.kblocks > b.kblocks; });
 }
 
-size_t saved_bytes_of(const plora_ctx* h, const HostPlan& P) {
-    return (size_t)P.h_rows * (size_t)P.RP * h->esize;
+// The `saved` buffer a forward fills and the backward reads: the zero-padded blocks of H' = s X A
+// ([h_rows][RP], at offset 0), then on the tensor-core path the packed factors of the call (packA
+// [n RP][d_in] and packB [n][d_out][RP], see pack_ab_kernel), each from a 256-byte boundary.
+struct SavedLayout {
+    size_t o_packA = 0, o_packB = 0, bytes = 0;
+};
+
+SavedLayout saved_layout(const plora_ctx* h, const HostPlan& P) {
+    SavedLayout L;
+    const size_t hb = (size_t)P.h_rows * (size_t)P.RP * h->esize;
+    if (!h->tc) {
+        L.bytes = hb;
+        return L;
+    }
+    L.o_packA = (size_t)round_up((int64_t)hb, 256);
+    L.o_packB = L.o_packA + (size_t)round_up((int64_t)P.n * P.RP * h->cfg.d_in * 2, 256);
+    L.bytes = L.o_packB + (size_t)P.n * (size_t)h->cfg.d_out * (size_t)P.RP * 2;
+    return L;
 }
+
+size_t saved_bytes_of(const plora_ctx* h, const HostPlan& P) { return saved_layout(h, P).bytes; }
 
 // Extents of every tensor a call reads or writes (see include/plora.h for the layouts).
 struct TensorArgs {
@@ -385,7 +403,9 @@ struct DevPlan {
 // Copies a call's schedule from the slot's mapped pinned staging buffer into device memory.  A kernel
 // rather than cudaMemcpyAsync: its reads of host memory do not wait in the copy-engine queue behind
 // bulk host-to-device copies that the caller may have in flight (the next step's inputs, say).
-__global__ void stage_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n16) {
+__global__ void stage_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n16, int64_t cap16,
+                                  int* err_flag) {
+    if (!dcheck(err_flag, n16 <= cap16)) return;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
         dst[i] = src[i];
 }
@@ -398,7 +418,7 @@ cudaError_t stage_copy(plora_ctx* h, const uint8_t* src, uint8_t* d, size_t byte
     const int blocks = (int)std::min<int64_t>(ceil_div(n16, 256), 64);
     tracked(h, kStage, st, [&] {
         stage_copy_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(d),
-                                                  n16);
+                                                  n16, (int64_t)(h->blob_bytes / 16), h->at<int>(h->r_err));
     });
     return cudaGetLastError();
 }
@@ -533,15 +553,16 @@ void launch_simt(plora_ctx* h, const SimtOp* d_ops, int n_ops, int tiles, cudaSt
 // ---------------------------------------------------------------------------
 // Tensor-core launches
 // ---------------------------------------------------------------------------
+// c: the output tensor map of a base GEMM (TMA-stored epilogue); other ops ignore it.
 template <Op OP>
 void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const CUtensorMap& b2,
-               const TcParams& p, cudaStream_t st) {
+               const CUtensorMap& c, const TcParams& p, cudaStream_t st) {
     if (p.num_tiles <= 0) return;
     const int grid = std::min(p.num_tiles, h->num_sms);
     constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : OP == Op::BaseDx ? kBaseDx : OP == Op::ShrinkX ? kShrinkX
                        : OP == Op::ShrinkDy ? kShrinkDy : OP == Op::ExpandY ? kExpandY : OP == Op::ExpandDx ? kExpandDx
                        : OP == Op::WgradB ? kWgradB : kWgradA;
-    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p, p); });
+    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, c, p, p); });
 }
 
 // Two independent ops in one persistent launch: OP's items (operands a, b) then OP2's (a2, b2).
@@ -551,7 +572,7 @@ void launch_tc2(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const 
     const int total = p.num_tiles + p2.num_tiles;
     if (total <= 0) return;
     const int grid = std::min(total, h->num_sms);
-    tracked(h, kind, st, [&] { tc_kernel<OP, OP2><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, p, p2); });
+    tracked(h, kind, st, [&] { tc_kernel<OP, OP2><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, a, p, p2); });
 }
 
 // Base GEMMs on SM pairs: a cluster of two CTAs per 256x256 tile, persistent over the pairs that
@@ -574,13 +595,13 @@ cudaLaunchConfig_t pair_config(int pairs, cudaStream_t st, cudaLaunchAttribute* 
 
 template <Op OP>
 void launch_pair(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                 const CUtensorMap& b2, const TcParams& p, cudaStream_t st) {
+                 const CUtensorMap& b2, const CUtensorMap& c, const TcParams& p, cudaStream_t st) {
     if (p.num_tiles <= 0) return;
     const int resident = OP == Op::BaseFwd ? h->pairs_fwd : h->pairs_dx;
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = pair_config<OP>(std::min(p.num_tiles, resident), st, attr);
     constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : kBaseDx;
-    tracked(h, kind, st, [&] { cudaLaunchKernelEx(&cfg, tc_pair_kernel<OP>, a, b, a2, b2, p); });
+    tracked(h, kind, st, [&] { cudaLaunchKernelEx(&cfg, tc_pair_kernel<OP>, a, b, a2, b2, c, p); });
 }
 
 template <Op OP>
@@ -637,37 +658,46 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     p.stage_bytes = kStageBytes;
     p.nblk = h->nblk;
     for (int b = 0; b < kMaxOutBlocks; ++b) p.blk_end[b] = h->blk_end[b];
+    p.part_elems = (int64_t)(h->r_part.bytes / sizeof(float));
+    p.n_counters = (int32_t)(h->r_cnt.bytes / sizeof(int32_t));
+    p.n_adapters = P.n;
+    p.n_mtrec = (int32_t)P.mt_rec.size();
+    p.n_mtseg = (int32_t)P.mt_seg.size();
     return p;
 }
 
-// Stages the factors in the layouts the tensor-core operands want: A as [n RP][d_in] (rows
-// padded to RP) always; B either row-padded, [n d_out][RP] (the fused forward's K-major expand
-// operand), or transposed, [n RP][d_out] (the shrink of the backward and the unfused expand).
-enum class BPack { RowPadded, Transposed };
-
-plora_status pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, BPack bp, cudaStream_t st) {
-    if (P.n == 0) return PLORA_OK;
-    __nv_bfloat16* pa = h->at<__nv_bfloat16>(h->r_packA);
-    __nv_bfloat16* pb = h->at<__nv_bfloat16>(h->r_packBT);
-    const int64_t grid_cap = (int64_t)h->num_sms * 8;
-    const int64_t vecs = (int64_t)P.n * P.RP * (h->cfg.d_in / 8);
-    const int grid_a = (int)std::min<int64_t>(ceil_div(vecs, 256), grid_cap);
-    tracked(h, kPackA, st, [&] { pack_a_kernel<<<grid_a, 256, 0, st>>>(D.ad, P.n, P.RP, h->cfg.d_in, pa); });
-    if (bp == BPack::RowPadded) {
-        int maxr16 = 16; for (const AdapterDev& a : P.ad) maxr16 = std::max(maxr16, a.rblk);
-        const int64_t per_adapter = h->cfg.d_out * (maxr16 / 8);
-        dim3 grid_b((unsigned)std::min<int64_t>(ceil_div(per_adapter, 256), 65535), (unsigned)P.n);
-        tracked(h, kPackB, st, [&] { pack_b_kernel<<<grid_b, 256, 0, st>>>(D.ad, P.RP, (int)h->cfg.d_out, pb); });
-        return PLORA_OK;
-    }
-    dim3 gb((unsigned)ceil_div(h->cfg.d_out, 128), (unsigned)P.n);
-    int maxr = 1; for (const AdapterDev& a : P.ad) maxr = std::max(maxr, a.rank);
-    const size_t smem_bt = (size_t)128 * (maxr + 2) * sizeof(__nv_bfloat16);
+// Packs every adapter's A and B into the saved buffer in the layouts the tensor-core operands want
+// (pack_ab_kernel), once per forward; the backward reads the same packs.
+void pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, void* saved, cudaStream_t st) {
+    if (P.n == 0) return;
+    const SavedLayout L = saved_layout(h, P);
+    uint8_t* sv = static_cast<uint8_t*>(saved);
+    int64_t most = 1;
+    for (const AdapterDev& a : P.ad)
+        most = std::max<int64_t>(most, (int64_t)a.rp16 * (h->cfg.d_in / 8) + h->cfg.d_out * (a.rp16 / 8));
+    const int gx = (int)std::min<int64_t>(ceil_div(most, 256), 1024);
     OutBlocks blocks{};
     blocks.n = h->nblk;
     for (int b = 0; b < kMaxOutBlocks; ++b) blocks.end[b] = h->blk_end[b];
-    tracked(h, kPackBT, st, [&] { pack_bt_kernel<<<gb, 256, smem_bt, st>>>(D.ad, P.RP, h->cfg.d_out, blocks, pb); });
-    return PLORA_OK;
+    tracked(h, kPack, st, [&] {
+        pack_ab_kernel<<<dim3((unsigned)gx, (unsigned)P.n), 256, 0, st>>>(
+            D.ad, P.RP, h->cfg.d_in, h->cfg.d_out, blocks, reinterpret_cast<__nv_bfloat16*>(sv + L.o_packA),
+            reinterpret_cast<__nv_bfloat16*>(sv + L.o_packB), (int64_t)((L.o_packB - L.o_packA) / 2),
+            (int64_t)((L.bytes - L.o_packB) / 2), h->at<int>(h->r_err));
+    });
+}
+
+// 3-D bf16 tensor map of the B pack [n][d_out][RP] (rank column innermost), 128-byte swizzle, a box of
+// 64 columns x box_rows rows of one adapter; rows past d_out read as zero.
+bool make_packb_map(CUtensorMap* m, const void* base, uint64_t RP, uint64_t d_out, uint64_t n, uint32_t box_rows) {
+    cuuint64_t dims[3] = {RP, d_out, n};
+    cuuint64_t strides[2] = {RP * 2, d_out * RP * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -685,13 +715,16 @@ const char* plora_status_string(plora_status s) {
         case PLORA_ERR_OOM: return "PLORA_ERR_OOM";
         case PLORA_ERR_CUDA: return "PLORA_ERR_CUDA";
         case PLORA_ERR_TIMEOUT: return "PLORA_ERR_TIMEOUT";
+        case PLORA_ERR_BOUNDS: return "PLORA_ERR_BOUNDS";
     }
     return "PLORA_ERR_UNKNOWN";
 }
 
 const char* plora_last_error(plora_handle h) { return h ? h->last_error.c_str() : ""; }
 
-int32_t plora_version(void) { return 101; }
+int32_t plora_version(void) { return 102; }
+
+int32_t plora_debug_build(void) { return kDeviceChecks ? 1 : 0; }
 
 // Output blocks of a config: 1 (one projection) or n_out_blocks, with the checks the header lists.
 plora_status check_out_blocks(const plora_config* cfg, int* nblk) {
@@ -776,8 +809,6 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
     carve(h->r_err, 256);
     carve(h->r_G, (size_t)h->max_h_rows * h->RPmax * h->esize);
     if (h->tc) {
-        carve(h->r_packA, (size_t)na * h->RPmax * cfg->d_in * 2);
-        carve(h->r_packBT, (size_t)na * h->RPmax * cfg->d_out * 2);
         carve(h->r_part, (size_t)h->max_slots * dtiles * kTileM * h->RPmax * sizeof(float));
         carve(h->r_cnt, (size_t)h->max_counters * sizeof(int32_t));
     }
@@ -803,9 +834,6 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
         if (e == cudaSuccess) e = (set_tc_attr<Op::ShrinkDy, Op::WgradB>());
         if (e == cudaSuccess) e = pair_setup<Op::BaseFwd>(h->pairs_fwd);
         if (e == cudaSuccess) e = pair_setup<Op::BaseDx>(h->pairs_dx);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(pack_bt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     128 * (PLORA_MAX_RANK + 2) * (int)sizeof(__nv_bfloat16));
     }
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -955,29 +983,31 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
     const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
-    pack_factors(h, P, D, fused ? BPack::RowPadded : BPack::Transposed, st);
-    // mPB: the transposed B pack (unfused expand, MN-major); mPBk / mPBk128: the row-padded B
-    // pack (fused expand, K-major; 256 rows for the 1-SM tile, 128 per CTA of an SM pair).
-    CUtensorMap mX, mW, mW128, mPA, mHk, mPB, mPBk, mPBk128;
-    const void* pb = h->at<void>(h->r_packBT);
+    pack_factors(h, P, D, saved, st);
+    // mPA16: the A pack in 16-row boxes (the shrink's K-major B); mPBk / mPBk128: the B pack, K-major,
+    // 256 rows for the 1-SM tile and the expand, 128 per CTA of an SM pair.
+    const SavedLayout L = saved_layout(h, P);
+    const uint8_t* sv = static_cast<const uint8_t*>(saved);
+    CUtensorMap mX, mW, mW128, mPA16, mHk, mPBk, mPBk128, mY;
     bool ok = make_map(&mX, X, d_in, P.T, d_in, 64, kTileM) &&
+              make_map(&mY, Y, d_out, P.T, d_out, 64, 32) &&
               make_map(&mW, W, d_in, d_out, d_in, 64, kTileN) &&
               make_map(&mW128, W, d_in, d_out, d_in, 64, kTileM) &&
-              make_map(&mPA, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, P.RP) &&
+              make_map(&mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
               make_map(&mHk, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
-              (fused ? make_map(&mPBk, pb, P.RP, (uint64_t)P.n * d_out, P.RP, 64, kTileN) &&
-                       make_map(&mPBk128, pb, P.RP, (uint64_t)P.n * d_out, P.RP, 64, kTileM)
-                     : make_map(&mPB, pb, d_out, (uint64_t)P.n * P.RP, d_out, 64, 64));
+              make_packb_map(&mPBk, sv + L.o_packB, P.RP, d_out, P.n, kTileN) &&
+              make_packb_map(&mPBk128, sv + L.o_packB, P.RP, d_out, P.n, kTileM);
     if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
     // K2: H'_i = s_i X_i A_i per 128-token tile (into the zero-padded blocks of `saved`).
     TcParams q = base_params(h, P, D);
     q.K_total = (int32_t)d_in;
     q.num_tiles = (int32_t)P.tok.size();
-    q.b_box_rows = P.RP;
     q.out = saved; q.out_ld = P.RP;
+    q.out_elems = P.h_rows * P.RP;
+    q.n_items = (int32_t)P.tok.size();
     narrow_ring(q, P.RP);
-    launch_tc<Op::ShrinkX>(h, mX, mPA, mX, mPA, q, st);
+    launch_tc<Op::ShrinkX>(h, mX, mPA16, mX, mPA16, mX, q, st);
     // K1 (+K3): Y = X W over all packed tokens; fused, each tile also accumulates H'_j B_j of
     // every adapter j overlapping it, so Y is written once.
     TcParams p = base_params(h, P, D);
@@ -989,9 +1019,9 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     p.fuse = fused ? 1 : 0;
     if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
         pair_params(p, P.T, d_out);
-        launch_pair<Op::BaseFwd>(h, mX, mW128, mHk, fused ? mPBk128 : mW128, p, st);
+        launch_pair<Op::BaseFwd>(h, mX, mW128, mHk, fused ? mPBk128 : mW128, mY, p, st);
     } else {
-        launch_tc<Op::BaseFwd>(h, mX, mW, mHk, fused ? mPBk : mW, p, st);
+        launch_tc<Op::BaseFwd>(h, mX, mW, mHk, fused ? mPBk : mW, mY, p, st);
     }
     if (!fused) {
         // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
@@ -1000,7 +1030,9 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
         r.tiles_n = (int32_t)ceil_div(d_out, kTileN);
         r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
         r.out = Y; r.out_ld = d_out;
-        launch_tc<Op::ExpandY>(h, mHk, mPB, mHk, mPB, r, st);
+        r.out_elems = P.T * d_out;
+        r.n_items = (int32_t)P.tok.size();
+        launch_tc<Op::ExpandY>(h, mHk, mPBk, mHk, mPBk, mHk, r, st);
     }
     return finish(h, D, st);
 }
@@ -1083,16 +1115,20 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     DevPlan D;
     s = upload(h, P, {}, st, D);
     if (s != PLORA_OK) return s;
-    pack_factors(h, P, D, BPack::Transposed, st);
-    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_k, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn;
-    bool ok = make_map(&mdY_k, dY, d_out, P.T, d_out, 64, kTileM) &&
+    // The factors were packed into `saved` by the forward; the backward packs nothing.
+    const SavedLayout L = saved_layout(h, P);
+    const uint8_t* sv = static_cast<const uint8_t*>(saved);
+    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_mn, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn, mdX;
+    // the output map of the dX GEMM (dX may be NULL: the GEMM is skipped then)
+    bool ok = (!dX || make_map(&mdX, dX, d_in, P.T, d_in, 64, 32)) &&
+              make_map(&mdY_k, dY, d_out, P.T, d_out, 64, kTileM) &&
               make_map(&mdY_mn, dY, d_out, P.T, d_out, 64, 64) &&
               make_map(&mW_mn, W, d_in, d_out, d_in, 64, 64) &&
-              make_map(&mPB_k, h->at<void>(h->r_packBT), d_out, (uint64_t)P.n * P.RP, d_out, 64, P.RP) &&
+              make_packb_map(&mPB_mn, sv + L.o_packB, P.RP, d_out, P.n, 64) &&
               make_map(&mG_k, G, P.RP, P.h_rows, P.RP, 64, kTileM) &&
               make_map(&mG_mn, G, P.RP, P.h_rows, P.RP, 64, 64) &&
-              make_map(&mPA_mn, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
-              make_map(&mPA16, h->at<void>(h->r_packA), d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
+              make_map(&mPA_mn, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
+              make_map(&mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
               make_map(&mH_mn, saved, P.RP, P.h_rows, P.RP, 64, 64) &&
               make_map(&mX_mn, X, d_in, P.T, d_in, 64, 64);
     if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
@@ -1102,8 +1138,9 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     TcParams q = base_params(h, P, D);
     q.K_total = (int32_t)d_out;
     q.num_tiles = (int32_t)P.tok.size();
-    q.b_box_rows = P.RP;
     q.out = G; q.out_ld = P.RP;
+    q.out_elems = (int64_t)(h->r_G.bytes / h->esize);
+    q.n_items = (int32_t)P.tok.size();
     narrow_ring(q, P.RP);
     // K7: dB_i = H'_i^T dY_i (a sum over each adapter's tokens) needs neither G nor dX, so its
     // items share K5's launch and fill the last wave of K5's equal-cost token tiles.
@@ -1111,8 +1148,9 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     wb.M_total = (int32_t)d_out;
     wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
     wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
+    wb.n_items = (int32_t)P.red.size();
     narrow_ring(wb, P.RP);
-    launch_tc2<Op::ShrinkDy, Op::WgradB>(h, mdY_k, mPB_k, mdY_mn, mH_mn, q, wb, kShrinkDyWgradB, st);
+    launch_tc2<Op::ShrinkDy, Op::WgradB>(h, mdY_k, mPB_mn, mdY_mn, mH_mn, q, wb, kShrinkDyWgradB, st);
     if (dX) {
         // K4 (+K6): dX = dY W^T; fused, each tile also accumulates G_j A_j^T of every adapter j
         // overlapping it, so dX is written once.
@@ -1124,9 +1162,9 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
         p.fuse = fused ? 1 : 0;
         if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
             pair_params(p, P.T, d_in);
-            launch_pair<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, p, st);
+            launch_pair<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, mdX, p, st);
         } else {
-            launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, p, st);
+            launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, mdX, p, st);
         }
         if (!fused) {
             // K6 as its own pass: dX_i += G_i A_i^T (read-modify-write of dX).
@@ -1135,7 +1173,9 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
             r.tiles_n = (int32_t)ceil_div(d_in, kTileN);
             r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
             r.out = dX; r.out_ld = d_in;
-            launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, mG_k, mPA_mn, r, st);
+            r.out_elems = P.T * d_in;
+            r.n_items = (int32_t)P.tok.size();
+            launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, mG_k, mPA_mn, mG_k, r, st);
         }
     }
     // K8: dA_i = X_i^T G_i (a sum over each adapter's tokens).
@@ -1143,8 +1183,9 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
     wa.M_total = (int32_t)d_in;
     wa.red_dtiles = (int32_t)ceil_div(d_in, kTileM);
     wa.num_tiles = (int32_t)P.red.size() * wa.red_dtiles;
+    wa.n_items = (int32_t)P.red.size();
     narrow_ring(wa, P.RP);
-    launch_tc<Op::WgradA>(h, mX_mn, mG_mn, mX_mn, mG_mn, wa, st);
+    launch_tc<Op::WgradA>(h, mX_mn, mG_mn, mX_mn, mG_mn, mX_mn, wa, st);
     return finish(h, D, st);
 }
 
@@ -1166,6 +1207,8 @@ plora_status plora_check(plora_handle h, void* stream) {
     if (flag != 0) {
         int zero = 0;
         cudaMemcpy(h->at<int>(h->r_err), &zero, sizeof(int), cudaMemcpyHostToDevice);
+        if (flag == kErrBounds)
+            return fail(h, PLORA_ERR_BOUNDS, "a device-side bounds check failed; the access was skipped");
         return fail(h, PLORA_ERR_TIMEOUT, "a device-side wait ran out of time (flag %d)", flag);
     }
     return PLORA_OK;
@@ -1600,8 +1643,13 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     p.M_total = (int32_t)d_out;
     p.red_dtiles = dtiles;
     p.num_tiles = (int32_t)P.red.size() * dtiles;
+    p.n_adapters = P.n;
+    p.n_items = (int32_t)P.red.size();
+    p.part_elems = (int64_t)((kStaticScratchBytes - L.o_part) / sizeof(float));
+    p.n_counters = (int32_t)(L.cnt_bytes / sizeof(int32_t));
     narrow_ring(p, P.RP);
     if (p.num_tiles > 0)
-        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, mdY, mH, p, p);
+        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, mdY, mH, mdY,
+                                                                                                    p, p);
     return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
 }

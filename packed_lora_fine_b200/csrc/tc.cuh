@@ -10,9 +10,9 @@
 //   BaseFwd    Y  = X W            (all tokens)          X      K-major          W_store    K-major
 //   BaseDx     dX = dY W^T         (all tokens)          dY     K-major          W_store    MN-major
 //   ShrinkX    H_i = X_i A_i       (per 128-token tile)   X      K-major          A pack     K-major
-//   ShrinkDy   G_i = s_i dY_i B_i^T                       dY     K-major          B^T pack   K-major
-//   ExpandY    Y_i += s_i H_i B_i                         H      K-major          B^T pack   MN-major
-//              (by default folded into BaseFwd instead: B row-padded pack, K-major)
+//   ShrinkDy   G_i = s_i dY_i B_i^T                       dY     K-major          B pack     MN-major
+//   ExpandY    Y_i += s_i H_i B_i                         H      K-major          B pack     K-major
+//              (by default folded into BaseFwd instead, with the same B pack)
 //   ExpandDx   dX_i += G_i A_i^T                          G      K-major          A pack     MN-major
 //   WgradB     dB_i = s_i dY_i^T H_i (sum over tokens)    dY     MN-major         H          MN-major
 //   WgradA     dA_i = X_i^T G_i      (sum over tokens)    X      MN-major         G          MN-major
@@ -50,7 +50,7 @@ enum class Op : int { BaseFwd = 0, BaseDx, ShrinkX, ShrinkDy, ExpandY, ExpandDx,
 
 template <Op OP> struct OpTraits {
     static constexpr bool kAmn = (OP == Op::WgradB || OP == Op::WgradA);
-    static constexpr bool kBmn = (OP == Op::BaseDx || OP == Op::ExpandY || OP == Op::ExpandDx ||
+    static constexpr bool kBmn = (OP == Op::BaseDx || OP == Op::ShrinkDy || OP == Op::ExpandDx ||
                                   OP == Op::WgradB || OP == Op::WgradA);
     static constexpr bool kBase = (OP == Op::BaseFwd || OP == Op::BaseDx);
     static constexpr bool kShrink = (OP == Op::ShrinkX || OP == Op::ShrinkDy);
@@ -67,8 +67,17 @@ constexpr int kStageBytes = kABytes + kBBytesMax;
 constexpr int kTmemCols = 512;                    // two 256-column fp32 accumulators
 constexpr int kTcThreads = 192;
 constexpr int kRingBytes = kStages * kStageBytes; // 192 KB of operand ring
-constexpr int kEpiStageFloats = 32 * 33;          // per epilogue warp: a 32 x 32 fp32 chunk (padded rows)
-constexpr int kTcSmemBytes = kRingBytes + 1024 /* align */ + 256 /* barriers */ + 4 * kEpiStageFloats * 4;
+// Epilogue staging, per epilogue warp: two 4 KB buffers, each one 128-byte-swizzled TMA box of 32 rows x
+// 64 bf16 (the base GEMMs' output stores); the dB epilogue uses the same space for a 32 x 33 fp32 chunk.
+constexpr int kEpiBufBytes = 32 * 64 * 2;
+constexpr int kEpiWarpBytes = 2 * kEpiBufBytes;
+constexpr int kEpiStageFloats = 32 * 33;
+static_assert(kEpiStageFloats * 4 <= kEpiWarpBytes, "dB staging fits a warp's epilogue space");
+// Layout: [operand ring][4 warps' epilogue staging][barriers], from a 1024-byte-aligned base.
+constexpr int kEpiOffset = kRingBytes;
+constexpr int kBarOffset = kRingBytes + 4 * kEpiWarpBytes;
+constexpr int kTcSmemBytes = kBarOffset + 256 /* barriers */ + 1024 /* align */;
+static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
 
 struct TcParams {
     int32_t M_total;        // Base: T; Wgrad: d (rows of dB_i or columns of dA_i)
@@ -77,7 +86,7 @@ struct TcParams {
     int32_t tiles_m, tiles_n, num_tiles;
     int32_t group_m;        // Base: rasterisation group (m tiles sharing an L2 window)
     int32_t RP;             // padded rank pitch of H / G / packs
-    int32_t b_box_rows;     // K-major B: rows of the B box (Base: 256, Shrink: RP)
+    int32_t b_box_rows;     // BaseFwd: rows of the K-major B box (256)
     int32_t red_dtiles;     // Wgrad: 128-row tiles along d
     const AdapterDev* adapters;
     const TokTile* tok;
@@ -99,6 +108,13 @@ struct TcParams {
     // columns [blk_end[b-1], blk_end[b]); nblk = 1 for a single projection.
     int32_t nblk;
     int32_t blk_end[kMaxOutBlocks];
+    // Extents of what the kernel addresses through plain pointers (checked by the PLORA_DEBUG build).
+    int64_t out_elems;      // elements of the output buffer `out`
+    int64_t part_elems;     // floats of the split partials
+    int32_t n_counters;     // ints of the arrival counters
+    int32_t n_adapters;     // entries of the adapter table
+    int32_t n_items;        // entries of tok (shrink, expand) or red (weight gradients)
+    int32_t n_mtrec, n_mtseg;   // entries of mt_rec, mt_seg
 };
 
 // The output block holding output column `col`.
@@ -109,19 +125,20 @@ __device__ __forceinline__ int out_block(const TcParams& p, int col) {
 }
 
 struct TileInfo {
-    int32_t a_x, a_y, b_x, b_y;
+    int32_t a_x, a_y, b_x, b_y, b_z;
     int32_t kblocks, last_ksteps, mma_n, nb_boxes;
-    int32_t adapter, out_row, rows_valid, n0, cols_valid, red_idx;
+    int32_t adapter, out_row, rows_valid, n0, cols_valid, cols_live, red_idx;
     int32_t mtile;
     float scale;
 };
 
 template <Op OP>
-__device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
+__device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {  // t: work item (a copy)
     using Tr = OpTraits<OP>;
     TileInfo ti;
     ti.last_ksteps = 4;
     ti.nb_boxes = 1;
+    ti.b_z = 0;
     ti.scale = 1.f;
     ti.adapter = -1;
     ti.red_idx = -1;
@@ -146,31 +163,55 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         ti.n0 = nb * kTileN;
         ti.cols_valid = min(kTileN, p.N_total - ti.n0);
     } else if constexpr (Tr::kShrink) {
-        const TokTile tt = p.tok[t];
+        if (!dcheck(p.err_flag, t >= 0 && t < p.n_items)) t = 0;
+        TokTile tt = p.tok[t];
+        if (!dcheck(p.err_flag, tt.adapter >= 0 && tt.adapter < p.n_adapters && tt.rows >= 1 && tt.rows <= kTileM))
+            tt = p.tok[0];
         const AdapterDev ad = p.adapters[tt.adapter];
         ti.adapter = tt.adapter;
         ti.a_x = 0;
         ti.a_y = tt.x_row;
         ti.b_x = 0;
-        ti.b_y = tt.adapter * p.RP;
+        if constexpr (OP == Op::ShrinkX) {
+            // B = the adapter's rp16 rows of the A pack, K-major, in 16-row boxes
+            ti.b_y = tt.adapter * p.RP;
+            ti.mma_n = ad.rp16;
+            ti.nb_boxes = ad.rp16 / 16;
+        } else {
+            // B = the adapter's B pack [d_out][RP] read MN-major (64 rank columns x 64 rows per box)
+            // over rp64 columns; the columns past rp16 are not the adapter's and are stored as zeros
+            ti.b_y = 0;
+            ti.b_z = tt.adapter;
+            ti.mma_n = ad.rp64;
+            ti.nb_boxes = ad.rp64 / 64;
+        }
         ti.kblocks = (p.K_total + kBlockK - 1) / kBlockK;
-        ti.mma_n = ad.rp16;
         ti.out_row = tt.h_row;
         ti.rows_valid = tt.rows;
         ti.n0 = 0;
         ti.cols_valid = p.RP;
+        ti.cols_live = ad.rp16;
         ti.scale = ad.scale;   // H' = s X A and G = s dY B^T carry the adapter's scale
     } else if constexpr (Tr::kExpand) {
-        const int mt = t / p.tiles_n;
+        int mt = t / p.tiles_n;
         const int nb = t - mt * p.tiles_n;
-        const TokTile tt = p.tok[mt];
+        if (!dcheck(p.err_flag, mt >= 0 && mt < p.n_items)) mt = 0;
+        TokTile tt = p.tok[mt];
+        if (!dcheck(p.err_flag, tt.adapter >= 0 && tt.adapter < p.n_adapters)) tt = p.tok[0];
         const AdapterDev ad = p.adapters[tt.adapter];
         ti.adapter = tt.adapter;
         ti.a_x = 0;
         ti.a_y = tt.h_row;
-        ti.b_x = nb * kTileN;
-        ti.b_y = tt.adapter * p.RP;
-        ti.nb_boxes = kTileN / 64;
+        if constexpr (OP == Op::ExpandY) {
+            // B = rows nb*256.. of the adapter's B pack, K-major (3-D map: rank column, row, adapter)
+            ti.b_x = 0;
+            ti.b_y = nb * kTileN;
+            ti.b_z = tt.adapter;
+        } else {
+            ti.b_x = nb * kTileN;
+            ti.b_y = tt.adapter * p.RP;
+            ti.nb_boxes = kTileN / 64;
+        }
         const int ksteps = ad.rp16 / 16;
         ti.kblocks = (ksteps + 3) / 4;
         ti.last_ksteps = ksteps - (ti.kblocks - 1) * 4;
@@ -181,9 +222,11 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {
         ti.cols_valid = min(kTileN, p.N_total - ti.n0);
         ti.scale = 1.f;        // H' and G already carry the scale
     } else {
-        const int e = t / p.red_dtiles;
+        int e = t / p.red_dtiles;
         const int db = t - e * p.red_dtiles;
-        const RedEntry re = p.red[e];
+        if (!dcheck(p.err_flag, e >= 0 && e < p.n_items)) e = 0;
+        RedEntry re = p.red[e];
+        if (!dcheck(p.err_flag, re.adapter >= 0 && re.adapter < p.n_adapters)) re = p.red[e = 0];
         const AdapterDev ad = p.adapters[re.adapter];
         ti.adapter = re.adapter;
         ti.red_idx = e;
@@ -216,7 +259,10 @@ __device__ __forceinline__ MTileRec load_mtile(const TcParams& p, int t) {
     r.q0 = r.q1 = 0;
     if (OpTraits<OP>::kBase && p.fuse && t < p.num_tiles) {
         const TileInfo ti = decode_tile<OP>(p, t);
-        r = p.mt_rec[ti.mtile / (kLoraTileM / kTileM)];
+        const int rec = ti.mtile / (kLoraTileM / kTileM);
+        if (!dcheck(p.err_flag, rec >= 0 && rec < p.n_mtrec)) return r;
+        r = p.mt_rec[rec];
+        if (!dcheck(p.err_flag, r.q0 >= 0 && r.q0 <= r.q1 && r.q1 <= p.n_mtseg)) r.q1 = r.q0;
         // a 128-row tile reads its half of the 256-row record's rows
         const int shift = (ti.mtile % (kLoraTileM / kTileM)) * kTileM;
         r.s[0].h_y += shift;
@@ -226,7 +272,8 @@ __device__ __forceinline__ MTileRec load_mtile(const TcParams& p, int t) {
     return r;
 }
 __device__ __forceinline__ LoraSeg mtile_seg(const TcParams& p, const MTileRec& r, int q) {
-    if (q - r.q0 < 2) return r.s[q - r.q0];
+    if (q == r.q0) return r.s[0];       // constant indices keep the record in registers
+    if (q == r.q0 + 1) return r.s[1];
     LoraSeg s = p.mt_seg[q];
     s.h_y += r.pad_[0];
     return s;
@@ -260,7 +307,11 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
                                              RingPos& rp, uint32_t& armed, uint32_t& armed_par,
                                              volatile int* abort_flag, uint64_t lim) {
     using Tr = OpTraits<OP>;
-    const uint32_t b_bytes = Tr::kBmn ? (uint32_t)ti.nb_boxes * 8192u : (uint32_t)p.b_box_rows * 128u;
+    uint32_t b_bytes;
+    if constexpr (OP == Op::ShrinkX) b_bytes = (uint32_t)ti.mma_n * 128u;        // rp16 rows of 64
+    else if constexpr (OP == Op::ExpandY) b_bytes = (uint32_t)kTileN * 128u;     // 256 rows of 64
+    else if constexpr (Tr::kBmn) b_bytes = (uint32_t)ti.nb_boxes * 8192u;        // 64 x 64 boxes
+    else b_bytes = (uint32_t)p.b_box_rows * 128u;
     for (int kb = 0; kb < ti.kblocks; ++kb) {
         if (!ptx::mbar_wait(&empty_bar[rp.stage], rp.phase ^ 1u, abort_flag, lim, p.err_flag)) return false;
         uint8_t* sA = smem + rp.stage * stb;
@@ -274,7 +325,15 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
         } else {
             ptx::tma_load_2d(sA, tmA, &full_bar[rp.stage], ti.a_x + kb * kBlockK, ti.a_y);
         }
-        if constexpr (Tr::kBmn) {
+        if constexpr (OP == Op::ShrinkX) {
+            for (int h = 0; h < ti.nb_boxes; ++h)
+                ptx::tma_load_2d(sB + h * 2048, tmB, &full_bar[rp.stage], kb * kBlockK, ti.b_y + 16 * h);
+        } else if constexpr (OP == Op::ShrinkDy) {
+            for (int h = 0; h < ti.nb_boxes; ++h)
+                ptx::tma_load_3d(sB + h * 8192, tmB, &full_bar[rp.stage], 64 * h, kb * kBlockK, ti.b_z);
+        } else if constexpr (OP == Op::ExpandY) {
+            ptx::tma_load_3d(sB, tmB, &full_bar[rp.stage], kb * kBlockK, ti.b_y, ti.b_z);
+        } else if constexpr (Tr::kBmn) {
             for (int h = 0; h < ti.nb_boxes; ++h)
                 ptx::tma_load_2d(sB + h * 8192, tmB, &full_bar[rp.stage], ti.b_x + 64 * h, ti.b_y + kb * kBlockK);
         } else {
@@ -287,10 +346,10 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
         // tokens overlap this m-tile, K-steps over its rank with A = its H' (or G) rows,
         // read at the tile's row offset inside j's zero-padded block (rows outside j's
         // segment load as zeros).  B has the base B's major-ness: for Y, rows n0.. of
-        // j's row-padded B (K-major, one 256 x 64 box); for dX, j's packed A
-        // (MN-major, 16-row boxes so that only the rank's rows are staged).  With output
-        // blocks, Y's tile reads only its block's columns of H' (K = rblk from b rblk); dX's
-        // sums over every block (K = P rblk).
+        // j's B pack (K-major, one 256 x 64 box); for dX, j's packed A (MN-major, 16-row
+        // boxes so that only the rank's rows are staged).  With output blocks, Y's tile reads
+        // only its block's columns of H' and of the block-diagonal B pack (K = rblk from
+        // b rblk); dX's sums over every block (K = P rblk).
         for (int q = lr.q0; q < lr.q1; ++q) {
             const LoraSeg sg = mtile_seg(p, lr, q);
             const int kext = Tr::kBmn ? sg.rp16 : sg.rblk;
@@ -311,7 +370,8 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
                             ptx::tma_load_2d(sB + h * R * 128 + r16 * 128, tmB2, &full_bar[rp.stage],
                                              ti.n0 + 64 * h, sg.adapter * p.RP + kb * kBlockK + r16);
                 } else {
-                    ptx::tma_load_2d(sB, tmB2, &full_bar[rp.stage], kb * kBlockK, sg.adapter * p.N_total + ti.n0);
+                    // the block-diagonal B pack holds block b's B in the same columns as H'
+                    ptx::tma_load_3d(sB, tmB2, &full_bar[rp.stage], hx0 + kb * kBlockK, ti.n0, sg.adapter);
                 }
                 rp.advance(nst);
             }
@@ -328,19 +388,21 @@ __device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, 
                                          uint32_t d_tmem, RingPos& rp, volatile int* abort_flag, uint64_t lim) {
     using Tr = OpTraits<OP>;
     const uint32_t idesc = ptx::idesc_bf16_f32(kTileM, ti.mma_n, Tr::kAmn, Tr::kBmn);
+    // Descriptors of stage 0; a stage and a k-step only move the start address (bits 0-13, in 16-byte
+    // units; shared addresses stay below 2^18 bytes, so the sum never carries out of the field).
+    const uint32_t s0 = ptx::smem_u32(smem);
+    const uint64_t adesc0 = Tr::kAmn ? ptx::smem_desc_sw128(s0, 8192, 1024) : ptx::smem_desc_sw128(s0, 16, 1024);
+    const uint64_t bdesc0 = Tr::kBmn ? ptx::smem_desc_sw128(s0 + kABytes, 8192, 1024)
+                                     : ptx::smem_desc_sw128(s0 + kABytes, 16, 1024);
+    constexpr uint32_t kAstep = Tr::kAmn ? 2048 / 16 : 32 / 16;
+    constexpr uint32_t kBstep = Tr::kBmn ? 2048 / 16 : 32 / 16;
     for (int kb = 0; kb < ti.kblocks; ++kb) {
         if (!ptx::mbar_wait(&full_bar[rp.stage], rp.phase, abort_flag, lim, p.err_flag)) return false;
         ptx::tc_fence_after();
-        const uint32_t sA = ptx::smem_u32(smem + rp.stage * stb);
-        const uint32_t sB = sA + kABytes;
+        const uint64_t so = (uint64_t)((uint32_t)(rp.stage * stb) >> 4);
         const int steps = (kb == ti.kblocks - 1) ? ti.last_ksteps : 4;
-        for (int ks = 0; ks < steps; ++ks) {
-            const uint64_t adesc = Tr::kAmn ? ptx::smem_desc_sw128(sA + ks * 2048, 8192, 1024)
-                                            : ptx::smem_desc_sw128(sA + ks * 32, 16, 1024);
-            const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, 8192, 1024)
-                                            : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
-            ptx::tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | ks) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < steps; ++ks)
+            ptx::tc_mma_f16(d_tmem, adesc0 + so + ks * kAstep, bdesc0 + so + ks * kBstep, idesc, (kb | ks) ? 1u : 0u);
         ptx::tc_commit(&empty_bar[rp.stage]);
         rp.advance(nst);
     }
@@ -368,39 +430,65 @@ __device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, 
     return true;
 }
 
+// Base-GEMM epilogue of one epilogue warp: its 32 accumulator rows (TMEM lanes from t_row) x 256
+// columns, rounded to bf16 (nearest even) and written to rows row0.. and columns n0.. of the output
+// through its two staging buffers: per 64 columns, the lanes write their rows into a 128-byte-swizzled
+// 32 x 64 box (16-byte stores, conflict-free) and one lane issues a TMA tensor store, so whole lines
+// reach L2 and the conversion of a chunk overlaps the store of the one before.  The store clips rows
+// and columns outside the output tensor.
+__device__ __forceinline__ void epilogue_store_tma(const CUtensorMap* tmC, uint32_t t_row, uint8_t* wbuf, int lane,
+                                                   int row0, int n0, int M_total, int N_total) {
+    if (row0 >= M_total) return;
+    const uint32_t sw = (uint32_t)(lane & 7);
+    for (int ch = 0; ch < kTileN / 64; ++ch) {
+        const int col0 = n0 + ch * 64;
+        if (col0 >= N_total) break;
+        uint32_t ra[32], rb[32];
+        ptx::tmem_ld32(t_row + ch * 64, ra);
+        ptx::tmem_ld32(t_row + ch * 64 + 32, rb);
+        ptx::tmem_ld_wait();
+        uint8_t* buf = wbuf + (ch & 1) * kEpiBufBytes;
+        if (lane == 0) ptx::bulk_wait_read<1>();   // the store that last read this buffer is done
+        __syncwarp();
+        const uint32_t rowaddr = ptx::smem_u32(buf) + (uint32_t)lane * 128u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t* v = j < 4 ? ra + 8 * j : rb + 8 * (j - 4);
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+            o.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+            o.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+            o.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+            ptx::st_shared_v4(rowaddr + ((((uint32_t)j) ^ sw) << 4), o);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            ptx::tma_store_2d(tmC, buf, col0, row0);
+            ptx::bulk_commit();
+        }
+    }
+}
+
 // Epilogue (warps 2..5, one accumulator row per thread): drains work item ti's accumulator
 // rows from TMEM at t_row and runs the op's output step.
 template <Op OP>
 __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo& ti, uint32_t t_row, int q, int lane,
-                                              float* epi_stage, int* red_flag) {
+                                              uint8_t* wbuf, const CUtensorMap* tmC, int* red_flag) {
     using Tr = OpTraits<OP>;
     const int row = q * 32 + lane;          // accumulator row handled by this thread
     const bool row_ok = row < ti.rows_valid;
+    float* epi_stage = reinterpret_cast<float*>(wbuf);
     if constexpr (Tr::kBase) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
-        for (int c = 0; c < kTileN; c += 16) {
-            uint32_t r[16];
-            ptx::tmem_ld16(t_row + c, r);
-            ptx::tmem_ld_wait();
-            if (row_ok) {
-                uint4 v0, v1;
-                v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                if (c + 8 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c) = v0;
-                if (c + 16 <= ti.cols_valid) *reinterpret_cast<uint4*>(out + c + 8) = v1;
-            }
-        }
+        epilogue_store_tma(tmC, t_row, wbuf, lane, ti.out_row + q * 32, ti.n0, p.M_total, p.N_total);
     } else if constexpr (Tr::kShrink) {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld;
+        // (the TMEM loads below are warp-collective: a failed check skips this thread's stores only)
+        const bool out_ok = dcheck(p.err_flag, ti.out_row + row >= 0 && ti.cols_valid <= p.out_ld &&
+                                                   (int64_t)(ti.out_row + row + 1) * p.out_ld <= p.out_elems);
         for (int c = 0; c < ti.cols_valid; c += 16) {
             uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-            if (c < ti.mma_n) {
+            if (c < ti.cols_live) {
                 uint32_t r[16];
                 ptx::tmem_ld16(t_row + c, r);
                 ptx::tmem_ld_wait();
@@ -416,8 +504,10 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
                     v1.w = pack_bf16x2(s * __uint_as_float(r[14]), s * __uint_as_float(r[15]));
                 }
             }
-            *reinterpret_cast<uint4*>(out + c) = v0;
-            *reinterpret_cast<uint4*>(out + c + 8) = v1;
+            if (out_ok) {
+                *reinterpret_cast<uint4*>(out + c) = v0;
+                *reinterpret_cast<uint4*>(out + c + 8) = v1;
+            }
         }
         // The adapter's block has kLoraPad zero rows before and after its (128-rounded) rows, so that
         // a base tile straddling the segment can read it at any row offset; the first and the last
@@ -429,7 +519,9 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
             const uint4 z = make_uint4(0, 0, 0, 0);
             __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.out);
             const int tail = ad.h_row + ((ad.n + kTileM - 1) / kTileM) * kTileM;
-            for (int pr = row; pr < kLoraPad; pr += kTileM) {
+            const bool pads_ok = dcheck(p.err_flag, ad.h_row - kLoraPad >= 0 && p.RP <= p.out_ld &&
+                                                        (int64_t)(tail + kLoraPad) * p.out_ld <= p.out_elems);
+            for (int pr = row; pr < kLoraPad && pads_ok; pr += kTileM) {
                 if (first) {
                     uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)(ad.h_row - kLoraPad + pr) * p.out_ld);
                     for (int c = 0; c < p.RP / 8; ++c) dst[c] = z;
@@ -443,9 +535,12 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
     } else if constexpr (Tr::kExpand) {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld + ti.n0;
         const float s = ti.scale;
+        // (the TMEM loads below are warp-collective: a failed check skips this thread's accesses only)
+        const bool rw = row_ok && dcheck(p.err_flag, ti.n0 + ti.cols_valid <= p.out_ld &&
+                                                         (int64_t)(ti.out_row + row + 1) * p.out_ld <= p.out_elems);
         for (int h = 0; h < kTileN; h += 128) {
             uint4 y[16];
-            if (row_ok) {
+            if (rw) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
                     if (h + 8 * u + 8 <= ti.cols_valid) y[u] = *reinterpret_cast<const uint4*>(out + h + 8 * u);
@@ -455,7 +550,7 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
                 uint32_t r[16];
                 ptx::tmem_ld16(t_row + h + 8 * u, r);
                 ptx::tmem_ld_wait();
-                if (row_ok) {
+                if (rw) {
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
                         if (h + 8 * (u + w) + 8 > ti.cols_valid) continue;
@@ -484,7 +579,7 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
             // dB_i's 128-row tile is one contiguous block ([row][rank]); stage 32 x 32 chunks of
             // this warp's rows in shared memory and store them with consecutive lanes on
             // consecutive addresses.
-            float* stg = epi_stage + q * kEpiStageFloats;
+            float* stg = epi_stage;
             const int row0 = ti.out_row + q * 32;                 // first hidden row of this warp
             const int nrows = min(32, p.M_total - row0);
             float* blk = ad.dB + (int64_t)row0 * rank;
@@ -536,6 +631,11 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
             // partial layout [slot][d-tile][rank column][128 rows]: a warp's lanes touch
             // consecutive rows, so both the writes here and the reduction below coalesce.
             float* mine = p.partials + ((int64_t)(re.slot + re.split) * p.red_dtiles + ti.n0) * slot_elems + row;
+            const bool split_ok = dcheck(p.err_flag, re.slot >= 0 && re.counter >= 0 && re.split < re.nsplit &&
+                                                         ((int64_t)(re.slot + re.nsplit - 1) * p.red_dtiles + ti.n0 + 1) *
+                                                                 slot_elems <= p.part_elems &&
+                                                         re.counter + ti.n0 < p.n_counters);
+            if (!split_ok) return;   // every thread of the tile takes the same branch
             for (int c = 0; c < ti.mma_n; c += 16) {
                 uint32_t r[16];
                 ptx::tmem_ld16(t_row + c, r);
@@ -597,8 +697,8 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
 template <Op OP, Op OP2 = OP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const TcParams p,
-          const TcParams p2) {
+          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+          const __grid_constant__ CUtensorMap tmC, const TcParams p, const TcParams p2) {
     using Tr = OpTraits<OP>;
     constexpr bool kDual = OP2 != OP;
     static_assert(!kDual || (!Tr::kBase && !OpTraits<OP2>::kBase),
@@ -606,7 +706,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int total = p.num_tiles + (kDual ? p2.num_tiles : 0);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
     uint64_t* full_bar = bars;                       // [kMaxStages]
     uint64_t* empty_bar = bars + kMaxStages;         // [kMaxStages]
     uint64_t* accf_bar = bars + 2 * kMaxStages;      // [2]
@@ -617,7 +717,6 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int stb = p.stage_bytes;                   // bytes per stage (multiple of 1024)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* red_flag = reinterpret_cast<int*>(tmem_slot + 2);
-    float* epi_stage = reinterpret_cast<float*>(smem + kRingBytes + 256);   // [4 warps][32][33]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -638,6 +737,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     if (warp == 0 && lane == 0) {
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
+        if (Tr::kBase) ptx::tma_prefetch_desc(&tmC);
         if ((Tr::kBase && p.fuse) || kDual) {
             ptx::tma_prefetch_desc(&tmA2);
             ptx::tma_prefetch_desc(&tmB2);
@@ -708,6 +808,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        uint8_t* wbuf = smem + kEpiOffset + q * kEpiWarpBytes;
         int abuf = 0;
         uint32_t aphase = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -715,14 +816,16 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
             if (kDual && t >= p.num_tiles)
-                epilogue_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), t_row, q, lane, epi_stage, red_flag);
+                epilogue_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), t_row, q, lane, wbuf, &tmC, red_flag);
             else
-                epilogue_item<OP>(p, decode_tile<OP>(p, t), t_row, q, lane, epi_stage, red_flag);
+                epilogue_item<OP>(p, decode_tile<OP>(p, t), t_row, q, lane, wbuf, &tmC, red_flag);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
             if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
         }
+        // Every output store has been performed before the CTA (and its staging) goes away.
+        if (Tr::kBase && lane == 0) ptx::bulk_wait<0>();
     }
 
     ptx::tc_fence_before();
@@ -732,109 +835,66 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 }
 
 // ---------------------------------------------------------------------------
-// Packing of the small per-adapter factors into the MMA-ready padded layouts.
-//   packA [n*RP][d_in]:  row i*RP + b*rblk_i + k = A_i[b*r_i + k][:] (k < r_i), zero up to rblk_i
-//   packBT[n*RP][d_out]: row i*RP + b*rblk_i + k = B_i[:][k] on block b's columns (k < r_i), else zero
-// (b = output block, rblk_i = r_i rounded up to 16; one block: b = 0 and rblk_i = rp16_i).
-// Rows rp16_i <= k < RP are never read by an MMA and are left unwritten.
+// Packing of the small per-adapter factors into the MMA-ready padded layouts, once per forward, into
+// the `saved` buffer that the backward reads as well (b = output block, rblk_i = r_i rounded up to 16,
+// rp16_i = P rblk_i; one block: b = 0 and rblk_i = rp16_i):
+//   packA [n RP][d_in]:    row i RP + b rblk_i + k = A_i[b r_i + k][:] for k < r_i, zero up to rblk_i
+//   packB [n][d_out][RP]:  packB[i][c][b rblk_i + k] = B_i[c][k] if column c lies in block b and k < r_i,
+//                          else zero (block-diagonal over the output blocks)
+// packA rows at or past rp16_i and packB columns at or past rp16_i are never multiplied (the shrink of
+// G reads them and discards the accumulator columns) and stay unwritten.
+//
+// packA feeds the shrink of H (K-major) and the fold of G A^T into dX (MN-major); packB feeds the fold
+// of H' B into Y (K-major, block b's columns) and the shrink of G = s dY B^T (MN-major: column
+// b rblk + k of G sums over block b's output columns only, as output blocks need).
 // ---------------------------------------------------------------------------
-__global__ void pack_a_kernel(const AdapterDev* __restrict__ ad, int n, int RP, int64_t d_in,
-                              __nv_bfloat16* __restrict__ packA) {
-    const int64_t vec_per_row = d_in / 8;
-    const int64_t total = (int64_t)n * RP * vec_per_row;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t rowi = e / vec_per_row;
-        const int64_t v = e - rowi * vec_per_row;
-        const int i = (int)(rowi / RP);
-        const int j = (int)(rowi - (int64_t)i * RP);
-        if (j >= ad[i].rp16) continue;   // rows past the MMA extent are never read
-        // row j is output block pb's rank row k (A_store row pb rank + k)
-        const int pb = j / ad[i].rblk, k = j - pb * ad[i].rblk;
+// grid (gx, n adapters), block 256: per adapter, a grid-stride loop over its 16-byte chunks, first the
+// rp16 x d_in/8 chunks of packA, then the d_out x rp16/8 chunks of packB (consecutive threads on
+// consecutive bytes of both sources and destinations).
+__global__ void __launch_bounds__(256) pack_ab_kernel(const AdapterDev* __restrict__ ad, int RP, int64_t d_in,
+                                                      int64_t d_out, OutBlocks blocks,
+                                                      __nv_bfloat16* __restrict__ packA,
+                                                      __nv_bfloat16* __restrict__ packB, int64_t packA_elems,
+                                                      int64_t packB_elems, int* err_flag) {
+    const int i = blockIdx.y;
+    const AdapterDev a = ad[i];
+    const int r = a.rank, rblk = a.rblk;
+    const int64_t va = d_in / 8;
+    const int64_t ua = (int64_t)a.rp16 * va;
+    const int vb = a.rp16 / 8;
+    const int64_t ub = d_out * vb;
+    const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A);
+    const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(a.B);
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < ua + ub; e += (int64_t)gridDim.x * blockDim.x) {
         uint4 val = make_uint4(0, 0, 0, 0);
-        if (k < ad[i].rank)
-            val = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ad[i].A) +
-                                                 (int64_t)(pb * ad[i].rank + k) * d_in)[v];
-        reinterpret_cast<uint4*>(packA + rowi * d_in)[v] = val;
-    }
-}
-
-// Row-padded copy of every B for the fused forward (the expand's B operand, K-major like W):
-// packB[(i d_out + c) RP + k] = B_i[c][k] for k < r_i, 0 for r_i <= k < rblk_i (r_i rounded up to
-// 16); columns at or past rblk_i are never multiplied and stay unwritten.  grid.y = adapter; one thread per 16-byte
-// chunk of the rp16_i columns, so consecutive threads read consecutive bytes of B_i.
-__global__ void __launch_bounds__(256) pack_b_kernel(const AdapterDev* __restrict__ ad, int RP, int d_out,
-                                                     __nv_bfloat16* __restrict__ packB) {
-    const int i = blockIdx.y;
-    const int r = ad[i].rank;
-    const unsigned vc = (unsigned)ad[i].rblk / 8u;          // chunks per row
-    const unsigned total = (unsigned)d_out * vc;
-    const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(ad[i].B);
-    __nv_bfloat16* dst = packB + (int64_t)i * d_out * RP;
-    for (unsigned e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-        const unsigned c = e / vc;
-        const int ch = (int)(e - c * vc);
-        const __nv_bfloat16* src = B + (int64_t)c * r;
-        uint4 val;
-        if ((r & 7) == 0 && ch * 8 < r) {
-            val = reinterpret_cast<const uint4*>(src)[ch];
+        if (e < ua) {
+            const int j = (int)(e / va);
+            const int64_t v = e - (int64_t)j * va;
+            const int pb = j / rblk, k = j - pb * rblk;      // output block pb's rank row k
+            if (!dcheck(err_flag, pb < blocks.n && j < RP && ((int64_t)i * RP + j) * d_in + (v + 1) * 8 <= packA_elems))
+                continue;
+            if (k < r) val = reinterpret_cast<const uint4*>(A + (int64_t)(pb * r + k) * d_in)[v];
+            reinterpret_cast<uint4*>(packA + ((int64_t)i * RP + j) * d_in)[v] = val;
         } else {
-            __nv_bfloat16 v[8];
+            const int64_t f = e - ua;
+            const int64_t c = f / vb;
+            const int col = (int)(f - c * vb) * 8;
+            const int pb = col / rblk, k0 = col - pb * rblk;  // 8 columns of one block (rblk % 16 == 0)
+            int cb = 0;
+            while (cb + 1 < blocks.n && c >= blocks.end[cb]) ++cb;
+            if (cb == pb && k0 < r) {
+                const __nv_bfloat16* src = B + c * r + k0;
+                if ((r & 7) == 0) {
+                    val = *reinterpret_cast<const uint4*>(src);
+                } else {
+                    __nv_bfloat16 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int k = ch * 8 + u;
-                v[u] = k < r ? src[k] : __float2bfloat16_rn(0.f);
+                    for (int u = 0; u < 8; ++u) v[u] = k0 + u < r ? src[u] : __float2bfloat16_rn(0.f);
+                    val = *reinterpret_cast<const uint4*>(v);
+                }
             }
-            val = *reinterpret_cast<const uint4*>(v);
-        }
-        *reinterpret_cast<uint4*>(dst + (int64_t)c * RP + ch * 8) = val;
-    }
-}
-
-// grid: (ceil(d_out/128), n); block 256.  Stages B_i[c0..c0+127][0..r) in shared memory (dynamic,
-// 128 x (r + 2) bf16), then writes rows k < rp16 of packBT, 128 columns each.
-__global__ void __launch_bounds__(256) pack_bt_kernel(const AdapterDev* __restrict__ ad, int RP, int64_t d_out,
-                                                      OutBlocks blocks, __nv_bfloat16* __restrict__ packBT) {
-    extern __shared__ __nv_bfloat16 tile[];
-    const int i = blockIdx.y;
-    const int64_t c0 = (int64_t)blockIdx.x * 128;
-    const int r = ad[i].rank;
-    const int ld = r + 2;
-    const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(ad[i].B);
-    const int cols = (int)(d_out - c0 < 128 ? d_out - c0 : 128);
-    if ((r & 7) == 0) {
-        // rows of B are 16-byte multiples: 16-byte loads, 8 ranks each
-        const int vr = r >> 3;
-        const uint4* src = reinterpret_cast<const uint4*>(B + c0 * r);
-        for (int e = threadIdx.x; e < cols * vr; e += blockDim.x) {
-            const int cc = e / vr, v = e - cc * vr;
-            const uint4 q = src[e];
-            const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&q);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) tile[cc * ld + v * 8 + u] = h[u];
-        }
-    } else {
-        for (int e = threadIdx.x; e < cols * r; e += blockDim.x) {
-            const int cc = e / r, k = e - cc * r;
-            tile[cc * ld + k] = B[(c0 + cc) * r + k];
-        }
-    }
-    __syncthreads();
-    // With output blocks the pack is block-diagonal: row pb rblk + k holds B's column k on block
-    // pb's output columns and zeros elsewhere, so block pb of G sums over block pb's columns only.
-    // A 128-column tile lies in one block (block ends are multiples of 256).
-    int cb = 0;
-    while (cb + 1 < blocks.n && c0 >= blocks.end[cb]) ++cb;
-    const int rblk = ad[i].rblk;
-    const int rows = ad[i].rp16;   // rows past the MMA extent are never read
-    for (int e = threadIdx.x; e < rows * 64; e += blockDim.x) {
-        const int j = e >> 6, cc = (e & 63) * 2;
-        const int pb = j / rblk, k = j - pb * rblk;
-        const bool live = pb == cb && k < r;
-        if (cc < cols) {
-            __nv_bfloat162 v;
-            v.x = live ? tile[cc * ld + k] : __float2bfloat16_rn(0.f);
-            v.y = live ? tile[(cc + 1) * ld + k] : __float2bfloat16_rn(0.f);
-            *reinterpret_cast<__nv_bfloat162*>(packBT + ((int64_t)i * RP + j) * d_out + c0 + cc) = v;
+            if (!dcheck(err_flag, col + 8 <= RP && ((int64_t)i * d_out + c) * RP + col + 8 <= packB_elems)) continue;
+            *reinterpret_cast<uint4*>(packB + ((int64_t)i * d_out + c) * RP + col) = val;
         }
     }
 }

@@ -18,12 +18,13 @@ constexpr int kPairStageBytes = kABytes + kABytes; // A: 128 x 64, B half: 128 x
 template <Op OP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+               const __grid_constant__ CUtensorMap tmC, const TcParams p) {
     static_assert(OP == Op::BaseFwd || OP == Op::BaseDx, "pair kernel covers the base GEMMs");
     constexpr bool kBmn = (OP == Op::BaseDx);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
     uint64_t* full_bar = bars;
     uint64_t* empty_bar = bars + kMaxStages;
     uint64_t* accf_bar = bars + 2 * kMaxStages;
@@ -57,6 +58,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (warp == 0 && lane == 0) {
         ptx::tma_prefetch_desc(&tmA);
         ptx::tma_prefetch_desc(&tmB);
+        ptx::tma_prefetch_desc(&tmC);
         if (p.fuse) {
             ptx::tma_prefetch_desc(&tmA2);
             ptx::tma_prefetch_desc(&tmB2);
@@ -132,7 +134,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 // Folded low-rank branch: A = this CTA's 128 rows of adapter j's zero-padded block,
                 // B = this CTA's 128 columns of j's factor, with the base B's major-ness (Y: the
-                // row-padded B, one K-major 128 x 64 box; dX: packed A, 16-row MN-major boxes).
+                // B pack, one K-major 128 x 64 box; dX: the A pack, 16-row MN-major boxes).
                 for (int q = lr.q0; q < lr.q1 && ok; ++q) {
                     const LoraSeg sg = mtile_seg(p, lr, q);
                     for (int kb = 0; kb * kBlockK < sg.rp16; ++kb) {
@@ -154,7 +156,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                     ptx::tma_load_2d_pair(sB + h * R * 128 + r16 * 128, &tmB2, fb, b_col + 64 * h,
                                                           sg.adapter * p.RP + kb * kBlockK + r16);
                         } else {
-                            ptx::tma_load_2d_pair(sB, &tmB2, fb, kb * kBlockK, sg.adapter * p.N_total + b_col);
+                            ptx::tma_load_3d_pair(sB, &tmB2, fb, kb * kBlockK, b_col, sg.adapter);
                         }
                         if (++stage == nst) { stage = 0; phase ^= 1u; }
                     }
@@ -230,7 +232,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
         const int q = warp & 3;
-        const int row = q * 32 + lane;
+        uint8_t* wbuf = smem + kEpiOffset + q * kEpiWarpBytes;
         int abuf = 0;
         uint32_t aphase = 0;
         for (int t = pair; t < p.num_tiles; t += npairs) {
@@ -240,33 +242,13 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
             const int out_row = mb * kPairTileM + (int)crank * kTileM;
-            const int n0 = nb * kTileN;
-            const bool row_ok = out_row + row < p.M_total;
-            const int cols_valid = min(kTileN, p.N_total - n0);
-            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(out_row + row) * p.out_ld + n0;
-            for (int c = 0; c < kTileN; c += 16) {
-                uint32_t r[16];
-                ptx::tmem_ld16(t_row + c, r);
-                ptx::tmem_ld_wait();
-                if (row_ok) {
-                    uint4 v0, v1;
-                    v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                    v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                    v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                    v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                    v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                    v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                    v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                    v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                    if (c + 8 <= cols_valid) *reinterpret_cast<uint4*>(out + c) = v0;
-                    if (c + 16 <= cols_valid) *reinterpret_cast<uint4*>(out + c + 8) = v1;
-                }
-            }
+            epilogue_store_tma(&tmC, t_row, wbuf, lane, out_row + q * 32, nb * kTileN, p.M_total, p.N_total);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cluster(&acce_bar[abuf], 0);
             if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
         }
+        if (lane == 0) ptx::bulk_wait<0>();   // every output store performed before the CTA exits
     }
 
     ptx::tc_fence_before();

@@ -34,9 +34,24 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(pl.EXPORTED)
 
 
+def test_debug_build_loads_and_exports_the_same_symbols():
+    """The PLORA_DEBUG build (device-side bounds checks) is a drop-in for the release library: it loads
+    without a GPU, exports every declared function and says which build it is."""
+    from packed_lora_fine_b200 import build as plbuild
+    rel = ctypes.CDLL(plbuild.LIB)
+    dbg = ctypes.CDLL(plbuild.DEBUG_LIB)
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+    rel.plora_debug_build.restype = dbg.plora_debug_build.restype = ctypes.c_int32
+    assert rel.plora_debug_build() == 0 and dbg.plora_debug_build() == 1
+    dbg.plora_status_string.restype = ctypes.c_char_p
+    assert dbg.plora_status_string(6) == b"PLORA_ERR_BOUNDS"
+
+
 def test_status_strings_and_version():
     for code, name in [(0, "PLORA_OK"), (1, "PLORA_ERR_INVALID_ARG"), (2, "PLORA_ERR_UNSUPPORTED"),
-                       (3, "PLORA_ERR_OOM"), (4, "PLORA_ERR_CUDA"), (5, "PLORA_ERR_TIMEOUT")]:
+                       (3, "PLORA_ERR_OOM"), (4, "PLORA_ERR_CUDA"), (5, "PLORA_ERR_TIMEOUT"),
+                       (6, "PLORA_ERR_BOUNDS")]:
         assert pl.status_string(code) == name
     assert pl.plora_version() >= 100
 
