@@ -47,7 +47,7 @@ WORKLOADS = {
     "llama_up_r16x1": "llama3-8b up_proj 4096->14336 bf16, one rank-16 adapter over the 32-adapter mix's tokens",
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-TC_KINDS = ("base_fwd", "base_dx")
+TC_KINDS = ("base_fwd", "base_dx", "base_dx+wgrad_a")
 
 
 def parse_args(argv=None):
@@ -63,6 +63,8 @@ def parse_args(argv=None):
                     help="run the expand products as separate passes (for comparison with the fused default)")
     ap.add_argument("--base-pair", action="store_true",
                     help="base GEMMs on SM pairs (cta_group::2) instead of single SMs")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="only the suite's one-layer line (seven calls, four calls with output blocks, one layer call)")
     ap.add_argument("--suite", action="store_true",
                     help="measure every workload (packed vs per-adapter sequential loop); one JSON line each")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="llama_up32",
@@ -110,8 +112,9 @@ def algorithmic_work(p):
         # one pack per step: reads each factor once, writes A's rows and B's columns up to rp16
         "pack_ab": (0.0, float(np.sum(2 * r * (di + do) + 2 * rp16 * (di + do)))),
     }
-    # K7's items share K5's launch
+    # K7's items share K5's launch; K8's share the dX GEMM's
     w["shrink_dy+wgrad_b"] = (w["shrink_dy"][0] + w["wgrad_b"][0], w["shrink_dy"][1] + w["wgrad_b"][1])
+    w["base_dx+wgrad_a"] = (w["base_dx"][0] + w["wgrad_a"][0], w["base_dx"][1] + w["wgrad_a"][1])
     return w
 
 
@@ -148,30 +151,72 @@ class EnergyMeter:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    """SM clock and clock-event (throttle) reasons during the timed region: NVML (the counters
+    nvidia-smi reads) polled every 5 ms from a background thread between start() and stop(), which
+    bracket the timed steps, so that a region of a few hundred milliseconds still gets dozens of
+    samples and none from the idle GPU around it.  Falls back to nvidia-smi -lms 100 without NVML."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = (("hw_slowdown", 0x8 | 0x80), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
+    def __init__(self, gpu_uuid: str):
+        self.gpu_uuid = gpu_uuid
+        self.h = None
         self.proc = None
-        self.path = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+        except Exception:
+            self.h = None
+
+    def _poll(self):
+        nv = self.nvml
+        while not self.done.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                why = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((float(mhz), int(why)))
+            except Exception:
+                pass
+            self.done.wait(0.005)
 
     def start(self):
+        import threading
+        self.samples = []
+        if self.h is not None:
+            self.done = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         fd, self.path = tempfile.mkstemp(prefix="plora_clocks_", suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", self.gpu_id, "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "--id=" + self.gpu_uuid, "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.h is not None:
+            self.done.set()
+            self.thread.join(timeout=5)
+            try:
+                mx = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+            except Exception:
+                mx = None
+            sm = [m for m, _ in self.samples]
+            reasons = sorted({name for _, why in self.samples for name, bit in self.REASONS if why & bit})
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                    "samples": len(sm), "source": "NVML every 5 ms during the timed region"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        time.sleep(0.25)
+        time.sleep(0.15)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -189,7 +234,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi -lms 100 around the timed region"}
 
 
 def reduce_max(x: float, dist) -> float:
@@ -314,6 +359,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.layer_only:
+        return layer_shared_inputs(args)
     if args.suite:
         return run_suite(args)
     if args.base_gemm_reference:
@@ -399,17 +446,16 @@ def main(argv=None):
     barrier()
     torch.cuda.synchronize()
     energy = EnergyMeter(gpu_uuid)
-    clocks.start()
-    time.sleep(0.3)
     energy.start()
+    clocks.start()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
+    clk = clocks.stop()
     joules, watts = energy.stop()
     barrier()
-    clk = clocks.stop()
     ms_local = ev0.elapsed_time(ev1) / args.steps
     prof = pl.plora_profile_read(eng.h)
     pl.plora_profile_enable(eng.h, False)
@@ -565,7 +611,8 @@ def main(argv=None):
                                X.numel() * 2 / 1e6, dY.numel() * 2 / 1e6),
                            "base_gemm": base_gemm},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-                "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+                "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
+                           "samples": clk["samples"], "source": clk.get("source")},
                 "energy": energy_line,
                 "l2_flushed": {"value": tokens_all / (ms_flushed / 1000.0), "unit": UNIT, "ms_per_step": ms_flushed,
                                "steps": k_fl, "how": "256 MB written before each step, outside its timed region; the inputs "
@@ -609,17 +656,16 @@ def run_base_gemm_reference(args):
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
     clocks, energy = ClockSampler(uuid), EnergyMeter(uuid)
-    clocks.start()
-    time.sleep(0.3)
     energy.start()
+    clocks.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         step()
     e1.record()
     torch.cuda.synchronize()
-    joules, watts = energy.stop()
     clk = clocks.stop()
+    joules, watts = energy.stop()
     ms = e0.elapsed_time(e1) / args.steps
     flops = 2 * 2.0 * T * di * do
     print(json.dumps({"impl": "cublas-base-gemms", "what": "torch.matmul Y = X W^T and dX = dY W only (no low-rank work)",
@@ -811,7 +857,9 @@ def run_suite(args):
 def layer_shared_inputs(args):
     """One LLaMA-3-8B layer whose LoRA targets read their inputs as in the model: q, k and v share
     one input, gate and up another, o and down have their own.  Timed as seven single-projection
-    calls and as four calls with q|k|v and gate|up stacked as output blocks (one base GEMM each).
+    calls, as four calls with q|k|v and gate|up stacked as output blocks (one base GEMM each), and as
+    one layer call over those four (plora_layer_*: one launch set, one persistent launch per product
+    kind).  The projections are independent here (no attention or activation between them).
     16 adapters x 8192 tokens, r ~ U{16,32,64}, alpha = 2r.  One JSON line."""
     import torch
     import packed_lora_fine_b200 as pl
@@ -891,14 +939,58 @@ def layer_shared_inputs(args):
     fused = [call(grp) for grp in groups]
     ms_fused = timed(fused, steps)
     same_q = bool(torch.equal(fused[0]["Y"][:, :shape["q"][1]], q_sep))
+    y_fused = [c["Y"].clone() for c in fused]
     for c in fused:
         c["eng"].close()
+    # The same four calls as ONE launch set (plora_layer_*): one persistent launch per product kind over
+    # all four projections, on the same buffers.
+    layer = pl.PackedLoRALayer([(c["X"].shape[1], c["Y"].shape[1]) + ((list(map(lambda nm: shape[nm][1], grp)),)
+                                if len(grp) > 1 else ()) for c, grp in zip(fused, groups)],
+                               max_adapters=n, max_rank=max(ranks), max_tokens=T)
+    offc = np.ascontiguousarray(off, dtype=np.int64)
+    keep = []
+
+    def projs(backward):
+        items = []
+        for c in fused:
+            keep.append(c["tb"] if backward else c["tf"])
+            items.append({"X": c["X"].data_ptr(), "W": c["W"].data_ptr(), "Y": c["Y"].data_ptr(),
+                          "dY": c["dY"].data_ptr(), "dX": c["dX"].data_ptr(), "tab": keep[-1],
+                          "saved": c["saved"].data_ptr()})
+        return pl.make_projs(items)
+    pf, pb = projs(False), projs(True)
+    lib = pl.load()
+
+    def layer_step(_):
+        assert lib.plora_layer_forward(layer.L, n, offc.ctypes.data, pf, st.cuda_stream) == pl.PLORA_OK
+        assert lib.plora_layer_backward(layer.L, n, offc.ctypes.data, pb, st.cuda_stream) == pl.PLORA_OK
+
+    def timed_layer(steps):
+        for _ in range(3):
+            layer_step(None)
+        torch.cuda.synchronize()
+        pl.plora_profile_read(layer.handle(0))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(steps):
+            layer_step(None)
+        e1.record(st)
+        torch.cuda.synchronize()
+        assert layer.check() == pl.PLORA_OK
+        return e0.elapsed_time(e1) / steps, sum(v[0] for v in pl.plora_profile_read(layer.handle(0)).values()) / steps
+    ms_layer, launches_layer = timed_layer(steps)
+    same_layer = all(bool(torch.equal(c["Y"], y)) for c, y in zip(fused, y_fused))
+    layer.close()
     print(json.dumps({"suite": "llama3-8b layer, shared inputs: q|k|v and gate|up as output blocks",
                       "tokens": T, "adapters": n, "projections": 7,
                       "separate_calls": 7, "separate_ms_per_step": ms_sep, "separate_tokens_per_s": T / (ms_sep / 1e3),
                       "fused_calls": len(groups), "fused_ms_per_step": ms_fused,
                       "fused_tokens_per_s": T / (ms_fused / 1e3), "fused_over_separate": ms_sep / ms_fused,
-                      "q_output_bit_identical": same_q}), flush=True)
+                      "q_output_bit_identical": same_q,
+                      "layer_call_ms_per_step": ms_layer, "layer_call_tokens_per_s": T / (ms_layer / 1e3),
+                      "layer_call_launches_per_step": launches_layer,
+                      "layer_call_over_fused_calls": ms_fused / ms_layer,
+                      "layer_call_outputs_bit_identical": same_layer}), flush=True)
     torch.cuda.empty_cache()
 
 

@@ -383,6 +383,70 @@ PLORA_API plora_status plora_grad_B_static(const plora_config* cfg, const void* 
                                            void* stream);
 
 /*
+ * Layer calls: several projections that share one segment map (the same adapters over the same
+ * packed token rows) and read and write independent tensors run as ONE launch set, one persistent
+ * launch per product kind over all of them, instead of one set per projection.  A LoRA fine-tuning
+ * job adapts several linear modules of each layer (query, key, value, output, and the MLP's gate, up
+ * and down projections; "LoRA加速集成方案", cloud.baidu.com, 七 › 2. 层的选择), and PLoRA packs each
+ * adapter's tokens through all of them.  Projections that read one input (q|k|v, gate|up) go in as
+ * one projection with output blocks.  Each projection is a segment of every launch, with its own
+ * parameters and tensor maps: a forward launches one schedule copy, one pack, one shrink and one
+ * base GEMM; a backward one schedule copy, one launch of G's shrink with dB, and one of the dX GEMMs
+ * with dA filling their last wave.  Results are bit for bit those of separate plora_forward /
+ * plora_backward calls on the projections' handles.
+ *
+ * The projections must not depend on each other within a call (the launch set runs them
+ * concurrently): in a model, a layer call groups projections whose inputs are all ready, for example
+ * the independent targets of a benchmark, or the weight and input gradients of projections whose
+ * output gradients are all known.
+ */
+#define PLORA_MAX_LAYER_PROJ 8
+typedef struct plora_layer_ctx* plora_layer;
+
+/* One projection of a layer call.  Shapes and layouts as for plora_forward / plora_backward with this
+ * projection's d_in, d_out: X [T][d_in], W [d_out][d_in], Y and dY [T][d_out], dX [T][d_in] (device);
+ * tab: host plora_adapter[n_adapters], this projection's factors (and gradients, for the backward);
+ * saved: device, 256-byte aligned, plora_layer_saved_bytes() bytes, filled by the forward.  The
+ * forward reads X, W, tab, saved and writes Y; the backward reads X, W, dY, tab, saved and writes dX
+ * (may be NULL to skip it) and every dA, dB. */
+typedef struct {
+    const void* X;
+    const void* W;
+    void* Y;
+    const void* dY;
+    void* dX;
+    const plora_adapter* tab;
+    void* saved;
+} plora_proj;
+
+/*
+ * Create a layer of n_proj in [1, PLORA_MAX_LAYER_PROJ] projections on the current device, one
+ * handle per configuration (as plora_create; the tensor-core path only: bf16 without PLORA_FLAG_SIMT,
+ * PLORA_FLAG_UNFUSED or PLORA_FLAG_BASE_PAIR, else PLORA_ERR_UNSUPPORTED).  *out is NULL on failure.
+ */
+PLORA_API plora_status plora_layer_create(plora_layer* out, int32_t n_proj, const plora_config* cfgs);
+/* Free the layer and its handles (synchronises the device first).  NULL is accepted. */
+PLORA_API plora_status plora_layer_destroy(plora_layer L);
+/* The handle of projection p (owned by the layer): for plora_check, plora_adamw_step, the profile
+ * calls (a layer call's launches are counted and timed on projection 0's handle) and the debug calls. */
+PLORA_API plora_status plora_layer_handle(plora_layer L, int32_t p, plora_handle* h);
+/* bytes (out): host size_t[n_proj], each projection's saved-buffer size for this call. */
+PLORA_API plora_status plora_layer_saved_bytes(plora_layer L, int32_t n_adapters, const int64_t* off,
+                                               const plora_proj* projs, size_t* bytes);
+/* Forward of every projection (projs: host plora_proj[n_proj]; off as for plora_forward, shared). */
+PLORA_API plora_status plora_layer_forward(plora_layer L, int32_t n_adapters, const int64_t* off,
+                                           const plora_proj* projs, void* stream);
+/* Backward of every projection, reading the saved buffers their layer forward filled. */
+PLORA_API plora_status plora_layer_backward(plora_layer L, int32_t n_adapters, const int64_t* off,
+                                            const plora_proj* projs, void* stream);
+/* Errors: every argument of every projection is checked before anything is enqueued (nothing is
+ * written on an error; plora_layer_last_error names the projection).  Device errors as for
+ * plora_check, through plora_layer_check (synchronises `stream`, reports the first projection's
+ * error, clears the flags). */
+PLORA_API plora_status plora_layer_check(plora_layer L, void* stream);
+PLORA_API const char* plora_layer_last_error(plora_layer L);
+
+/*
  * Multi-GPU sharding of one adapter set: assign each adapter to one of n_parts GPUs (one process
  * per GPU, each running its own handle over its share), balancing the parts' costs.  PLoRA runs
  * each packed job on a chosen number of GPUs (PLoRA summary, gist.science, arXiv 2508.02932,

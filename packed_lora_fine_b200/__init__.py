@@ -45,7 +45,9 @@ EXPORTED = ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward
             "plora_check", "plora_status_string", "plora_last_error", "plora_debug_unpack_saved",
             "plora_version", "plora_debug_schedule", "plora_profile_enable", "plora_profile_read",
             "plora_grad_B_static", "plora_adamw_step", "plora_debug_timeout_probe", "plora_device_info",
-            "plora_capture_reserve", "plora_capture_release", "plora_partition", "plora_debug_build")
+            "plora_capture_reserve", "plora_capture_release", "plora_partition", "plora_debug_build",
+            "plora_layer_create", "plora_layer_destroy", "plora_layer_handle", "plora_layer_saved_bytes",
+            "plora_layer_forward", "plora_layer_backward", "plora_layer_check", "plora_layer_last_error")
 
 
 class plora_config(ctypes.Structure):
@@ -133,6 +135,18 @@ def load(path: str = LIB_PATH):
     lib.plora_version.restype = ctypes.c_int32
     lib.plora_debug_build.argtypes = []
     lib.plora_debug_build.restype = ctypes.c_int32
+    lib.plora_layer_create.argtypes = [ctypes.POINTER(H), I32, P]
+    lib.plora_layer_destroy.argtypes = [H]
+    lib.plora_layer_handle.argtypes = [H, I32, ctypes.POINTER(H)]
+    lib.plora_layer_saved_bytes.argtypes = [H, I32, P, P, P]
+    lib.plora_layer_forward.argtypes = [H, I32, P, P, P]
+    lib.plora_layer_backward.argtypes = [H, I32, P, P, P]
+    lib.plora_layer_check.argtypes = [H, P]
+    lib.plora_layer_last_error.argtypes = [H]
+    lib.plora_layer_last_error.restype = ctypes.c_char_p
+    for fn in ("plora_layer_create", "plora_layer_destroy", "plora_layer_handle", "plora_layer_saved_bytes",
+               "plora_layer_forward", "plora_layer_backward", "plora_layer_check"):
+        getattr(lib, fn).restype = ctypes.c_int
     lib.plora_partition.argtypes = [I32, P, P, I64, I64, ctypes.c_double, ctypes.c_double, I32, P, P]
     lib.plora_partition.restype = ctypes.c_int
     for fn in ("plora_create", "plora_destroy", "plora_saved_bytes", "plora_forward", "plora_backward",
@@ -427,6 +441,118 @@ class PackedLoRA:
         plora_backward(self.h, X.data_ptr(), W.data_ptr(), dY.data_ptr(), dX.data_ptr() if want_dX else None,
                        n, off, tab, saved.data_ptr(), st)
         return dX, dA, dB
+
+
+# ---------------------------------------------------------------- layer calls
+class plora_proj(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("W", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("dY", ctypes.c_void_p),
+                ("dX", ctypes.c_void_p), ("tab", ctypes.c_void_p), ("saved", ctypes.c_void_p)]
+
+
+def make_projs(items) -> "ctypes.Array":
+    """plora_proj[n] from dicts with keys X, W, Y, dY, dX (device pointers or None), tab (a table from
+    make_table) and saved (device pointer or None)."""
+    arr = (plora_proj * len(items))()
+    keep = []
+    for k, it in enumerate(items):
+        tab = it.get("tab")
+        keep.append(tab)
+        arr[k] = plora_proj(it.get("X"), it.get("W"), it.get("Y"), it.get("dY"), it.get("dX"),
+                            ctypes.addressof(tab) if tab is not None else None, it.get("saved"))
+    arr._keep = keep
+    return arr
+
+
+class PackedLoRALayer:
+    """A layer call: several projections over one segment map (the same adapters over the same packed
+    token rows) run as one launch set, one persistent launch per product kind over all of them.
+
+    ``projections`` lists each projection as ``(d_in, d_out)`` or ``(d_in, d_out, out_blocks)``.
+    ``forward(io, off, scales)`` takes one dict per projection with its ``X``, ``W``, ``A``, ``B``
+    torch tensors and returns ``[(Y, saved)]``; ``backward(io, off, scales, saved)`` takes the same
+    dicts with ``dY`` added and returns ``[(dX, dA, dB)]``.  Results equal separate calls bit for bit.
+    """
+
+    def __init__(self, projections, max_adapters=64, max_rank=PLORA_MAX_RANK, max_tokens=1 << 16):
+        self.proj = [tuple(p) for p in projections]
+        cfgs = (plora_config * len(self.proj))()
+        for k, p in enumerate(self.proj):
+            cfgs[k] = make_config(p[0], p[1], PLORA_BF16, max_adapters, max_rank, max_tokens, 0,
+                                  p[2] if len(p) > 2 else None)
+        h = ctypes.c_void_p()
+        st = load().plora_layer_create(ctypes.byref(h), len(self.proj), cfgs)
+        if st != PLORA_OK:
+            raise PloraError(st, "plora_layer_create")
+        self.L = h.value
+
+    def handle(self, p: int) -> int:
+        h = ctypes.c_void_p()
+        st = load().plora_layer_handle(self.L, p, ctypes.byref(h))
+        if st != PLORA_OK:
+            raise PloraError(st, "plora_layer_handle")
+        return h.value
+
+    def close(self):
+        if self.L:
+            load().plora_layer_destroy(self.L)
+            self.L = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _err(self, st, what):
+        if st != PLORA_OK:
+            raise PloraError(st, f"{what}: {load().plora_layer_last_error(self.L).decode()}")
+
+    @staticmethod
+    def _table(scales, A, B, dA=None, dB=None):
+        return make_table([b.shape[1] for b in B], scales, [a.data_ptr() for a in A], [b.data_ptr() for b in B],
+                          None if dA is None else [x.data_ptr() for x in dA],
+                          None if dB is None else [x.data_ptr() for x in dB])
+
+    def forward(self, io, off, scales, stream=None):
+        import torch
+        off = np.ascontiguousarray(off, dtype=np.int64)
+        n = len(off) - 1
+        items, outs = [], []
+        for k, d in enumerate(io):
+            tab = self._table(scales, d["A"], d["B"])
+            Y = torch.empty((d["X"].shape[0], self.proj[k][1]), dtype=d["X"].dtype, device=d["X"].device)
+            items.append({"X": d["X"].data_ptr(), "W": d["W"].data_ptr(), "Y": Y.data_ptr(), "tab": tab})
+            outs.append(Y)
+        projs = make_projs(items)
+        sizes = (ctypes.c_size_t * len(io))()
+        self._err(load().plora_layer_saved_bytes(self.L, n, off.ctypes.data, projs, sizes), "plora_layer_saved_bytes")
+        saved = [torch.empty(max(int(b), 256), dtype=torch.uint8, device=d["X"].device) for b, d in zip(sizes, io)]
+        for k in range(len(io)):
+            projs[k].saved = saved[k].data_ptr()
+        st = (stream or torch.cuda.current_stream()).cuda_stream
+        self._err(load().plora_layer_forward(self.L, n, off.ctypes.data, projs, st), "plora_layer_forward")
+        return list(zip(outs, saved))
+
+    def backward(self, io, off, scales, saved, want_dX=True, stream=None):
+        import torch
+        off = np.ascontiguousarray(off, dtype=np.int64)
+        n = len(off) - 1
+        items, outs = [], []
+        for k, d in enumerate(io):
+            dA = [torch.empty(a.shape, dtype=torch.float32, device=a.device) for a in d["A"]]
+            dB = [torch.empty(b.shape, dtype=torch.float32, device=b.device) for b in d["B"]]
+            dX = torch.empty_like(d["X"]) if want_dX else None
+            tab = self._table(scales, d["A"], d["B"], dA, dB)
+            items.append({"X": d["X"].data_ptr(), "W": d["W"].data_ptr(), "dY": d["dY"].data_ptr(),
+                          "dX": dX.data_ptr() if want_dX else None, "tab": tab, "saved": saved[k].data_ptr()})
+            outs.append((dX, dA, dB))
+        projs = make_projs(items)
+        st = (stream or torch.cuda.current_stream()).cuda_stream
+        self._err(load().plora_layer_backward(self.L, n, off.ctypes.data, projs, st), "plora_layer_backward")
+        return outs
+
+    def check(self, stream=None) -> int:
+        return int(load().plora_layer_check(self.L, stream))
 
 
 # ---------------------------------------------------------------- autograd

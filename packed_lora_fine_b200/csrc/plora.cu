@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <memory>
 #include <mutex>
 #include <new>
 #include <string>
@@ -36,6 +37,17 @@ struct Region {
 };
 
 }  // namespace
+
+// The segments of one tc_kernel launch (see GroupParams): segment parameters and their five tensor
+// maps (operands A, B; a base GEMM's folded branch A2, B2 and output C; unused slots hold copies of A).
+// The launch copies them when it is enqueued, so one host copy serves every launch.
+struct Segments {
+    GroupParams g{};
+    GroupMaps m{};
+    int n_op2 = 0;
+    TcParams p2[kMaxSeg];
+    CUtensorMap m2[kMaxSeg][5];
+};
 
 struct plora_ctx {
     plora_config cfg{};
@@ -80,6 +92,9 @@ struct plora_ctx {
     struct Rec { int kind; cudaEvent_t a, b; };
     std::vector<Rec> pending;
     std::vector<cudaEvent_t> pool;
+
+    // host scratch for building one launch's segment table (kernel parameters, ~14 KB)
+    std::unique_ptr<Segments> segs;
 
     template <typename T> T* at(const Region& r) const { return reinterpret_cast<T*>(ws + r.off); }
 };
@@ -162,10 +177,10 @@ __global__ void timeout_probe_kernel(int* err_flag, uint64_t limit_ns) {
 
 // Kernel kinds for launch accounting / profiling.
 enum Kind { kPack = 0, kBaseFwd, kShrinkX, kExpandY, kBaseDx, kShrinkDy, kExpandDx, kWgradB, kWgradA,
-            kSimt, kAdamw, kShrinkDyWgradB, kStage, kKinds };
+            kSimt, kAdamw, kShrinkDyWgradB, kStage, kBaseDxWgradA, kKinds };
 const char* const kKindNames[kKinds] = {"pack_ab", "base_fwd", "shrink_x", "expand_y", "base_dx",
                                         "shrink_dy", "expand_dx", "wgrad_b", "wgrad_a", "simt_gemm", "adamw",
-                                        "shrink_dy+wgrad_b", "stage_copy"};
+                                        "shrink_dy+wgrad_b", "stage_copy", "base_dx+wgrad_a"};
 
 cudaEvent_t take_event(plora_ctx* h) {
     if (!h->pool.empty()) {
@@ -400,27 +415,54 @@ struct DevPlan {
     int slot = 0;
 };
 
-// Copies a call's schedule from the slot's mapped pinned staging buffer into device memory.  A kernel
-// rather than cudaMemcpyAsync: its reads of host memory do not wait in the copy-engine queue behind
-// bulk host-to-device copies that the caller may have in flight (the next step's inputs, say).
-__global__ void stage_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n16, int64_t cap16,
-                                  int* err_flag) {
-    if (!dcheck(err_flag, n16 <= cap16)) return;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
+// Copies calls' schedules from their slots' mapped pinned staging buffers into device memory, one
+// copy per blockIdx.y.  A kernel rather than cudaMemcpyAsync: its reads of host memory do not wait in
+// the copy-engine queue behind bulk host-to-device copies that the caller may have in flight (the next
+// step's inputs, say).
+struct StageCopies {
+    int32_t n;
+    int32_t pad_;
+    const uint4* src[kMaxSeg];
+    uint4* dst[kMaxSeg];
+    int64_t n16[kMaxSeg];
+    int64_t cap16[kMaxSeg];        // 16-byte words of each destination region
+    int* err_flag;
+};
+
+__global__ void stage_copy_kernel(const __grid_constant__ StageCopies cs) {
+    const int k = blockIdx.y;
+    if (k >= cs.n || !dcheck(cs.err_flag, cs.n16[k] <= cs.cap16[k])) return;
+    const uint4* __restrict__ src = cs.src[k];
+    uint4* __restrict__ dst = cs.dst[k];
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < cs.n16[k]; i += (int64_t)gridDim.x * blockDim.x)
         dst[i] = src[i];
 }
 
-// `bytes` of staging (device view `src`) into device memory at d (rounded up to 16 bytes; the
-// staging and the device region are both whole multiples of 256 bytes).
-cudaError_t stage_copy(plora_ctx* h, const uint8_t* src, uint8_t* d, size_t bytes, cudaStream_t st) {
-    const int64_t n16 = (int64_t)((bytes + 15) / 16);
-    if (n16 == 0) return cudaSuccess;
-    const int blocks = (int)std::min<int64_t>(ceil_div(n16, 256), 64);
-    tracked(h, kStage, st, [&] {
-        stage_copy_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(d),
-                                                  n16, (int64_t)(h->blob_bytes / 16), h->at<int>(h->r_err));
-    });
+// One launch copying every schedule queued in `cs` (device views of the staging in src).
+cudaError_t stage_copy_run(plora_ctx* h, const StageCopies& cs, cudaStream_t st) {
+    if (cs.n == 0) return cudaSuccess;
+    int64_t most = 0;
+    for (int k = 0; k < cs.n; ++k) most = std::max(most, cs.n16[k]);
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(most, 256), 64));
+    tracked(h, kStage, st, [&] { stage_copy_kernel<<<dim3((unsigned)blocks, (unsigned)cs.n), 256, 0, st>>>(cs); });
     return cudaGetLastError();
+}
+
+// Queues `bytes` of staging (device view `src`) for the device region at d (rounded up to 16 bytes;
+// the staging and the device region are both whole multiples of 256 bytes).
+void stage_copy_add(plora_ctx* h, StageCopies& cs, const uint8_t* src, uint8_t* d, size_t bytes) {
+    if (cs.n == 0) cs.err_flag = h->at<int>(h->r_err);
+    cs.cap16[cs.n] = (int64_t)(h->blob_bytes / 16);
+    cs.src[cs.n] = reinterpret_cast<const uint4*>(src);
+    cs.dst[cs.n] = reinterpret_cast<uint4*>(d);
+    cs.n16[cs.n] = (int64_t)((bytes + 15) / 16);
+    ++cs.n;
+}
+
+cudaError_t stage_copy(plora_ctx* h, const uint8_t* src, uint8_t* d, size_t bytes, cudaStream_t st) {
+    StageCopies cs{};
+    stage_copy_add(h, cs, src, d, bytes);
+    return stage_copy_run(h, cs, st);
 }
 
 bool stream_capturing(cudaStream_t st) {
@@ -462,8 +504,10 @@ plora_status take_slot(plora_ctx* h, cudaStream_t st, Slot& sl) {
     return PLORA_OK;
 }
 
+// With `defer`, the copy is queued there instead of launched (a layer call stages every projection's
+// schedule with one launch).
 plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& ops, cudaStream_t st,
-                    DevPlan& D) {
+                    DevPlan& D, StageCopies* defer = nullptr) {
     Slot sl;
     plora_status ps = take_slot(h, st, sl);
     if (ps != PLORA_OK) return ps;
@@ -482,8 +526,12 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     const size_t o_mtl = put(P.mt_seg.data(), P.mt_seg.size() * sizeof(LoraSeg));
     if (o > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "schedule exceeds the handle's staging size");
     uint8_t* d = sl.dev;
-    cudaError_t e = stage_copy(h, sl.host_dev, d, o, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "copying the schedule to the device");
+    if (defer) {
+        stage_copy_add(h, *defer, sl.host_dev, d, o);
+    } else {
+        cudaError_t e = stage_copy(h, sl.host_dev, d, o, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "copying the schedule to the device");
+    }
     D.ad = reinterpret_cast<AdapterDev*>(d + o_ad);
     D.tok = reinterpret_cast<TokTile*>(d + o_tok);
     D.red = reinterpret_cast<RedEntry*>(d + o_red);
@@ -553,26 +601,68 @@ void launch_simt(plora_ctx* h, const SimtOp* d_ops, int n_ops, int tiles, cudaSt
 // ---------------------------------------------------------------------------
 // Tensor-core launches
 // ---------------------------------------------------------------------------
+struct SegMaps {
+    const CUtensorMap *a, *b, *a2, *b2, *c;
+};
+
+// Appends a segment of the first op (op2 = false) or of the second (op2 = true).
+void seg_add(Segments& S, const TcParams& p, const SegMaps& mp, bool op2) {
+    const CUtensorMap* src[5] = {mp.a, mp.b, mp.a2 ? mp.a2 : mp.a, mp.b2 ? mp.b2 : mp.a, mp.c ? mp.c : mp.a};
+    if (op2) {
+        for (int k = 0; k < 5; ++k) S.m2[S.n_op2][k] = *src[k];
+        S.p2[S.n_op2++] = p;
+    } else {
+        for (int k = 0; k < 5; ++k) S.m.m[S.g.n_op1][k] = *src[k];
+        S.g.p[S.g.n_op1++] = p;
+    }
+}
+
+// Orders the segments (first op's, then second op's), sets the item ranges; returns the item count.
+int seg_finish(Segments& S) {
+    S.g.n_seg = S.g.n_op1 + S.n_op2;
+    for (int j = 0; j < S.n_op2; ++j) {
+        S.g.p[S.g.n_op1 + j] = S.p2[j];
+        for (int k = 0; k < 5; ++k) S.m.m[S.g.n_op1 + j][k] = S.m2[j][k];
+    }
+    S.g.begin[0] = 0;
+    for (int j = 0; j < S.g.n_seg; ++j) S.g.begin[j + 1] = S.g.begin[j] + std::max(0, S.g.p[j].num_tiles);
+    return S.g.begin[S.g.n_seg];
+}
+
+template <Op OP, Op OP2 = OP>
+cudaError_t launch_segments(Segments& S, int num_sms, cudaStream_t st) {
+    const int total = seg_finish(S);
+    if (total <= 0) return cudaSuccess;
+    tc_kernel<OP, OP2><<<std::min(total, num_sms), kTcThreads, kTcSmemBytes, st>>>(S.m, S.g);
+    return cudaGetLastError();
+}
+
 // c: the output tensor map of a base GEMM (TMA-stored epilogue); other ops ignore it.
 template <Op OP>
 void launch_tc(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2, const CUtensorMap& b2,
                const CUtensorMap& c, const TcParams& p, cudaStream_t st) {
     if (p.num_tiles <= 0) return;
-    const int grid = std::min(p.num_tiles, h->num_sms);
     constexpr int kind = OP == Op::BaseFwd ? kBaseFwd : OP == Op::BaseDx ? kBaseDx : OP == Op::ShrinkX ? kShrinkX
                        : OP == Op::ShrinkDy ? kShrinkDy : OP == Op::ExpandY ? kExpandY : OP == Op::ExpandDx ? kExpandDx
                        : OP == Op::WgradB ? kWgradB : kWgradA;
-    tracked(h, kind, st, [&] { tc_kernel<OP><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, c, p, p); });
+    Segments& S = *h->segs;
+    S = Segments{};
+    seg_add(S, p, SegMaps{&a, &b, &a2, &b2, &c}, false);
+    tracked(h, kind, st, [&] { launch_segments<OP>(S, h->num_sms, st); });
 }
 
-// Two independent ops in one persistent launch: OP's items (operands a, b) then OP2's (a2, b2).
+// Two independent ops in one persistent launch: OP's items (operands a, b; a base GEMM's fold a2, b2
+// and output c) then OP2's (a3, b3).
 template <Op OP, Op OP2>
 void launch_tc2(plora_ctx* h, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                const CUtensorMap& b2, const TcParams& p, const TcParams& p2, int kind, cudaStream_t st) {
-    const int total = p.num_tiles + p2.num_tiles;
-    if (total <= 0) return;
-    const int grid = std::min(total, h->num_sms);
-    tracked(h, kind, st, [&] { tc_kernel<OP, OP2><<<grid, kTcThreads, kTcSmemBytes, st>>>(a, b, a2, b2, a, p, p2); });
+                const CUtensorMap& b2, const CUtensorMap& c, const CUtensorMap& a3, const CUtensorMap& b3,
+                const TcParams& p, const TcParams& p2, int kind, cudaStream_t st) {
+    if (p.num_tiles + p2.num_tiles <= 0) return;
+    Segments& S = *h->segs;
+    S = Segments{};
+    seg_add(S, p, SegMaps{&a, &b, &a2, &b2, &c}, false);
+    seg_add(S, p2, SegMaps{&a3, &b3, nullptr, nullptr, nullptr}, true);
+    tracked(h, kind, st, [&] { launch_segments<OP, OP2>(S, h->num_sms, st); });
 }
 
 // Base GEMMs on SM pairs: a cluster of two CTAs per 256x256 tile, persistent over the pairs that
@@ -667,25 +757,43 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
 }
 
 // Packs every adapter's A and B into the saved buffer in the layouts the tensor-core operands want
-// (pack_ab_kernel), once per forward; the backward reads the same packs.
-void pack_factors(plora_ctx* h, const HostPlan& P, const DevPlan& D, void* saved, cudaStream_t st) {
-    if (P.n == 0) return;
+// (pack_ab_kernel), once per forward; the backward reads the same packs.  pack_job describes one
+// call's pack; pack_run launches one grid over every queued job.
+PackJob pack_job(plora_ctx* h, const HostPlan& P, const DevPlan& D, void* saved) {
     const SavedLayout L = saved_layout(h, P);
     uint8_t* sv = static_cast<uint8_t*>(saved);
+    PackJob J{};
+    J.ad = D.ad;
+    J.packA = reinterpret_cast<__nv_bfloat16*>(sv + L.o_packA);
+    J.packB = reinterpret_cast<__nv_bfloat16*>(sv + L.o_packB);
+    J.d_in = h->cfg.d_in;
+    J.d_out = h->cfg.d_out;
+    J.packA_elems = (int64_t)((L.o_packB - L.o_packA) / 2);
+    J.packB_elems = (int64_t)((L.bytes - L.o_packB) / 2);
+    J.n = P.n;
+    J.RP = P.RP;
+    J.blocks.n = h->nblk;
+    for (int b = 0; b < kMaxOutBlocks; ++b) J.blocks.end[b] = h->blk_end[b];
+    J.err_flag = h->at<int>(h->r_err);
+    return J;
+}
+
+// Chunks of the largest adapter of a job (sizes the grid's x extent).
+int64_t pack_chunks(const plora_ctx* h, const HostPlan& P) {
     int64_t most = 1;
     for (const AdapterDev& a : P.ad)
         most = std::max<int64_t>(most, (int64_t)a.rp16 * (h->cfg.d_in / 8) + h->cfg.d_out * (a.rp16 / 8));
-    const int gx = (int)std::min<int64_t>(ceil_div(most, 256), 1024);
-    OutBlocks blocks{};
-    blocks.n = h->nblk;
-    for (int b = 0; b < kMaxOutBlocks; ++b) blocks.end[b] = h->blk_end[b];
+    return most;
+}
+
+void pack_run(plora_ctx* h, const PackJobs& jobs, int64_t most_chunks, int most_adapters, cudaStream_t st) {
+    if (jobs.n == 0 || most_adapters == 0) return;
+    const int gx = (int)std::min<int64_t>(ceil_div(most_chunks, 256), 1024);
     tracked(h, kPack, st, [&] {
-        pack_ab_kernel<<<dim3((unsigned)gx, (unsigned)P.n), 256, 0, st>>>(
-            D.ad, P.RP, h->cfg.d_in, h->cfg.d_out, blocks, reinterpret_cast<__nv_bfloat16*>(sv + L.o_packA),
-            reinterpret_cast<__nv_bfloat16*>(sv + L.o_packB), (int64_t)((L.o_packB - L.o_packA) / 2),
-            (int64_t)((L.bytes - L.o_packB) / 2), h->at<int>(h->r_err));
+        pack_ab_kernel<<<dim3((unsigned)gx, (unsigned)most_adapters, (unsigned)jobs.n), 256, 0, st>>>(jobs);
     });
 }
+
 
 // 3-D bf16 tensor map of the B pack [n][d_out][RP] (rank column innermost), 128-byte swizzle, a box of
 // 64 columns x box_rows rows of one adapter; rows past d_out read as zero.
@@ -698,6 +806,346 @@ bool make_packb_map(CUtensorMap* m, const void* base, uint64_t RP, uint64_t d_ou
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// The argument checks of a forward (everything before the first enqueue); builds the call's plan.
+plora_status fwd_args(plora_ctx* h, const void* X, const void* W, const void* Y, int32_t n, const int64_t* off,
+                      const plora_adapter* tab, const void* saved, HostPlan& P) {
+    plora_status s = check_table(h, n, off, tab, false);
+    if (s != PLORA_OK) return s;
+    const bool any_tokens = off[n] > 0;   // with no tokens, X, Y and saved are never touched
+    if (!W || (any_tokens && (!X || !Y || !saved)))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, Y or saved is NULL");
+    if (!aligned16(X) || !aligned16(W) || !aligned16(Y))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W or Y not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0)
+        return fail(h, PLORA_ERR_INVALID_ARG, "saved not 256-byte aligned");
+    cudaError_t ce = cudaSetDevice(h->device);
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
+    build_plan(h, n, off, tab, P);
+    if (P.T == 0) return PLORA_OK;
+    TensorArgs ta;
+    ta.X = X; ta.W = W; ta.Y = Y; ta.saved = saved;
+    return check_extents(h, P, tab, ta);
+}
+
+// The argument checks of a backward; builds the call's plan.
+plora_status bwd_args(plora_ctx* h, const void* X, const void* W, const void* dY, const void* dX, int32_t n,
+                      const int64_t* off, const plora_adapter* tab, const void* saved, HostPlan& P) {
+    plora_status s = check_table(h, n, off, tab, true);
+    if (s != PLORA_OK) return s;
+    const bool any_tokens = off[n] > 0;   // with no tokens, only dA and dB are written (zeros)
+    if (!W || (any_tokens && (!X || !dY || !saved)))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, dY or saved is NULL");
+    if (!aligned16(X) || !aligned16(W) || !aligned16(dY) || (dX && !aligned16(dX)))
+        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, dY or dX not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0)
+        return fail(h, PLORA_ERR_INVALID_ARG, "saved not 256-byte aligned");
+    cudaError_t ce = cudaSetDevice(h->device);
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
+    build_plan(h, n, off, tab, P);
+    TensorArgs ta;
+    if (P.T > 0) { ta.X = X; ta.W = W; ta.dY = dY; ta.dX = dX; ta.saved = saved; }
+    ta.adapters_AB = P.T > 0;
+    ta.adapters_dA = ta.adapters_dB = true;
+    return check_extents(h, P, tab, ta);
+}
+
+// Adapters without tokens get zero weight gradients (enqueued once every check has passed).
+plora_status zero_empty_grads(plora_ctx* h, const HostPlan& P, const plora_adapter* tab, cudaStream_t st) {
+    for (int32_t i : P.empty) {
+        cudaError_t ce = cudaMemsetAsync(tab[i].dA, 0, (size_t)tab[i].rank * h->nblk * h->cfg.d_in * sizeof(float), st);
+        if (ce == cudaSuccess) ce = cudaMemsetAsync(tab[i].dB, 0, (size_t)tab[i].rank * h->cfg.d_out * sizeof(float), st);
+        if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaMemsetAsync(dA/dB of an empty adapter)");
+    }
+    return PLORA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core calls, prepared one by one and launched together: a single call, or the projections of
+// a layer call, whose products of one kind run as one persistent launch over all of them (each
+// projection a segment of the launch, with its own parameters and tensor maps).
+// ---------------------------------------------------------------------------
+struct FwdCall {
+    plora_ctx* h = nullptr;
+    const void* X = nullptr;
+    const void* W = nullptr;
+    void* Y = nullptr;
+    void* saved = nullptr;
+    HostPlan P;
+    DevPlan D;
+    CUtensorMap mX, mW, mW128, mPA16, mHk, mPBk, mPBk128, mY;
+    TcParams q{}, p{};
+};
+
+// After the argument checks: stages the call's schedule (queued into cs), encodes its tensor maps and
+// fills the parameters of its shrink (q) and base GEMM (p).
+plora_status fwd_prepare(FwdCall& c, cudaStream_t st, StageCopies& cs) {
+    plora_ctx* h = c.h;
+    const HostPlan& P = c.P;
+    plora_status s = upload(h, P, {}, st, c.D, &cs);
+    if (s != PLORA_OK) return s;
+    const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
+    // mPA16: the A pack in 16-row boxes (the shrink's K-major B); mPBk / mPBk128: the B pack, K-major,
+    // 256 rows for the 1-SM tile and the expand, 128 per CTA of an SM pair.
+    const SavedLayout L = saved_layout(h, P);
+    const uint8_t* sv = static_cast<const uint8_t*>(c.saved);
+    bool ok = make_map(&c.mX, c.X, d_in, P.T, d_in, 64, kTileM) &&
+              make_map(&c.mY, c.Y, d_out, P.T, d_out, 64, 32) &&
+              make_map(&c.mW, c.W, d_in, d_out, d_in, 64, kTileN) &&
+              make_map(&c.mW128, c.W, d_in, d_out, d_in, 64, kTileM) &&
+              make_map(&c.mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
+              make_map(&c.mHk, c.saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_packb_map(&c.mPBk, sv + L.o_packB, P.RP, d_out, P.n, kTileN) &&
+              make_packb_map(&c.mPBk128, sv + L.o_packB, P.RP, d_out, P.n, kTileM);
+    if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    // K2: H'_i = s_i X_i A_i per 128-token tile (into the zero-padded blocks of `saved`).
+    TcParams& q = c.q;
+    q = base_params(h, P, c.D);
+    q.K_total = (int32_t)d_in;
+    q.num_tiles = (int32_t)P.tok.size();
+    q.out = c.saved; q.out_ld = P.RP;
+    q.out_elems = P.h_rows * P.RP;
+    q.n_items = (int32_t)P.tok.size();
+    // K1 (+K3): Y = X W over all packed tokens; fused, each tile also accumulates H'_j B_j of every
+    // adapter j overlapping it, so Y is written once.
+    TcParams& p = c.p;
+    p = base_params(h, P, c.D);
+    p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_out; p.K_total = (int32_t)d_in;
+    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_out, kTileN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.b_box_rows = kTileN;
+    p.out = c.Y; p.out_ld = d_out;
+    p.fuse = (h->cfg.flags & PLORA_FLAG_UNFUSED) ? 0 : 1;
+    return PLORA_OK;
+}
+
+// The calls in decreasing order of their K (the cost of one work item of a given kind): items are dealt
+// round-robin in segment order, so the longest come first and the last wave holds the shortest.  The
+// order changes no result: every item is computed on its own.
+template <typename C, typename F>
+std::vector<int> by_k(const C* calls, int nc, F k_of) {
+    std::vector<int> o(nc);
+    for (int k = 0; k < nc; ++k) o[k] = k;
+    std::stable_sort(o.begin(), o.end(), [&](int a, int b) { return k_of(calls[a]) > k_of(calls[b]); });
+    return o;
+}
+
+// The forward of every prepared call: one schedule copy, one pack, one shrink launch, one base-GEMM
+// launch (the SM-pair and unfused variants, single calls only, keep their own launches).
+plora_status fwd_launch(FwdCall* calls, int nc, cudaStream_t st, StageCopies& cs) {
+    plora_ctx* h0 = calls[0].h;
+    cudaError_t e = stage_copy_run(h0, cs, st);
+    if (e != cudaSuccess) return cuda_fail(h0, e, "copying the schedule to the device");
+    PackJobs jobs{};
+    int64_t most = 1;
+    int most_n = 0, RPmax = kRankAlign;
+    for (int k = 0; k < nc; ++k) {
+        FwdCall& c = calls[k];
+        jobs.j[jobs.n++] = pack_job(c.h, c.P, c.D, c.saved);
+        most = std::max(most, pack_chunks(c.h, c.P));
+        most_n = std::max(most_n, c.P.n);
+        RPmax = std::max(RPmax, c.P.RP);
+    }
+    pack_run(h0, jobs, most, most_n, st);
+    Segments& S = *h0->segs;
+    S = Segments{};
+    const std::vector<int> order = by_k(calls, nc, [](const FwdCall& c) { return c.p.K_total; });
+    for (int k : order) {   // one narrow ring that holds every call's widest B tile
+        FwdCall& c = calls[k];
+        narrow_ring(c.q, RPmax);
+        seg_add(S, c.q, SegMaps{&c.mX, &c.mPA16, nullptr, nullptr, nullptr}, false);
+    }
+    tracked(h0, kShrinkX, st, [&] { launch_segments<Op::ShrinkX>(S, h0->num_sms, st); });
+    const uint32_t flags = h0->cfg.flags;
+    if (nc == 1 && (flags & (PLORA_FLAG_BASE_PAIR | PLORA_FLAG_UNFUSED))) {
+        FwdCall& c = calls[0];
+        plora_ctx* h = c.h;
+        const bool fused = c.p.fuse != 0;
+        if (flags & PLORA_FLAG_BASE_PAIR) {
+            pair_params(c.p, c.P.T, h->cfg.d_out);
+            launch_pair<Op::BaseFwd>(h, c.mX, c.mW128, c.mHk, fused ? c.mPBk128 : c.mW128, c.mY, c.p, st);
+        } else {
+            launch_tc<Op::BaseFwd>(h, c.mX, c.mW, c.mHk, c.mW, c.mY, c.p, st);
+        }
+        if (!fused) {
+            // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
+            TcParams r = base_params(h, c.P, c.D);
+            r.N_total = (int32_t)h->cfg.d_out;
+            r.tiles_n = (int32_t)ceil_div(h->cfg.d_out, kTileN);
+            r.num_tiles = (int32_t)c.P.tok.size() * r.tiles_n;
+            r.out = c.Y; r.out_ld = h->cfg.d_out;
+            r.out_elems = c.P.T * h->cfg.d_out;
+            r.n_items = (int32_t)c.P.tok.size();
+            launch_tc<Op::ExpandY>(h, c.mHk, c.mPBk, c.mHk, c.mPBk, c.mHk, r, st);
+        }
+    } else {
+        S = Segments{};
+        for (int k : order) {
+            FwdCall& c = calls[k];
+            seg_add(S, c.p, SegMaps{&c.mX, &c.mW, &c.mHk, &c.mPBk, &c.mY}, false);
+        }
+        tracked(h0, kBaseFwd, st, [&] { launch_segments<Op::BaseFwd>(S, h0->num_sms, st); });
+    }
+    for (int k = 0; k < nc; ++k) {
+        const plora_status s = finish(calls[k].h, calls[k].D, st);
+        if (s != PLORA_OK) return s;
+    }
+    return PLORA_OK;
+}
+
+struct BwdCall {
+    plora_ctx* h = nullptr;
+    const void* X = nullptr;
+    const void* W = nullptr;
+    const void* dY = nullptr;
+    void* dX = nullptr;
+    const void* saved = nullptr;
+    HostPlan P;
+    DevPlan D;
+    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_mn, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn, mdX;
+    TcParams q{}, wb{}, p{}, wa{};
+};
+
+// After the argument checks (and the zero gradients of empty adapters): stages the call's schedule
+// (queued into cs), encodes its tensor maps and fills the parameters of the shrink of G (q), dB (wb),
+// the dX GEMM (p) and dA (wa).
+plora_status bwd_prepare(BwdCall& c, cudaStream_t st, StageCopies& cs) {
+    plora_ctx* h = c.h;
+    const HostPlan& P = c.P;
+    plora_status s = upload(h, P, {}, st, c.D, &cs);
+    if (s != PLORA_OK) return s;
+    const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
+    void* G = h->at<void>(h->r_G);
+    // The factors were packed into `saved` by the forward; the backward packs nothing.
+    const SavedLayout L = saved_layout(h, P);
+    const uint8_t* sv = static_cast<const uint8_t*>(c.saved);
+    // the output map of the dX GEMM (dX may be NULL: the GEMM is skipped then)
+    bool ok = (!c.dX || make_map(&c.mdX, c.dX, d_in, P.T, d_in, 64, 32)) &&
+              make_map(&c.mdY_k, c.dY, d_out, P.T, d_out, 64, kTileM) &&
+              make_map(&c.mdY_mn, c.dY, d_out, P.T, d_out, 64, 64) &&
+              make_map(&c.mW_mn, c.W, d_in, d_out, d_in, 64, 64) &&
+              make_packb_map(&c.mPB_mn, sv + L.o_packB, P.RP, d_out, P.n, 64) &&
+              make_map(&c.mG_k, G, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_map(&c.mG_mn, G, P.RP, P.h_rows, P.RP, 64, 64) &&
+              make_map(&c.mPA_mn, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
+              make_map(&c.mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
+              make_map(&c.mH_mn, c.saved, P.RP, P.h_rows, P.RP, 64, 64) &&
+              make_map(&c.mX_mn, c.X, d_in, P.T, d_in, 64, 64);
+    if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    if (!c.dX) c.mdX = c.mdY_k;   // an unused slot still holds a valid map
+    // K5: G_i = s_i dY_i B_i^T per 128-token tile (into the zero-padded workspace blocks).
+    TcParams& q = c.q;
+    q = base_params(h, P, c.D);
+    q.K_total = (int32_t)d_out;
+    q.num_tiles = (int32_t)P.tok.size();
+    q.out = G; q.out_ld = P.RP;
+    q.out_elems = (int64_t)(h->r_G.bytes / h->esize);
+    q.n_items = (int32_t)P.tok.size();
+    // K7: dB_i = H'_i^T dY_i (a sum over each adapter's tokens) needs neither G nor dX, so its items
+    // share K5's launch and fill the last wave of K5's equal-cost token tiles.
+    TcParams& wb = c.wb;
+    wb = base_params(h, P, c.D);
+    wb.M_total = (int32_t)d_out;
+    wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
+    wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
+    wb.n_items = (int32_t)P.red.size();
+    // K4 (+K6): dX = dY W^T; fused, each tile also accumulates G_j A_j^T of every adapter j
+    // overlapping it, so dX is written once.
+    TcParams& p = c.p;
+    p = base_params(h, P, c.D);
+    p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
+    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
+    p.num_tiles = c.dX ? p.tiles_m * p.tiles_n : 0;
+    p.out = c.dX; p.out_ld = d_in;
+    p.fuse = (h->cfg.flags & PLORA_FLAG_UNFUSED) ? 0 : 1;
+    // K8: dA_i = X_i^T G_i (a sum over each adapter's tokens).
+    TcParams& wa = c.wa;
+    wa = base_params(h, P, c.D);
+    wa.M_total = (int32_t)d_in;
+    wa.red_dtiles = (int32_t)ceil_div(d_in, kTileM);
+    wa.num_tiles = (int32_t)P.red.size() * wa.red_dtiles;
+    wa.n_items = (int32_t)P.red.size();
+    return PLORA_OK;
+}
+
+// The backward of every prepared call: one schedule copy, one launch of the shrink of G with dB's
+// items, one launch of the dX GEMM with dA's items filling its last wave (the SM-pair variant, single
+// calls only, keeps dA in a launch of its own; the unfused one adds its expand pass).
+plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs) {
+    plora_ctx* h0 = calls[0].h;
+    cudaError_t e = stage_copy_run(h0, cs, st);
+    if (e != cudaSuccess) return cuda_fail(h0, e, "copying the schedule to the device");
+    int RPmax = kRankAlign;
+    for (int k = 0; k < nc; ++k) RPmax = std::max(RPmax, calls[k].P.RP);
+    Segments& S = *h0->segs;
+    S = Segments{};
+    // G's shrink reduces over d_out, the dX GEMM too: the calls with the widest d_out first
+    const std::vector<int> order = by_k(calls, nc, [](const BwdCall& c) { return c.p.K_total; });
+    for (int k : order) {   // one narrow ring that holds every call's widest tiles
+        BwdCall& c = calls[k];
+        narrow_ring(c.q, RPmax);
+        narrow_ring(c.wb, RPmax);
+        seg_add(S, c.q, SegMaps{&c.mdY_k, &c.mPB_mn, nullptr, nullptr, nullptr}, false);
+        seg_add(S, c.wb, SegMaps{&c.mdY_mn, &c.mH_mn, nullptr, nullptr, nullptr}, true);
+    }
+    tracked(h0, kShrinkDyWgradB, st, [&] { launch_segments<Op::ShrinkDy, Op::WgradB>(S, h0->num_sms, st); });
+    const uint32_t flags = h0->cfg.flags;
+    if (nc == 1 && (flags & PLORA_FLAG_BASE_PAIR)) {
+        BwdCall& c = calls[0];
+        plora_ctx* h = c.h;
+        if (c.dX) {
+            pair_params(c.p, c.P.T, h->cfg.d_in);
+            launch_pair<Op::BaseDx>(h, c.mdY_k, c.mW_mn, c.mG_k, c.mPA16, c.mdX, c.p, st);
+        }
+        narrow_ring(c.wa, c.P.RP);
+        launch_tc<Op::WgradA>(h, c.mX_mn, c.mG_mn, c.mX_mn, c.mG_mn, c.mX_mn, c.wa, st);
+    } else {
+        // K8 needs neither dX nor K6, so its items follow the dX tiles in the same persistent launch and
+        // fill its last, partial wave (on the dX GEMM's 48 KB ring, which holds them).  Without dX, K8's
+        // items run on their own narrow ring.
+        bool any_dx = false;
+        for (int k = 0; k < nc; ++k) any_dx = any_dx || calls[k].dX != nullptr;
+        S = Segments{};
+        if (any_dx) {
+            for (int k : order) {
+                BwdCall& c = calls[k];
+                seg_add(S, c.p, SegMaps{&c.mdY_k, &c.mW_mn, &c.mG_k, &c.mPA16, &c.mdX}, false);
+            }
+            for (int k : order) {
+                BwdCall& c = calls[k];
+                c.wa.stages = c.p.stages;
+                c.wa.stage_bytes = c.p.stage_bytes;
+                seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, true);
+            }
+            tracked(h0, kBaseDxWgradA, st, [&] { launch_segments<Op::BaseDx, Op::WgradA>(S, h0->num_sms, st); });
+        } else {
+            for (int k = 0; k < nc; ++k) {
+                BwdCall& c = calls[k];
+                narrow_ring(c.wa, RPmax);
+                seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, false);
+            }
+            tracked(h0, kWgradA, st, [&] { launch_segments<Op::WgradA>(S, h0->num_sms, st); });
+        }
+        if (nc == 1 && (flags & PLORA_FLAG_UNFUSED) && calls[0].dX) {
+            // K6 as its own pass: dX_i += G_i A_i^T (read-modify-write of dX).
+            BwdCall& c = calls[0];
+            plora_ctx* h = c.h;
+            TcParams r = base_params(h, c.P, c.D);
+            r.N_total = (int32_t)h->cfg.d_in;
+            r.tiles_n = (int32_t)ceil_div(h->cfg.d_in, kTileN);
+            r.num_tiles = (int32_t)c.P.tok.size() * r.tiles_n;
+            r.out = c.dX; r.out_ld = h->cfg.d_in;
+            r.out_elems = c.P.T * h->cfg.d_in;
+            r.n_items = (int32_t)c.P.tok.size();
+            launch_tc<Op::ExpandDx>(h, c.mG_k, c.mPA_mn, c.mG_k, c.mPA_mn, c.mG_k, r, st);
+        }
+    }
+    for (int k = 0; k < nc; ++k) {
+        const plora_status s = finish(calls[k].h, calls[k].D, st);
+        if (s != PLORA_OK) return s;
+    }
+    return PLORA_OK;
 }
 
 }  // namespace
@@ -763,6 +1211,8 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
 
     plora_ctx* h = new (std::nothrow) plora_ctx();
     if (!h) return PLORA_ERR_OOM;
+    h->segs.reset(new (std::nothrow) Segments());
+    if (!h->segs) { delete h; return PLORA_ERR_OOM; }
     h->cfg = *cfg;
     h->nblk = nblk;
     for (int b = 0; b < nblk; ++b) h->blk_end[b] = (int32_t)(nblk > 1 ? cfg->out_block_end[b] : cfg->d_out);
@@ -832,6 +1282,7 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradB>();
         if (e == cudaSuccess) e = set_tc_attr<Op::WgradA>();
         if (e == cudaSuccess) e = (set_tc_attr<Op::ShrinkDy, Op::WgradB>());
+        if (e == cudaSuccess) e = (set_tc_attr<Op::BaseDx, Op::WgradA>());
         if (e == cudaSuccess) e = pair_setup<Op::BaseFwd>(h->pairs_fwd);
         if (e == cudaSuccess) e = pair_setup<Op::BaseDx>(h->pairs_dx);
     }
@@ -923,27 +1374,10 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
                            const plora_adapter* tab, void* saved, void* stream) {
     if (!h) return PLORA_ERR_INVALID_ARG;
     h->last_error.clear();
-    plora_status s = check_table(h, n, off, tab, false);
-    if (s != PLORA_OK) return s;
-    const bool any_tokens = off[n] > 0;   // with no tokens, X, Y and saved are never touched
-    if (!W || (any_tokens && (!X || !Y || !saved)))
-        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, Y or saved is NULL");
-    if (!aligned16(X) || !aligned16(W) || !aligned16(Y))
-        return fail(h, PLORA_ERR_INVALID_ARG, "X, W or Y not 16-byte aligned");
-    if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0)
-        return fail(h, PLORA_ERR_INVALID_ARG, "saved not 256-byte aligned");
-    cudaError_t ce = cudaSetDevice(h->device);
-    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     HostPlan P;
-    build_plan(h, n, off, tab, P);
-    if (P.T == 0) return PLORA_OK;
-    {
-        TensorArgs ta;
-        ta.X = X; ta.W = W; ta.Y = Y; ta.saved = saved;
-        s = check_extents(h, P, tab, ta);
-        if (s != PLORA_OK) return s;
-    }
+    plora_status s = fwd_args(h, X, W, Y, n, off, tab, saved, P);
+    if (s != PLORA_OK || P.T == 0) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
 
     if (!h->tc) {
@@ -979,98 +1413,26 @@ plora_status plora_forward(plora_handle h, const void* X, const void* W, void* Y
     }
 
     // Tensor-core path.
-    DevPlan D;
-    s = upload(h, P, {}, st, D);
+    FwdCall c;
+    c.h = h; c.X = X; c.W = W; c.Y = Y; c.saved = saved;
+    c.P = std::move(P);
+    StageCopies cs{};
+    s = fwd_prepare(c, st, cs);
     if (s != PLORA_OK) return s;
-    const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
-    pack_factors(h, P, D, saved, st);
-    // mPA16: the A pack in 16-row boxes (the shrink's K-major B); mPBk / mPBk128: the B pack, K-major,
-    // 256 rows for the 1-SM tile and the expand, 128 per CTA of an SM pair.
-    const SavedLayout L = saved_layout(h, P);
-    const uint8_t* sv = static_cast<const uint8_t*>(saved);
-    CUtensorMap mX, mW, mW128, mPA16, mHk, mPBk, mPBk128, mY;
-    bool ok = make_map(&mX, X, d_in, P.T, d_in, 64, kTileM) &&
-              make_map(&mY, Y, d_out, P.T, d_out, 64, 32) &&
-              make_map(&mW, W, d_in, d_out, d_in, 64, kTileN) &&
-              make_map(&mW128, W, d_in, d_out, d_in, 64, kTileM) &&
-              make_map(&mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
-              make_map(&mHk, saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
-              make_packb_map(&mPBk, sv + L.o_packB, P.RP, d_out, P.n, kTileN) &&
-              make_packb_map(&mPBk128, sv + L.o_packB, P.RP, d_out, P.n, kTileM);
-    if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-
-    // K2: H'_i = s_i X_i A_i per 128-token tile (into the zero-padded blocks of `saved`).
-    TcParams q = base_params(h, P, D);
-    q.K_total = (int32_t)d_in;
-    q.num_tiles = (int32_t)P.tok.size();
-    q.out = saved; q.out_ld = P.RP;
-    q.out_elems = P.h_rows * P.RP;
-    q.n_items = (int32_t)P.tok.size();
-    narrow_ring(q, P.RP);
-    launch_tc<Op::ShrinkX>(h, mX, mPA16, mX, mPA16, mX, q, st);
-    // K1 (+K3): Y = X W over all packed tokens; fused, each tile also accumulates H'_j B_j of
-    // every adapter j overlapping it, so Y is written once.
-    TcParams p = base_params(h, P, D);
-    p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_out; p.K_total = (int32_t)d_in;
-    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_out, kTileN);
-    p.num_tiles = p.tiles_m * p.tiles_n;
-    p.b_box_rows = kTileN;
-    p.out = Y; p.out_ld = d_out;
-    p.fuse = fused ? 1 : 0;
-    if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
-        pair_params(p, P.T, d_out);
-        launch_pair<Op::BaseFwd>(h, mX, mW128, mHk, fused ? mPBk128 : mW128, mY, p, st);
-    } else {
-        launch_tc<Op::BaseFwd>(h, mX, mW, mHk, fused ? mPBk : mW, mY, p, st);
-    }
-    if (!fused) {
-        // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
-        TcParams r = base_params(h, P, D);
-        r.N_total = (int32_t)d_out;
-        r.tiles_n = (int32_t)ceil_div(d_out, kTileN);
-        r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
-        r.out = Y; r.out_ld = d_out;
-        r.out_elems = P.T * d_out;
-        r.n_items = (int32_t)P.tok.size();
-        launch_tc<Op::ExpandY>(h, mHk, mPBk, mHk, mPBk, mHk, r, st);
-    }
-    return finish(h, D, st);
+    return fwd_launch(&c, 1, st, cs);
 }
 
 plora_status plora_backward(plora_handle h, const void* X, const void* W, const void* dY, void* dX, int32_t n,
                             const int64_t* off, const plora_adapter* tab, const void* saved, void* stream) {
     if (!h) return PLORA_ERR_INVALID_ARG;
     h->last_error.clear();
-    plora_status s = check_table(h, n, off, tab, true);
-    if (s != PLORA_OK) return s;
-    const bool any_tokens = off[n] > 0;   // with no tokens, only dA and dB are written (zeros)
-    if (!W || (any_tokens && (!X || !dY || !saved)))
-        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, dY or saved is NULL");
-    if (!aligned16(X) || !aligned16(W) || !aligned16(dY) || (dX && !aligned16(dX)))
-        return fail(h, PLORA_ERR_INVALID_ARG, "X, W, dY or dX not 16-byte aligned");
-    if ((reinterpret_cast<uintptr_t>(saved) & 255u) != 0)
-        return fail(h, PLORA_ERR_INVALID_ARG, "saved not 256-byte aligned");
-    cudaError_t ce = cudaSetDevice(h->device);
-    if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaSetDevice");
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     HostPlan P;
-    build_plan(h, n, off, tab, P);
-    {
-        TensorArgs ta;
-        if (P.T > 0) { ta.X = X; ta.W = W; ta.dY = dY; ta.dX = dX; ta.saved = saved; }
-        ta.adapters_AB = P.T > 0;
-        ta.adapters_dA = ta.adapters_dB = true;
-        s = check_extents(h, P, tab, ta);
-        if (s != PLORA_OK) return s;
-    }
+    plora_status s = bwd_args(h, X, W, dY, dX, n, off, tab, saved, P);
+    if (s != PLORA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
-    // Adapters without tokens: their weight gradients are zero.
-    for (int32_t i : P.empty) {
-        ce = cudaMemsetAsync(tab[i].dA, 0, (size_t)tab[i].rank * h->nblk * d_in * sizeof(float), st);
-        if (ce == cudaSuccess) ce = cudaMemsetAsync(tab[i].dB, 0, (size_t)tab[i].rank * d_out * sizeof(float), st);
-        if (ce != cudaSuccess) return cuda_fail(h, ce, "cudaMemsetAsync(dA/dB of an empty adapter)");
-    }
-    if (P.T == 0) return PLORA_OK;
+    s = zero_empty_grads(h, P, tab, st);
+    if (s != PLORA_OK || P.T == 0) return s;
     void* G = h->at<void>(h->r_G);
 
     if (!h->tc) {
@@ -1112,81 +1474,13 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
         return finish(h, D, st);
     }
 
-    DevPlan D;
-    s = upload(h, P, {}, st, D);
+    BwdCall c;
+    c.h = h; c.X = X; c.W = W; c.dY = dY; c.dX = dX; c.saved = saved;
+    c.P = std::move(P);
+    StageCopies cs{};
+    s = bwd_prepare(c, st, cs);
     if (s != PLORA_OK) return s;
-    // The factors were packed into `saved` by the forward; the backward packs nothing.
-    const SavedLayout L = saved_layout(h, P);
-    const uint8_t* sv = static_cast<const uint8_t*>(saved);
-    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_mn, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn, mdX;
-    // the output map of the dX GEMM (dX may be NULL: the GEMM is skipped then)
-    bool ok = (!dX || make_map(&mdX, dX, d_in, P.T, d_in, 64, 32)) &&
-              make_map(&mdY_k, dY, d_out, P.T, d_out, 64, kTileM) &&
-              make_map(&mdY_mn, dY, d_out, P.T, d_out, 64, 64) &&
-              make_map(&mW_mn, W, d_in, d_out, d_in, 64, 64) &&
-              make_packb_map(&mPB_mn, sv + L.o_packB, P.RP, d_out, P.n, 64) &&
-              make_map(&mG_k, G, P.RP, P.h_rows, P.RP, 64, kTileM) &&
-              make_map(&mG_mn, G, P.RP, P.h_rows, P.RP, 64, 64) &&
-              make_map(&mPA_mn, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
-              make_map(&mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
-              make_map(&mH_mn, saved, P.RP, P.h_rows, P.RP, 64, 64) &&
-              make_map(&mX_mn, X, d_in, P.T, d_in, 64, 64);
-    if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-
-    const bool fused = !(h->cfg.flags & PLORA_FLAG_UNFUSED);
-    // K5: G_i = s_i dY_i B_i^T per 128-token tile (into the zero-padded workspace blocks).
-    TcParams q = base_params(h, P, D);
-    q.K_total = (int32_t)d_out;
-    q.num_tiles = (int32_t)P.tok.size();
-    q.out = G; q.out_ld = P.RP;
-    q.out_elems = (int64_t)(h->r_G.bytes / h->esize);
-    q.n_items = (int32_t)P.tok.size();
-    narrow_ring(q, P.RP);
-    // K7: dB_i = H'_i^T dY_i (a sum over each adapter's tokens) needs neither G nor dX, so its
-    // items share K5's launch and fill the last wave of K5's equal-cost token tiles.
-    TcParams wb = base_params(h, P, D);
-    wb.M_total = (int32_t)d_out;
-    wb.red_dtiles = (int32_t)ceil_div(d_out, kTileM);
-    wb.num_tiles = (int32_t)P.red.size() * wb.red_dtiles;
-    wb.n_items = (int32_t)P.red.size();
-    narrow_ring(wb, P.RP);
-    launch_tc2<Op::ShrinkDy, Op::WgradB>(h, mdY_k, mPB_mn, mdY_mn, mH_mn, q, wb, kShrinkDyWgradB, st);
-    if (dX) {
-        // K4 (+K6): dX = dY W^T; fused, each tile also accumulates G_j A_j^T of every adapter j
-        // overlapping it, so dX is written once.
-        TcParams p = base_params(h, P, D);
-        p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
-        p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
-        p.num_tiles = p.tiles_m * p.tiles_n;
-        p.out = dX; p.out_ld = d_in;
-        p.fuse = fused ? 1 : 0;
-        if (h->cfg.flags & PLORA_FLAG_BASE_PAIR) {
-            pair_params(p, P.T, d_in);
-            launch_pair<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, mdX, p, st);
-        } else {
-            launch_tc<Op::BaseDx>(h, mdY_k, mW_mn, mG_k, mPA16, mdX, p, st);
-        }
-        if (!fused) {
-            // K6 as its own pass: dX_i += G_i A_i^T (read-modify-write of dX).
-            TcParams r = base_params(h, P, D);
-            r.N_total = (int32_t)d_in;
-            r.tiles_n = (int32_t)ceil_div(d_in, kTileN);
-            r.num_tiles = (int32_t)P.tok.size() * r.tiles_n;
-            r.out = dX; r.out_ld = d_in;
-            r.out_elems = P.T * d_in;
-            r.n_items = (int32_t)P.tok.size();
-            launch_tc<Op::ExpandDx>(h, mG_k, mPA_mn, mG_k, mPA_mn, mG_k, r, st);
-        }
-    }
-    // K8: dA_i = X_i^T G_i (a sum over each adapter's tokens).
-    TcParams wa = base_params(h, P, D);
-    wa.M_total = (int32_t)d_in;
-    wa.red_dtiles = (int32_t)ceil_div(d_in, kTileM);
-    wa.num_tiles = (int32_t)P.red.size() * wa.red_dtiles;
-    wa.n_items = (int32_t)P.red.size();
-    narrow_ring(wa, P.RP);
-    launch_tc<Op::WgradA>(h, mX_mn, mG_mn, mX_mn, mG_mn, mX_mn, wa, st);
-    return finish(h, D, st);
+    return bwd_launch(&c, 1, st, cs);
 }
 
 plora_status plora_device_info(plora_handle h, int32_t* out, int32_t capacity, int32_t* count) {
@@ -1445,6 +1739,158 @@ plora_status plora_partition(int32_t n, const int64_t* counts, const int32_t* ra
     return PLORA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Layer calls: several projections over one segment map as one launch set.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+struct plora_layer_ctx {
+    int n = 0;
+    plora_ctx* h[PLORA_MAX_LAYER_PROJ] = {};
+    std::string last_error;
+};
+
+namespace {
+
+// A projection's failure, reported on the layer with the projection's index.
+plora_status layer_fail(plora_layer_ctx* L, int p, plora_status s) {
+    L->last_error = "projection " + std::to_string(p) + ": " + L->h[p]->last_error;
+    return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+plora_status plora_layer_create(plora_layer* out, int32_t n_proj, const plora_config* cfgs) {
+    if (!out) return PLORA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (n_proj < 1 || n_proj > PLORA_MAX_LAYER_PROJ || !cfgs) return PLORA_ERR_INVALID_ARG;
+    for (int32_t p = 0; p < n_proj; ++p)
+        if (cfgs[p].dtype != PLORA_BF16 || (cfgs[p].flags & (PLORA_FLAG_SIMT | PLORA_FLAG_UNFUSED | PLORA_FLAG_BASE_PAIR)))
+            return PLORA_ERR_UNSUPPORTED;
+    plora_layer_ctx* L = new (std::nothrow) plora_layer_ctx();
+    if (!L) return PLORA_ERR_OOM;
+    for (int32_t p = 0; p < n_proj; ++p) {
+        const plora_status s = plora_create(&L->h[p], &cfgs[p]);
+        if (s != PLORA_OK) {
+            plora_layer_destroy(L);
+            return s;
+        }
+        L->n = p + 1;
+        if (L->h[p]->device != L->h[0]->device) {
+            plora_layer_destroy(L);
+            return PLORA_ERR_INVALID_ARG;
+        }
+    }
+    *out = L;
+    return PLORA_OK;
+}
+
+plora_status plora_layer_destroy(plora_layer L) {
+    if (!L) return PLORA_OK;
+    for (int p = 0; p < L->n; ++p) plora_destroy(L->h[p]);
+    delete L;
+    return PLORA_OK;
+}
+
+plora_status plora_layer_handle(plora_layer L, int32_t p, plora_handle* h) {
+    if (!L || !h || p < 0 || p >= L->n) return PLORA_ERR_INVALID_ARG;
+    *h = L->h[p];
+    return PLORA_OK;
+}
+
+const char* plora_layer_last_error(plora_layer L) { return L ? L->last_error.c_str() : ""; }
+
+plora_status plora_layer_saved_bytes(plora_layer L, int32_t n, const int64_t* off, const plora_proj* projs,
+                                     size_t* bytes) {
+    if (!L) return PLORA_ERR_INVALID_ARG;
+    L->last_error.clear();
+    if (!projs || !bytes) {
+        L->last_error = "projs or bytes is NULL";
+        return PLORA_ERR_INVALID_ARG;
+    }
+    for (int p = 0; p < L->n; ++p) {
+        const plora_status s = plora_saved_bytes(L->h[p], n, off, projs[p].tab, &bytes[p]);
+        if (s != PLORA_OK) return layer_fail(L, p, s);
+    }
+    return PLORA_OK;
+}
+
+plora_status plora_layer_forward(plora_layer L, int32_t n, const int64_t* off, const plora_proj* projs, void* stream) {
+    if (!L) return PLORA_ERR_INVALID_ARG;
+    L->last_error.clear();
+    if (!projs) {
+        L->last_error = "projs is NULL";
+        return PLORA_ERR_INVALID_ARG;
+    }
+    std::vector<FwdCall> calls(L->n);
+    for (int p = 0; p < L->n; ++p) {   // every check of every projection before anything is enqueued
+        plora_ctx* h = L->h[p];
+        h->last_error.clear();
+        const plora_proj& io = projs[p];
+        const plora_status s = fwd_args(h, io.X, io.W, io.Y, n, off, io.tab, io.saved, calls[p].P);
+        if (s != PLORA_OK) return layer_fail(L, p, s);
+        calls[p].h = h;
+        calls[p].X = io.X; calls[p].W = io.W; calls[p].Y = io.Y; calls[p].saved = io.saved;
+    }
+    if (calls[0].P.T == 0) return PLORA_OK;   // the segment map is shared: no tokens anywhere
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    StageCopies cs{};
+    for (int p = 0; p < L->n; ++p) {
+        const plora_status s = fwd_prepare(calls[p], st, cs);
+        if (s != PLORA_OK) return layer_fail(L, p, s);
+    }
+    const plora_status s = fwd_launch(calls.data(), L->n, st, cs);
+    return s == PLORA_OK ? s : layer_fail(L, 0, s);
+}
+
+plora_status plora_layer_backward(plora_layer L, int32_t n, const int64_t* off, const plora_proj* projs, void* stream) {
+    if (!L) return PLORA_ERR_INVALID_ARG;
+    L->last_error.clear();
+    if (!projs) {
+        L->last_error = "projs is NULL";
+        return PLORA_ERR_INVALID_ARG;
+    }
+    std::vector<BwdCall> calls(L->n);
+    for (int p = 0; p < L->n; ++p) {
+        plora_ctx* h = L->h[p];
+        h->last_error.clear();
+        const plora_proj& io = projs[p];
+        const plora_status s = bwd_args(h, io.X, io.W, io.dY, io.dX, n, off, io.tab, io.saved, calls[p].P);
+        if (s != PLORA_OK) return layer_fail(L, p, s);
+        calls[p].h = h;
+        calls[p].X = io.X; calls[p].W = io.W; calls[p].dY = io.dY; calls[p].dX = io.dX; calls[p].saved = io.saved;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int p = 0; p < L->n; ++p) {
+        const plora_status s = zero_empty_grads(L->h[p], calls[p].P, projs[p].tab, st);
+        if (s != PLORA_OK) return layer_fail(L, p, s);
+    }
+    if (calls[0].P.T == 0) return PLORA_OK;
+    StageCopies cs{};
+    for (int p = 0; p < L->n; ++p) {
+        const plora_status s = bwd_prepare(calls[p], st, cs);
+        if (s != PLORA_OK) return layer_fail(L, p, s);
+    }
+    const plora_status s = bwd_launch(calls.data(), L->n, st, cs);
+    return s == PLORA_OK ? s : layer_fail(L, 0, s);
+}
+
+plora_status plora_layer_check(plora_layer L, void* stream) {
+    if (!L) return PLORA_ERR_INVALID_ARG;
+    L->last_error.clear();
+    plora_status first = PLORA_OK;
+    for (int p = 0; p < L->n; ++p) {   // every projection's flag is read (and cleared)
+        const plora_status s = plora_check(L->h[p], stream);
+        if (s != PLORA_OK && first == PLORA_OK) {
+            first = s;
+            layer_fail(L, p, s);
+        }
+    }
+    return first;
+}
+
 }  // extern "C"
 
 // ===========================================================================
@@ -1648,8 +2094,9 @@ extern "C" plora_status plora_grad_B_static(const plora_config* cfg, const void*
     p.part_elems = (int64_t)((kStaticScratchBytes - L.o_part) / sizeof(float));
     p.n_counters = (int32_t)(L.cnt_bytes / sizeof(int32_t));
     narrow_ring(p, P.RP);
-    if (p.num_tiles > 0)
-        tc_kernel<Op::WgradB><<<std::min(p.num_tiles, sd.num_sms), kTcThreads, kTcSmemBytes, st>>>(mdY, mH, mdY, mH, mdY,
-                                                                                                    p, p);
+    std::unique_ptr<Segments> S(new (std::nothrow) Segments());   // host memory, not device
+    if (!S) return PLORA_ERR_OOM;
+    seg_add(*S, p, SegMaps{&mdY, &mH, nullptr, nullptr, nullptr}, false);
+    if (launch_segments<Op::WgradB>(*S, sd.num_sms, st) != cudaSuccess) return PLORA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? PLORA_OK : PLORA_ERR_CUDA;
 }

@@ -30,8 +30,10 @@
 // op's epilogue while the next tile is being multiplied.
 //
 // A launch may carry a second, independent op (tc_kernel<OP, OP2>): its work
-// items follow OP's in the same persistent grid (the backward runs dB's items
-// after G's, filling the last wave of G's equal-cost token tiles).
+// items follow OP's in the same persistent grid, with operands from their own
+// tensor maps (the backward runs dB's items after G's, filling the last wave of
+// G's equal-cost token tiles, and dA's after the dX GEMM's tiles, filling its
+// last, partial wave).
 //
 // Output blocks: W may stack P projections that read the same X (q|k|v).  Each
 // adapter then has one rank-r pair per block; H' and G hold block b in columns
@@ -690,20 +692,32 @@ __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo&
     }
 }
 
-// One persistent launch runs the work items of OP (p.num_tiles of them) followed, when OP2
-// differs from OP, by those of OP2 (p2.num_tiles, with operands from tmA2 / tmB2).  Both ops
-// use the ring layout of p (stages, stage_bytes).  Items are dealt round-robin over the CTAs,
-// so the second op's items fill the last, partial wave of the first op's.
+// One persistent launch runs the work items of up to kMaxSeg independent products ("segments"):
+// segments [0, n_op1) run OP and the others OP2 (the backward runs dB's items after G's, filling the
+// last wave of G's equal-cost token tiles, and dA's after the dX GEMM's tiles, filling its last,
+// partial wave; the layer calls run one product kind of several projections together).  Segment j
+// owns items [begin[j], begin[j+1]) and has its own parameters and tensor maps: m[j][0..1] the
+// operands, m[j][2..3] a base GEMM's folded low-rank branch, m[j][4] a base GEMM's output.  Every
+// segment uses the ring layout of segment 0 (stages, stage_bytes), which must hold all their tiles.
+// Items are dealt round-robin over the CTAs.
+constexpr int kMaxSeg = 16;
+
+struct GroupParams {
+    int32_t n_seg, n_op1;
+    int32_t begin[kMaxSeg + 1];
+    TcParams p[kMaxSeg];
+};
+struct GroupMaps {
+    CUtensorMap m[kMaxSeg][5];
+};
+
 template <Op OP, Op OP2 = OP>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-          const __grid_constant__ CUtensorMap tmC, const TcParams p, const TcParams p2) {
+tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupParams g) {
     using Tr = OpTraits<OP>;
-    constexpr bool kDual = OP2 != OP;
-    static_assert(!kDual || (!Tr::kBase && !OpTraits<OP2>::kBase),
-                  "a base GEMM reads its low-rank branch through tmA2 / tmB2");
-    const int total = p.num_tiles + (kDual ? p2.num_tiles : 0);
+    static_assert(OP2 == OP || !OpTraits<OP2>::kBase, "the second op of a launch is not a base GEMM");
+    const TcParams& p0 = g.p[0];
+    const int total = g.begin[g.n_seg];
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
@@ -713,13 +727,28 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     uint64_t* acce_bar = bars + 2 * kMaxStages + 2;  // [2]
     uint64_t* drain_bar = bars + 2 * kMaxStages + 4;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 5);
-    const int nst = p.stages;                        // ring depth of this launch
-    const int stb = p.stage_bytes;                   // bytes per stage (multiple of 1024)
+    const int nst = p0.stages;                       // ring depth of this launch
+    const int stb = p0.stage_bytes;                  // bytes per stage (multiple of 1024)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* red_flag = reinterpret_cast<int*>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+
+    // The segment of item t (a short scan: at most kMaxSeg segments).
+    auto seg_of = [&](int t) {
+        int j = 0;
+        while (j + 1 < g.n_seg && t >= g.begin[j + 1]) ++j;
+        return j;
+    };
+    // The folded low-rank record of item t of a base GEMM (empty otherwise, and past the end).
+    auto rec_of = [&](int t) {
+        MTileRec r;
+        r.q0 = r.q1 = 0;
+        if (!Tr::kBase || t >= total) return r;
+        const int j = seg_of(t);
+        return j < g.n_op1 ? load_mtile<OP>(g.p[j], t - g.begin[j]) : r;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
@@ -735,13 +764,9 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         ptx::fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        ptx::tma_prefetch_desc(&tmA);
-        ptx::tma_prefetch_desc(&tmB);
-        if (Tr::kBase) ptx::tma_prefetch_desc(&tmC);
-        if ((Tr::kBase && p.fuse) || kDual) {
-            ptx::tma_prefetch_desc(&tmA2);
-            ptx::tma_prefetch_desc(&tmB2);
-        }
+        // every map slot of every segment holds a valid map (the host fills unused slots with copies)
+        for (int j = 0; j < g.n_seg; ++j)
+            for (int k = 0; k < 5; ++k) ptx::tma_prefetch_desc(&maps.m[j][k]);
     }
     if (warp == 1) {
         ptx::tmem_alloc<kTmemCols>(tmem_slot);
@@ -751,7 +776,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const uint64_t lim = p.timeout_ns;
+    const uint64_t lim = p0.timeout_ns;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -760,22 +785,25 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             uint32_t armed = 0, armed_par = 0;
             bool ok = true;
             // The folded low-rank record of a base tile is fetched one tile ahead.
-            MTileRec lr_next = load_mtile<OP>(p, blockIdx.x);
+            MTileRec lr_next = rec_of(blockIdx.x);
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const MTileRec lr = lr_next;
-                lr_next = load_mtile<OP>(p, t + gridDim.x);
-                if (kDual && t >= p.num_tiles)
-                    ok = produce_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), lr, &tmA2, &tmB2, &tmA2, &tmB2,
+                lr_next = rec_of(t + gridDim.x);
+                const int j = seg_of(t);
+                const CUtensorMap* m = maps.m[j];
+                const TcParams& pj = g.p[j];
+                if (j >= g.n_op1)
+                    ok = produce_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), lr, &m[0], &m[1], &m[2], &m[3],
                                            smem, stb, nst, full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
                 else
-                    ok = produce_item<OP>(p, decode_tile<OP>(p, t), lr, &tmA, &tmB, &tmA2, &tmB2, smem, stb, nst,
-                                          full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
+                    ok = produce_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, &m[0], &m[1], &m[2], &m[3],
+                                          smem, stb, nst, full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
             }
             // Drain: every load this thread issued must have landed before the CTA exits.
             for (int s = 0; s < nst; ++s)
                 if (armed & (1u << s)) {
                     int dummy = 0;
-                    ptx::mbar_wait(&full_bar[s], (armed_par >> s) & 1u, &dummy, lim, p.err_flag);
+                    ptx::mbar_wait(&full_bar[s], (armed_par >> s) & 1u, &dummy, lim, p0.err_flag);
                 }
         }
     } else if (warp == 1) {
@@ -784,18 +812,20 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             RingPos rp{0, 0u};
             int abuf = 0;
             uint32_t aphase = 0;
-            MTileRec lr_next = load_mtile<OP>(p, blockIdx.x);
+            MTileRec lr_next = rec_of(blockIdx.x);
             for (int t = blockIdx.x; t < total; t += gridDim.x) {
                 const MTileRec lr = lr_next;
-                lr_next = load_mtile<OP>(p, t + gridDim.x);
-                if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p.err_flag)) break;
+                lr_next = rec_of(t + gridDim.x);
+                if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p0.err_flag)) break;
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
-                const bool ok = (kDual && t >= p.num_tiles)
-                    ? mma_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), lr, smem, stb, nst, full_bar,
+                const int j = seg_of(t);
+                const TcParams& pj = g.p[j];
+                const bool ok = (j >= g.n_op1)
+                    ? mma_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar,
                                     empty_bar, d_tmem, rp, abort_flag, lim)
-                    : mma_item<OP>(p, decode_tile<OP>(p, t), lr, smem, stb, nst, full_bar, empty_bar, d_tmem, rp,
-                                   abort_flag, lim);
+                    : mma_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar, empty_bar,
+                                   d_tmem, rp, abort_flag, lim);
                 if (!ok) break;
                 ptx::tc_commit(&accf_bar[abuf]);
                 if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
@@ -803,7 +833,7 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
             // Drain: all issued MMAs complete before TMEM is released.
             ptx::tc_commit(drain_bar);
             int dummy = 0;
-            ptx::mbar_wait(drain_bar, 0, &dummy, lim, p.err_flag);
+            ptx::mbar_wait(drain_bar, 0, &dummy, lim, p0.err_flag);
         }
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..5)
@@ -812,13 +842,17 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         int abuf = 0;
         uint32_t aphase = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            if (!ptx::mbar_wait(&accf_bar[abuf], aphase, abort_flag, lim, p.err_flag)) break;
+            if (!ptx::mbar_wait(&accf_bar[abuf], aphase, abort_flag, lim, p0.err_flag)) break;
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
-            if (kDual && t >= p.num_tiles)
-                epilogue_item<OP2>(p2, decode_tile<OP2>(p2, t - p.num_tiles), t_row, q, lane, wbuf, &tmC, red_flag);
+            const int j = seg_of(t);
+            const TcParams& pj = g.p[j];
+            if (j >= g.n_op1)
+                epilogue_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), t_row, q, lane, wbuf, &maps.m[j][4],
+                                   red_flag);
             else
-                epilogue_item<OP>(p, decode_tile<OP>(p, t), t_row, q, lane, wbuf, &tmC, red_flag);
+                epilogue_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), t_row, q, lane, wbuf, &maps.m[j][4],
+                                  red_flag);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
@@ -848,16 +882,36 @@ tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 // of H' B into Y (K-major, block b's columns) and the shrink of G = s dY B^T (MN-major: column
 // b rblk + k of G sums over block b's output columns only, as output blocks need).
 // ---------------------------------------------------------------------------
-// grid (gx, n adapters), block 256: per adapter, a grid-stride loop over its 16-byte chunks, first the
-// rp16 x d_in/8 chunks of packA, then the d_out x rp16/8 chunks of packB (consecutive threads on
-// consecutive bytes of both sources and destinations).
-__global__ void __launch_bounds__(256) pack_ab_kernel(const AdapterDev* __restrict__ ad, int RP, int64_t d_in,
-                                                      int64_t d_out, OutBlocks blocks,
-                                                      __nv_bfloat16* __restrict__ packA,
-                                                      __nv_bfloat16* __restrict__ packB, int64_t packA_elems,
-                                                      int64_t packB_elems, int* err_flag) {
+// One projection's pack: its adapter table, the pitch RP, the sizes, the output blocks and where the
+// two packs go (with their extents, for the PLORA_DEBUG checks).
+struct PackJob {
+    const AdapterDev* ad;
+    __nv_bfloat16* packA;
+    __nv_bfloat16* packB;
+    int64_t d_in, d_out, packA_elems, packB_elems;
+    int32_t n, RP;
+    OutBlocks blocks;
+    int* err_flag;
+};
+constexpr int kMaxPackJobs = 16;
+struct PackJobs {
+    int32_t n;
+    PackJob j[kMaxPackJobs];
+};
+
+// grid (gx, adapters, jobs), block 256: per adapter of a job, a grid-stride loop over its 16-byte
+// chunks, first the rp16 x d_in/8 chunks of packA, then the d_out x rp16/8 chunks of packB (consecutive
+// threads on consecutive bytes of both sources and destinations).
+__global__ void __launch_bounds__(256) pack_ab_kernel(const __grid_constant__ PackJobs jobs) {
+    if ((int)blockIdx.z >= jobs.n) return;
+    const PackJob& J = jobs.j[blockIdx.z];
     const int i = blockIdx.y;
-    const AdapterDev a = ad[i];
+    if (i >= J.n) return;
+    const AdapterDev a = J.ad[i];
+    const int RP = J.RP;
+    const int64_t d_in = J.d_in, d_out = J.d_out;
+    __nv_bfloat16* __restrict__ packA = J.packA;
+    __nv_bfloat16* __restrict__ packB = J.packB;
     const int r = a.rank, rblk = a.rblk;
     const int64_t va = d_in / 8;
     const int64_t ua = (int64_t)a.rp16 * va;
@@ -871,7 +925,8 @@ __global__ void __launch_bounds__(256) pack_ab_kernel(const AdapterDev* __restri
             const int j = (int)(e / va);
             const int64_t v = e - (int64_t)j * va;
             const int pb = j / rblk, k = j - pb * rblk;      // output block pb's rank row k
-            if (!dcheck(err_flag, pb < blocks.n && j < RP && ((int64_t)i * RP + j) * d_in + (v + 1) * 8 <= packA_elems))
+            if (!dcheck(J.err_flag, pb < J.blocks.n && j < RP &&
+                                        ((int64_t)i * RP + j) * d_in + (v + 1) * 8 <= J.packA_elems))
                 continue;
             if (k < r) val = reinterpret_cast<const uint4*>(A + (int64_t)(pb * r + k) * d_in)[v];
             reinterpret_cast<uint4*>(packA + ((int64_t)i * RP + j) * d_in)[v] = val;
@@ -881,7 +936,7 @@ __global__ void __launch_bounds__(256) pack_ab_kernel(const AdapterDev* __restri
             const int col = (int)(f - c * vb) * 8;
             const int pb = col / rblk, k0 = col - pb * rblk;  // 8 columns of one block (rblk % 16 == 0)
             int cb = 0;
-            while (cb + 1 < blocks.n && c >= blocks.end[cb]) ++cb;
+            while (cb + 1 < J.blocks.n && c >= J.blocks.end[cb]) ++cb;
             if (cb == pb && k0 < r) {
                 const __nv_bfloat16* src = B + c * r + k0;
                 if ((r & 7) == 0) {
@@ -893,7 +948,7 @@ __global__ void __launch_bounds__(256) pack_ab_kernel(const AdapterDev* __restri
                     val = *reinterpret_cast<const uint4*>(v);
                 }
             }
-            if (!dcheck(err_flag, col + 8 <= RP && ((int64_t)i * d_out + c) * RP + col + 8 <= packB_elems)) continue;
+            if (!dcheck(J.err_flag, col + 8 <= RP && ((int64_t)i * d_out + c) * RP + col + 8 <= J.packB_elems)) continue;
             *reinterpret_cast<uint4*>(packB + ((int64_t)i * d_out + c) * RP + col) = val;
         }
     }

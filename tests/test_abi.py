@@ -270,3 +270,22 @@ def test_make_config_writes_cumulative_block_ends():
     off = np.array([0, 10], np.int64)
     s, v = pl.plora_debug_schedule(c, 1, off, fake_table([16]), False, 3)
     assert s == pl.PLORA_OK and v[0] == 3 * 16 + 16        # RP: 3 blocks x 16, rounded up to 64
+
+
+def test_layer_create_refuses_bad_layers_without_a_device():
+    """plora_layer_create checks the projection count and each configuration's path before it creates
+    any handle, so these refusals need no GPU."""
+    lib = pl.load()
+    L = ctypes.c_void_p()
+    cfg = pl.make_config(256, 256, pl.PLORA_BF16, 4, 16, 1024)
+    cfgs = (pl.plora_config * 9)(*([cfg] * 9))
+    assert lib.plora_layer_create(ctypes.byref(L), 0, cfgs) == pl.PLORA_ERR_INVALID_ARG
+    assert lib.plora_layer_create(ctypes.byref(L), 9, cfgs) == pl.PLORA_ERR_INVALID_ARG
+    assert lib.plora_layer_create(ctypes.byref(L), 2, None) == pl.PLORA_ERR_INVALID_ARG
+    for flags in (pl.PLORA_FLAG_SIMT, pl.PLORA_FLAG_UNFUSED, pl.PLORA_FLAG_BASE_PAIR):
+        bad = (pl.plora_config * 2)(cfg, pl.make_config(256, 256, pl.PLORA_BF16, 4, 16, 1024, flags))
+        assert lib.plora_layer_create(ctypes.byref(L), 2, bad) == pl.PLORA_ERR_UNSUPPORTED
+    f32 = (pl.plora_config * 1)(pl.make_config(256, 256, pl.PLORA_FP32, 4, 16, 1024))
+    assert lib.plora_layer_create(ctypes.byref(L), 1, f32) == pl.PLORA_ERR_UNSUPPORTED
+    assert L.value is None
+    assert lib.plora_layer_destroy(None) == pl.PLORA_OK
