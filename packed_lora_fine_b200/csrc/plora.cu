@@ -30,6 +30,16 @@ using namespace plora;
 namespace {
 
 constexpr int kSlots = 4;                   // host staging / device schedule ring depth
+// Rasterisation windows of the base GEMMs (rows of A whose tiles walk every n-tile together):
+// 4096 rows keeps X's window (32 MB for d_in = 4096) in L2 while W streams past it.
+#ifndef PLORA_WINDOW_ROWS
+#define PLORA_WINDOW_ROWS 4096
+#endif
+#ifndef PLORA_DX_WINDOW_ROWS
+#define PLORA_DX_WINDOW_ROWS 4096
+#endif
+constexpr int kWindowRows = PLORA_WINDOW_ROWS;
+constexpr int kDxWindowRows = PLORA_DX_WINDOW_ROWS;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 struct Region {
@@ -714,7 +724,7 @@ void pair_params(TcParams& p, int64_t T, int64_t N) {
     p.tiles_m = (int32_t)ceil_div(T, 2 * kTileM);
     p.tiles_n = (int32_t)ceil_div(N, kTileN);
     p.num_tiles = p.tiles_m * p.tiles_n;
-    p.group_m = 16;   // the same 4096-row window in 256-row pair tiles
+    p.group_m = std::max(1, p.group_m / 2);   // the same row window in 256-row pair tiles
     p.stage_bytes = kPairStageBytes;
     p.stages = std::min(kMaxStages, kRingBytes / kPairStageBytes);
 }
@@ -740,7 +750,7 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     p.timeout_ns = kTimeoutNs;
     p.partials = h->at<float>(h->r_part);
     p.counters = h->at<int32_t>(h->r_cnt);
-    p.group_m = 32;   // 32 x 128 rows: a 4096-row window of A stays in L2 while W streams past it
+    p.group_m = kWindowRows / kTileM;   // a window of A's rows stays in L2 while W streams past it
     p.mt_rec = D.mt_rec;
     p.mt_seg = D.mt_seg;
     p.fuse = 0;
@@ -1057,6 +1067,7 @@ plora_status bwd_prepare(BwdCall& c, cudaStream_t st, StageCopies& cs) {
     p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
     p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
     p.num_tiles = c.dX ? p.tiles_m * p.tiles_n : 0;
+    p.group_m = kDxWindowRows / kTileM;
     p.out = c.dX; p.out_ld = d_in;
     p.fuse = (h->cfg.flags & PLORA_FLAG_UNFUSED) ? 0 : 1;
     // K8: dA_i = X_i^T G_i (a sum over each adapter's tokens).

@@ -46,6 +46,8 @@
 #include "plan.cuh"
 #include "ptx.cuh"
 
+
+
 namespace plora {
 
 enum class Op : int { BaseFwd = 0, BaseDx, ShrinkX, ShrinkDy, ExpandY, ExpandDx, WgradB, WgradA };
@@ -151,7 +153,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {  // 
         const int first_m = g * p.group_m;
         const int gm = min(p.tiles_m - first_m, p.group_m);
         const int r = t - g * per_group;
-        const int mb = first_m + r % gm;
+        const int mb = first_m + r % gm;          // m-tiles fastest within the window
         const int nb = r / gm;
         ti.mtile = mb;
         ti.a_x = 0;
