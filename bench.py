@@ -63,6 +63,8 @@ def parse_args(argv=None):
                     help="run the expand products as separate passes (for comparison with the fused default)")
     ap.add_argument("--base-pair", action="store_true",
                     help="base GEMMs on SM pairs (cta_group::2) instead of single SMs")
+    ap.add_argument("--layer-tokens", type=int, default=8192,
+                    help="tokens per adapter of the one-layer line (the stated workload has 8192)")
     ap.add_argument("--layer-only", action="store_true",
                     help="only the suite's one-layer line (seven calls, four calls with output blocks, one layer call)")
     ap.add_argument("--suite", action="store_true",
@@ -860,7 +862,7 @@ def layer_shared_inputs(args):
     calls, as four calls with q|k|v and gate|up stacked as output blocks (one base GEMM each), and as
     one layer call over those four (plora_layer_*: one launch set, one persistent launch per product
     kind).  The projections are independent here (no attention or activation between them).
-    16 adapters x 8192 tokens, r ~ U{16,32,64}, alpha = 2r.  One JSON line."""
+    16 adapters x 8192 tokens (--layer-tokens), r ~ U{16,32,64}, alpha = 2r.  One JSON line."""
     import torch
     import packed_lora_fine_b200 as pl
     dev = torch.device("cuda", 0)
@@ -869,7 +871,7 @@ def layer_shared_inputs(args):
     g.manual_seed(args.seed + 7)
     ranks = [int(x) for x in wl.rng_for(1004, 1).choice(np.array([16, 32, 64]), size=16)]
     n = len(ranks)
-    off = np.arange(n + 1, dtype=np.int64) * 8192
+    off = np.arange(n + 1, dtype=np.int64) * args.layer_tokens
     T = int(off[-1])
     scales = [2.0] * n
     shape = {nm: (di, do) for nm, di, do in wl.LLAMA3_LAYER}
@@ -914,16 +916,36 @@ def layer_shared_inputs(args):
             pl.plora_backward(e.h, c["X"].data_ptr(), c["W"].data_ptr(), c["dY"].data_ptr(), c["dX"].data_ptr(),
                               n, off, c["tb"], c["saved"].data_ptr(), st.cuda_stream)
 
-    def timed(calls, steps):
+    gpu_uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    if not gpu_uuid.startswith("GPU-"):
+        gpu_uuid = "GPU-" + gpu_uuid
+    power = {"fused_calls": [], "layer_call": []}
+
+    def metered(key, run, steps):
+        # energy per step and median SM clock over the timed steps of run (after its warm-up)
+        energy, clocks = EnergyMeter(gpu_uuid), ClockSampler(gpu_uuid)
+        energy.start()
+        clocks.start()
+        out = run()
+        clk = clocks.stop()
+        joules, _ = energy.stop()
+        power[key].append({"j_per_step": None if joules is None else round(joules / steps, 2),
+                           "sm_mhz": clk["sm_mhz"]})
+        return out
+
+    def timed(calls, steps, meter=None):
         for _ in range(3):
             step(calls)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(st)
-        for _ in range(steps):
-            step(calls)
-        e1.record(st)
-        torch.cuda.synchronize()
+
+        def run():
+            e0.record(st)
+            for _ in range(steps):
+                step(calls)
+            e1.record(st)
+            torch.cuda.synchronize()
+        metered(meter, run, steps) if meter else run()
         for c in calls:
             assert pl.plora_check(c["eng"].h, 0) == pl.PLORA_OK
         return e0.elapsed_time(e1) / steps
@@ -965,21 +987,61 @@ def layer_shared_inputs(args):
         assert lib.plora_layer_forward(layer.L, n, offc.ctypes.data, pf, st.cuda_stream) == pl.PLORA_OK
         assert lib.plora_layer_backward(layer.L, n, offc.ctypes.data, pb, st.cuda_stream) == pl.PLORA_OK
 
-    def timed_layer(steps):
+    def timed_layer(steps, profile=False, meter=None):
         for _ in range(3):
             layer_step(None)
         torch.cuda.synchronize()
         pl.plora_profile_read(layer.handle(0))
+        pl.plora_profile_enable(layer.handle(0), profile)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(st)
-        for _ in range(steps):
-            layer_step(None)
-        e1.record(st)
-        torch.cuda.synchronize()
+
+        def run():
+            e0.record(st)
+            for _ in range(steps):
+                layer_step(None)
+            e1.record(st)
+            torch.cuda.synchronize()
+        metered(meter, run, steps) if meter else run()
         assert layer.check() == pl.PLORA_OK
-        return e0.elapsed_time(e1) / steps, sum(v[0] for v in pl.plora_profile_read(layer.handle(0)).values()) / steps
-    ms_layer, launches_layer = timed_layer(steps)
+        prof = pl.plora_profile_read(layer.handle(0))
+        pl.plora_profile_enable(layer.handle(0), False)
+        return e0.elapsed_time(e1) / steps, prof
+
+    # the four calls again on the same buffers, alternated with the layer call (the power-capped clock
+    # drifts over a run), and one profiled pass of each for the per-kernel split
+    refused = []
+    for c, grp in zip(fused, groups):
+        c["eng"] = pl.PackedLoRA(c["X"].shape[1], c["Y"].shape[1], "bf16", max_adapters=n, max_rank=max(ranks),
+                                 max_tokens=T, out_blocks=[shape[nm][1] for nm in grp] if len(grp) > 1 else None)
+        refused.append(c["eng"])
+    ms_layer_runs, ms_fused_runs = [], []
+    for _ in range(2):
+        ms_fused_runs.append(timed(fused, steps, meter="fused_calls"))
+        ms_layer_runs.append(timed_layer(steps, meter="layer_call")[0])
+    ms_layer, ms_fused = min(ms_layer_runs), min(ms_fused_runs)
+
+    def kernel_split(prof, steps_):
+        return {k: round(v[1] / steps_, 4) for k, v in prof.items() if v[0]}
+    _, prof_layer = timed_layer(steps, profile=True)
+    launches_layer = sum(v[0] for v in prof_layer.values()) / steps
+    for _ in range(3):
+        step(fused)
+    torch.cuda.synchronize()
+    for c in fused:
+        pl.plora_profile_read(c["eng"].h)
+        pl.plora_profile_enable(c["eng"].h, True)
+    for _ in range(steps):
+        step(fused)
+    torch.cuda.synchronize()
+    prof_fused = {}
+    for c in fused:
+        for k, (cnt, tot) in pl.plora_profile_read(c["eng"].h).items():
+            a, b = prof_fused.get(k, (0, 0.0))
+            prof_fused[k] = (a + cnt, b + tot)
+        pl.plora_profile_enable(c["eng"].h, False)
     same_layer = all(bool(torch.equal(c["Y"], y)) for c, y in zip(fused, y_fused))
+    for e in refused:
+        e.close()
     layer.close()
     print(json.dumps({"suite": "llama3-8b layer, shared inputs: q|k|v and gate|up as output blocks",
                       "tokens": T, "adapters": n, "projections": 7,
@@ -990,6 +1052,10 @@ def layer_shared_inputs(args):
                       "layer_call_ms_per_step": ms_layer, "layer_call_tokens_per_s": T / (ms_layer / 1e3),
                       "layer_call_launches_per_step": launches_layer,
                       "layer_call_over_fused_calls": ms_fused / ms_layer,
+                      "alternated_ms": {"fused_calls": ms_fused_runs, "layer_call": ms_layer_runs},
+                      "alternated_power": power,
+                      "kernels_ms_per_step": {"fused_calls": kernel_split(prof_fused, steps),
+                                              "layer_call": kernel_split(prof_layer, steps)},
                       "layer_call_outputs_bit_identical": same_layer}), flush=True)
     torch.cuda.empty_cache()
 

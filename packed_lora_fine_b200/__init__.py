@@ -470,7 +470,9 @@ class PackedLoRALayer:
     ``projections`` lists each projection as ``(d_in, d_out)`` or ``(d_in, d_out, out_blocks)``.
     ``forward(io, off, scales)`` takes one dict per projection with its ``X``, ``W``, ``A``, ``B``
     torch tensors and returns ``[(Y, saved)]``; ``backward(io, off, scales, saved)`` takes the same
-    dicts with ``dY`` added and returns ``[(dX, dA, dB)]``.  Results equal separate calls bit for bit.
+    dicts with ``dY`` added and returns ``[(dX, dA, dB)]``.  ``scales`` is one list of per-adapter
+    scales for every projection, or one such list per projection (an adapter's alpha / r differs
+    between projections where its rank does).  Results equal separate calls bit for bit.
     """
 
     def __init__(self, projections, max_adapters=64, max_rank=PLORA_MAX_RANK, max_tokens=1 << 16):
@@ -508,6 +510,12 @@ class PackedLoRALayer:
             raise PloraError(st, f"{what}: {load().plora_layer_last_error(self.L).decode()}")
 
     @staticmethod
+    def _scales(scales, k):
+        """Projection k's per-adapter scales from one shared list or a list per projection."""
+        first = scales[0] if len(scales) else None
+        return scales[k] if isinstance(first, (list, tuple, np.ndarray)) else scales
+
+    @staticmethod
     def _table(scales, A, B, dA=None, dB=None):
         return make_table([b.shape[1] for b in B], scales, [a.data_ptr() for a in A], [b.data_ptr() for b in B],
                           None if dA is None else [x.data_ptr() for x in dA],
@@ -519,7 +527,7 @@ class PackedLoRALayer:
         n = len(off) - 1
         items, outs = [], []
         for k, d in enumerate(io):
-            tab = self._table(scales, d["A"], d["B"])
+            tab = self._table(self._scales(scales, k), d["A"], d["B"])
             Y = torch.empty((d["X"].shape[0], self.proj[k][1]), dtype=d["X"].dtype, device=d["X"].device)
             items.append({"X": d["X"].data_ptr(), "W": d["W"].data_ptr(), "Y": Y.data_ptr(), "tab": tab})
             outs.append(Y)
@@ -542,7 +550,7 @@ class PackedLoRALayer:
             dA = [torch.empty(a.shape, dtype=torch.float32, device=a.device) for a in d["A"]]
             dB = [torch.empty(b.shape, dtype=torch.float32, device=b.device) for b in d["B"]]
             dX = torch.empty_like(d["X"]) if want_dX else None
-            tab = self._table(scales, d["A"], d["B"], dA, dB)
+            tab = self._table(self._scales(scales, k), d["A"], d["B"], dA, dB)
             items.append({"X": d["X"].data_ptr(), "W": d["W"].data_ptr(), "dY": d["dY"].data_ptr(),
                           "dX": dX.data_ptr() if want_dX else None, "tab": tab, "saved": saved[k].data_ptr()})
             outs.append((dX, dA, dB))

@@ -108,3 +108,40 @@ def test_layer_call_rejects_a_bad_projection_and_writes_nothing():
     torch.cuda.synchronize()
     assert all(bool(torch.all(y == 7.0)) for y in Y)
     layer.close()
+
+
+def test_layer_call_with_different_ranks_per_projection_and_a_skipped_dX():
+    """Each projection has its own adapter table: here the same adapters carry ranks up to 16 in one
+    projection and up to 200 in the other (so the shared narrow ring must hold the wider pitch), and
+    the second projection's backward skips dX.  Results equal separate calls bit for bit."""
+    counts = [257, 1, 0, 640]
+    r1, r2 = np.array([4, 16, 8, 1]), np.array([200, 3, 64, 33])
+    p1 = wl.make_problem("l1", "bf16", 320, 512, r1, counts, 2.0 * r1, wl.init_llm(320), 1401)
+    p2 = wl.make_problem("l2", "bf16", 768, 264, r2, counts, 2.0 * r2, wl.init_llm(768), 1402)
+    d1, d2 = DeviceProblem(p1), DeviceProblem(p2)
+    layer = pl.PackedLoRALayer([(320, 512), (768, 264)], max_adapters=4, max_rank=200, max_tokens=p1.T)
+    io = [{"X": d.X, "W": d.W, "A": d.A, "B": d.B, "dY": d.dY} for d in (d1, d2)]
+    scales = [p1.scales, p2.scales]          # alpha / r per adapter differs between the projections
+    fw = layer.forward(io, p1.off, scales)
+    bw1 = layer.backward(io, p1.off, scales, [s for _, s in fw])
+    torch.cuda.synchronize()
+    assert layer.check() == pl.PLORA_OK
+    for k, (p, d) in enumerate(((p1, d1), (p2, d2))):
+        eng = pl.PackedLoRA(p.d_in, p.d_out, "bf16", max_adapters=4, max_rank=200, max_tokens=p.T)
+        Y1, s1 = eng.forward(d.X, d.W, p1.off, p.scales, d.A, d.B)
+        dX1, dA1, dB1 = eng.backward(d.X, d.W, d.dY, p1.off, p.scales, d.A, d.B, s1)
+        torch.cuda.synchronize()
+        assert torch.equal(fw[k][0], Y1), k
+        assert torch.equal(bw1[k][0], dX1), k
+        for i in range(4):
+            assert torch.equal(bw1[k][1][i], dA1[i]) and torch.equal(bw1[k][2][i], dB1[i]), (k, i)
+        eng.close()
+    # a backward that skips every dX gives the same weight gradients
+    bw2 = layer.backward(io, p1.off, scales, [s for _, s in fw], want_dX=False)
+    torch.cuda.synchronize()
+    assert layer.check() == pl.PLORA_OK
+    for k in range(2):
+        assert bw2[k][0] is None
+        for i in range(4):
+            assert torch.equal(bw2[k][1][i], bw1[k][1][i]) and torch.equal(bw2[k][2][i], bw1[k][2][i]), (k, i)
+    layer.close()
