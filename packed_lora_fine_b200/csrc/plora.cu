@@ -720,11 +720,11 @@ cudaError_t pair_setup(int& pairs) {
 }
 
 // Pair-tile parameters of a base GEMM over T rows: 256-row m-tiles, 32 KB stages, a 6-deep ring.
-void pair_params(TcParams& p, int64_t T, int64_t N) {
+void pair_params(TcParams& p, int64_t T, int64_t N, int window_rows) {
     p.tiles_m = (int32_t)ceil_div(T, 2 * kTileM);
     p.tiles_n = (int32_t)ceil_div(N, kTileN);
     p.num_tiles = p.tiles_m * p.tiles_n;
-    p.group_m = std::max(1, p.group_m / 2);   // the same row window in 256-row pair tiles
+    p.group_m = std::max(1, window_rows / (2 * kTileM));   // the row window in 256-row pair tiles
     p.stage_bytes = kPairStageBytes;
     p.stages = std::min(kMaxStages, kRingBytes / kPairStageBytes);
 }
@@ -733,6 +733,20 @@ void pair_params(TcParams& p, int64_t T, int64_t N) {
 void narrow_ring(TcParams& p, int RP) {
     p.stage_bytes = kABytes + RP * kBlockK * 2;
     p.stages = std::min(kMaxStages, kRingBytes / p.stage_bytes);
+}
+
+// Tile geometry of a single-SM base GEMM over T rows and N output columns: kBaseRows-row m-tiles, the
+// rasterisation window in those tiles, and the ring layout of that tile (three 64 KB stages for
+// 256-row tiles).
+void base_tiles(TcParams& p, int64_t T, int64_t N, int window_rows) {
+    p.tiles_m = (int32_t)ceil_div(T, kBaseRows);
+    p.tiles_n = (int32_t)ceil_div(N, kTileN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.group_m = std::max(1, window_rows / kBaseRows);
+    if (kBaseRows == 256) {
+        p.stages = kWideStages;
+        p.stage_bytes = kWideStageBytes;
+    }
 }
 
 template <Op OP, Op OP2 = OP>
@@ -750,7 +764,6 @@ TcParams base_params(const plora_ctx* h, const HostPlan& P, const DevPlan& D) {
     p.timeout_ns = kTimeoutNs;
     p.partials = h->at<float>(h->r_part);
     p.counters = h->at<int32_t>(h->r_cnt);
-    p.group_m = kWindowRows / kTileM;   // a window of A's rows stays in L2 while W streams past it
     p.mt_rec = D.mt_rec;
     p.mt_seg = D.mt_seg;
     p.fuse = 0;
@@ -884,7 +897,7 @@ struct FwdCall {
     void* saved = nullptr;
     HostPlan P;
     DevPlan D;
-    CUtensorMap mX, mW, mW128, mPA16, mHk, mPBk, mPBk128, mY;
+    CUtensorMap mX, mXb, mW, mW128, mPA16, mHk, mHkb, mPBk, mPBk128, mY;
     TcParams q{}, p{};
 };
 
@@ -897,7 +910,8 @@ plora_status fwd_prepare(FwdCall& c, cudaStream_t st, StageCopies& cs) {
     if (s != PLORA_OK) return s;
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
     // mPA16: the A pack in 16-row boxes (the shrink's K-major B); mPBk / mPBk128: the B pack, K-major,
-    // 256 rows for the 1-SM tile and the expand, 128 per CTA of an SM pair.
+    // 256 rows for the 1-SM tile and the expand, 128 per CTA of an SM pair; mXb / mHkb: X and H' in
+    // boxes of a 1-SM base tile's rows.
     const SavedLayout L = saved_layout(h, P);
     const uint8_t* sv = static_cast<const uint8_t*>(c.saved);
     bool ok = make_map(&c.mX, c.X, d_in, P.T, d_in, 64, kTileM) &&
@@ -906,6 +920,8 @@ plora_status fwd_prepare(FwdCall& c, cudaStream_t st, StageCopies& cs) {
               make_map(&c.mW128, c.W, d_in, d_out, d_in, 64, kTileM) &&
               make_map(&c.mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
               make_map(&c.mHk, c.saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_map(&c.mXb, c.X, d_in, P.T, d_in, 64, kBaseRows) &&
+              make_map(&c.mHkb, c.saved, P.RP, P.h_rows, P.RP, 64, kBaseRows) &&
               make_packb_map(&c.mPBk, sv + L.o_packB, P.RP, d_out, P.n, kTileN) &&
               make_packb_map(&c.mPBk128, sv + L.o_packB, P.RP, d_out, P.n, kTileM);
     if (!ok) return fail(h, PLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
@@ -922,8 +938,7 @@ plora_status fwd_prepare(FwdCall& c, cudaStream_t st, StageCopies& cs) {
     TcParams& p = c.p;
     p = base_params(h, P, c.D);
     p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_out; p.K_total = (int32_t)d_in;
-    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_out, kTileN);
-    p.num_tiles = p.tiles_m * p.tiles_n;
+    base_tiles(p, P.T, d_out, kWindowRows);
     p.b_box_rows = kTileN;
     p.out = c.Y; p.out_ld = d_out;
     p.fuse = (h->cfg.flags & PLORA_FLAG_UNFUSED) ? 0 : 1;
@@ -973,10 +988,10 @@ plora_status fwd_launch(FwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
         plora_ctx* h = c.h;
         const bool fused = c.p.fuse != 0;
         if (flags & PLORA_FLAG_BASE_PAIR) {
-            pair_params(c.p, c.P.T, h->cfg.d_out);
+            pair_params(c.p, c.P.T, h->cfg.d_out, kWindowRows);
             launch_pair<Op::BaseFwd>(h, c.mX, c.mW128, c.mHk, fused ? c.mPBk128 : c.mW128, c.mY, c.p, st);
         } else {
-            launch_tc<Op::BaseFwd>(h, c.mX, c.mW, c.mHk, c.mW, c.mY, c.p, st);
+            launch_tc<Op::BaseFwd>(h, c.mXb, c.mW, c.mHkb, c.mW, c.mY, c.p, st);
         }
         if (!fused) {
             // K3 as its own pass: Y_i += H'_i B_i (read-modify-write of Y).
@@ -993,7 +1008,7 @@ plora_status fwd_launch(FwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
         S = Segments{};
         for (int k : order) {
             FwdCall& c = calls[k];
-            seg_add(S, c.p, SegMaps{&c.mX, &c.mW, &c.mHk, &c.mPBk, &c.mY}, false);
+            seg_add(S, c.p, SegMaps{&c.mXb, &c.mW, &c.mHkb, &c.mPBk, &c.mY}, false);
         }
         tracked(h0, kBaseFwd, st, [&] { launch_segments<Op::BaseFwd>(S, h0->num_sms, st); });
     }
@@ -1013,7 +1028,7 @@ struct BwdCall {
     const void* saved = nullptr;
     HostPlan P;
     DevPlan D;
-    CUtensorMap mdY_k, mdY_mn, mW_mn, mPB_mn, mG_k, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn, mdX;
+    CUtensorMap mdY_k, mdY_kb, mdY_mn, mW_mn, mPB_mn, mG_k, mG_kb, mG_mn, mPA_mn, mPA16, mH_mn, mX_mn, mdX;
     TcParams q{}, wb{}, p{}, wa{};
 };
 
@@ -1037,6 +1052,8 @@ plora_status bwd_prepare(BwdCall& c, cudaStream_t st, StageCopies& cs) {
               make_map(&c.mW_mn, c.W, d_in, d_out, d_in, 64, 64) &&
               make_packb_map(&c.mPB_mn, sv + L.o_packB, P.RP, d_out, P.n, 64) &&
               make_map(&c.mG_k, G, P.RP, P.h_rows, P.RP, 64, kTileM) &&
+              make_map(&c.mdY_kb, c.dY, d_out, P.T, d_out, 64, kBaseRows) &&   // boxes of a 1-SM base tile
+              make_map(&c.mG_kb, G, P.RP, P.h_rows, P.RP, 64, kBaseRows) &&
               make_map(&c.mG_mn, G, P.RP, P.h_rows, P.RP, 64, 64) &&
               make_map(&c.mPA_mn, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
               make_map(&c.mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
@@ -1065,9 +1082,8 @@ plora_status bwd_prepare(BwdCall& c, cudaStream_t st, StageCopies& cs) {
     TcParams& p = c.p;
     p = base_params(h, P, c.D);
     p.M_total = (int32_t)P.T; p.N_total = (int32_t)d_in; p.K_total = (int32_t)d_out;
-    p.tiles_m = (int32_t)ceil_div(P.T, kTileM); p.tiles_n = (int32_t)ceil_div(d_in, kTileN);
-    p.num_tiles = c.dX ? p.tiles_m * p.tiles_n : 0;
-    p.group_m = kDxWindowRows / kTileM;
+    base_tiles(p, P.T, d_in, kDxWindowRows);
+    if (!c.dX) p.num_tiles = 0;
     p.out = c.dX; p.out_ld = d_in;
     p.fuse = (h->cfg.flags & PLORA_FLAG_UNFUSED) ? 0 : 1;
     // K8: dA_i = X_i^T G_i (a sum over each adapter's tokens).
@@ -1106,14 +1122,14 @@ plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
         BwdCall& c = calls[0];
         plora_ctx* h = c.h;
         if (c.dX) {
-            pair_params(c.p, c.P.T, h->cfg.d_in);
+            pair_params(c.p, c.P.T, h->cfg.d_in, kDxWindowRows);
             launch_pair<Op::BaseDx>(h, c.mdY_k, c.mW_mn, c.mG_k, c.mPA16, c.mdX, c.p, st);
         }
         narrow_ring(c.wa, c.P.RP);
         launch_tc<Op::WgradA>(h, c.mX_mn, c.mG_mn, c.mX_mn, c.mG_mn, c.mX_mn, c.wa, st);
     } else {
         // K8 needs neither dX nor K6, so its items follow the dX tiles in the same persistent launch and
-        // fill its last, partial wave (on the dX GEMM's 48 KB ring, which holds them).  Without dX, K8's
+        // fill its last, partial wave (on the dX GEMM's ring, whose stages hold them).  Without dX, K8's
         // items run on their own narrow ring.
         bool any_dx = false;
         for (int k = 0; k < nc; ++k) any_dx = any_dx || calls[k].dX != nullptr;
@@ -1121,7 +1137,7 @@ plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
         if (any_dx) {
             for (int k : order) {
                 BwdCall& c = calls[k];
-                seg_add(S, c.p, SegMaps{&c.mdY_k, &c.mW_mn, &c.mG_k, &c.mPA16, &c.mdX}, false);
+                seg_add(S, c.p, SegMaps{&c.mdY_kb, &c.mW_mn, &c.mG_kb, &c.mPA16, &c.mdX}, false);
             }
             for (int k : order) {
                 BwdCall& c = calls[k];

@@ -24,10 +24,12 @@
 // item of a static persistent schedule over all SMs, so adapters of unequal
 // rank and token count share one launch (the load balancing of 算子设计).
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a 4-stage ring,
+// Warp roles (192 threads): warp 0 issues TMA loads into the operand ring,
 // warp 1 owns TMEM and issues tcgen05.mma into one of two 128x256 fp32
 // accumulators, warps 2-5 drain an accumulator (tcgen05.ld) and run the
-// op's epilogue while the next tile is being multiplied.
+// op's epilogue while the next tile is being multiplied.  A base-GEMM tile
+// is 256 x 256: its two 128-row halves use both accumulators and share each
+// k-block's B tile (see mma_wide for how the halves overlap the epilogue).
 //
 // A launch may carry a second, independent op (tc_kernel<OP, OP2>): its work
 // items follow OP's in the same persistent grid, with operands from their own
@@ -52,17 +54,7 @@ namespace plora {
 
 enum class Op : int { BaseFwd = 0, BaseDx, ShrinkX, ShrinkDy, ExpandY, ExpandDx, WgradB, WgradA };
 
-template <Op OP> struct OpTraits {
-    static constexpr bool kAmn = (OP == Op::WgradB || OP == Op::WgradA);
-    static constexpr bool kBmn = (OP == Op::BaseDx || OP == Op::ShrinkDy || OP == Op::ExpandDx ||
-                                  OP == Op::WgradB || OP == Op::WgradA);
-    static constexpr bool kBase = (OP == Op::BaseFwd || OP == Op::BaseDx);
-    static constexpr bool kShrink = (OP == Op::ShrinkX || OP == Op::ShrinkDy);
-    static constexpr bool kExpand = (OP == Op::ExpandY || OP == Op::ExpandDx);
-    static constexpr bool kWgrad = (OP == Op::WgradB || OP == Op::WgradA);
-};
-
-constexpr int kStages = 4;                        // stages of the largest (48 KB) layout
+constexpr int kStages = 4;                        // stages of the 48 KB layout (128-row A, 256-row B)
 constexpr int kMaxStages = 8;                     // ring slots when the op's stages are smaller
 constexpr int kTileN = 256;                       // N of the base / expand tiles (TMEM columns)
 constexpr int kABytes = kTileM * kBlockK * 2;     // 16 KB: 128 rows x 64 bf16
@@ -71,6 +63,31 @@ constexpr int kStageBytes = kABytes + kBBytesMax;
 constexpr int kTmemCols = 512;                    // two 256-column fp32 accumulators
 constexpr int kTcThreads = 192;
 constexpr int kRingBytes = kStages * kStageBytes; // 192 KB of operand ring
+
+// Rows of a base-GEMM tile.  256: two M = 128 accumulators share every k-block's 256 x 64 B tile, so a
+// k-block stages 64 KB of operands for 8.4 MFLOP (64 bytes per clock at the full tensor rate, within
+// what L2 delivers to an SM); the ring then holds three 64 KB stages.  128: one accumulator per tile,
+// 48 KB for 4.2 MFLOP (96 bytes per clock).
+#ifndef PLORA_BASE_TILE_ROWS
+#define PLORA_BASE_TILE_ROWS 256
+#endif
+constexpr int kBaseRows = PLORA_BASE_TILE_ROWS;
+static_assert(kBaseRows == 128 || kBaseRows == 256, "base tile rows");
+constexpr int kWideStageBytes = 2 * kABytes + kBBytesMax;   // 64 KB
+constexpr int kWideStages = kRingBytes / kWideStageBytes;   // 3
+
+template <Op OP> struct OpTraits {
+    static constexpr bool kAmn = (OP == Op::WgradB || OP == Op::WgradA);
+    static constexpr bool kBmn = (OP == Op::BaseDx || OP == Op::ShrinkDy || OP == Op::ExpandDx ||
+                                  OP == Op::WgradB || OP == Op::WgradA);
+    static constexpr bool kBase = (OP == Op::BaseFwd || OP == Op::BaseDx);
+    static constexpr bool kShrink = (OP == Op::ShrinkX || OP == Op::ShrinkDy);
+    static constexpr bool kExpand = (OP == Op::ExpandY || OP == Op::ExpandDx);
+    static constexpr bool kWgrad = (OP == Op::WgradB || OP == Op::WgradA);
+    static constexpr bool kWide = kBase && kBaseRows == 256;   // 256-row tile, two accumulators
+    static constexpr int kARows = kWide ? 256 : kTileM;        // rows of A per tile
+    static constexpr uint32_t kAStage = (uint32_t)kARows * kBlockK * 2;   // A bytes per stage
+};
 // Epilogue staging, per epilogue warp: two 4 KB buffers, each one 128-byte-swizzled TMA box of 32 rows x
 // 64 bf16 (the base GEMMs' output stores); the dB epilogue uses the same space for a 32 x 33 fp32 chunk.
 constexpr int kEpiBufBytes = 32 * 64 * 2;
@@ -147,6 +164,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {  // 
     ti.adapter = -1;
     ti.red_idx = -1;
     if constexpr (Tr::kBase) {
+        constexpr int kRows = Tr::kARows;
         // Grouped rasterisation: group_m m-tiles walk all n-tiles together.
         const int per_group = p.group_m * p.tiles_n;
         const int g = t / per_group;
@@ -157,13 +175,13 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& p, int t) {  // 
         const int nb = r / gm;
         ti.mtile = mb;
         ti.a_x = 0;
-        ti.a_y = mb * kTileM;
+        ti.a_y = mb * kRows;
         if constexpr (OP == Op::BaseFwd) { ti.b_x = 0; ti.b_y = nb * kTileN; }
         else { ti.b_x = nb * kTileN; ti.b_y = 0; ti.nb_boxes = kTileN / 64; }
         ti.kblocks = (p.K_total + kBlockK - 1) / kBlockK;
         ti.mma_n = kTileN;
-        ti.out_row = mb * kTileM;
-        ti.rows_valid = min(kTileM, p.M_total - ti.out_row);
+        ti.out_row = mb * kRows;
+        ti.rows_valid = min(kRows, p.M_total - ti.out_row);
         ti.n0 = nb * kTileN;
         ti.cols_valid = min(kTileN, p.N_total - ti.n0);
     } else if constexpr (Tr::kShrink) {
@@ -263,12 +281,13 @@ __device__ __forceinline__ MTileRec load_mtile(const TcParams& p, int t) {
     r.q0 = r.q1 = 0;
     if (OpTraits<OP>::kBase && p.fuse && t < p.num_tiles) {
         const TileInfo ti = decode_tile<OP>(p, t);
-        const int rec = ti.mtile / (kLoraTileM / kTileM);
+        constexpr int kPer = kLoraTileM / OpTraits<OP>::kARows;   // tiles per 256-row record
+        const int rec = ti.mtile / kPer;
         if (!dcheck(p.err_flag, rec >= 0 && rec < p.n_mtrec)) return r;
         r = p.mt_rec[rec];
         if (!dcheck(p.err_flag, r.q0 >= 0 && r.q0 <= r.q1 && r.q1 <= p.n_mtseg)) r.q1 = r.q0;
         // a 128-row tile reads its half of the 256-row record's rows
-        const int shift = (ti.mtile % (kLoraTileM / kTileM)) * kTileM;
+        const int shift = (ti.mtile % kPer) * kTileM;
         r.s[0].h_y += shift;
         r.s[1].h_y += shift;
         r.pad_[0] = shift;
@@ -319,8 +338,8 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
     for (int kb = 0; kb < ti.kblocks; ++kb) {
         if (!ptx::mbar_wait(&empty_bar[rp.stage], rp.phase ^ 1u, abort_flag, lim, p.err_flag)) return false;
         uint8_t* sA = smem + rp.stage * stb;
-        uint8_t* sB = sA + kABytes;
-        ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], (uint32_t)kABytes + b_bytes);
+        uint8_t* sB = sA + Tr::kAStage;
+        ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], Tr::kAStage + b_bytes);
         armed |= 1u << rp.stage;
         armed_par = (armed_par & ~(1u << rp.stage)) | (rp.phase << rp.stage);
         if constexpr (Tr::kAmn) {
@@ -349,7 +368,7 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
         // Low-rank branch folded into the same accumulator: for every adapter j whose
         // tokens overlap this m-tile, K-steps over its rank with A = its H' (or G) rows,
         // read at the tile's row offset inside j's zero-padded block (rows outside j's
-        // segment load as zeros).  B has the base B's major-ness: for Y, rows n0.. of
+        // segment load as zeros; a 256-row tile stages both halves' rows in one box).  B has the base B's major-ness: for Y, rows n0.. of
         // j's B pack (K-major, one 256 x 64 box); for dX, j's packed A (MN-major, 16-row
         // boxes so that only the rank's rows are staged).  With output blocks, Y's tile reads
         // only its block's columns of H' and of the block-diagonal B pack (K = rblk from
@@ -362,9 +381,9 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
                 const int R = min(kBlockK, kext - kb * kBlockK);
                 if (!ptx::mbar_wait(&empty_bar[rp.stage], rp.phase ^ 1u, abort_flag, lim, p.err_flag)) return false;
                 uint8_t* sA = smem + rp.stage * stb;
-                uint8_t* sB = sA + kABytes;
+                uint8_t* sB = sA + Tr::kAStage;
                 const uint32_t lb_bytes = Tr::kBmn ? 4u * (uint32_t)R * 128u : (uint32_t)kTileN * 128u;
-                ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], (uint32_t)kABytes + lb_bytes);
+                ptx::mbar_arrive_expect_tx(&full_bar[rp.stage], Tr::kAStage + lb_bytes);
                 armed |= 1u << rp.stage;
                 armed_par = (armed_par & ~(1u << rp.stage)) | (rp.phase << rp.stage);
                 ptx::tma_load_2d(sA, tmA2, &full_bar[rp.stage], hx0 + kb * kBlockK, sg.h_y);
@@ -396,8 +415,8 @@ __device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, 
     // units; shared addresses stay below 2^18 bytes, so the sum never carries out of the field).
     const uint32_t s0 = ptx::smem_u32(smem);
     const uint64_t adesc0 = Tr::kAmn ? ptx::smem_desc_sw128(s0, 8192, 1024) : ptx::smem_desc_sw128(s0, 16, 1024);
-    const uint64_t bdesc0 = Tr::kBmn ? ptx::smem_desc_sw128(s0 + kABytes, 8192, 1024)
-                                     : ptx::smem_desc_sw128(s0 + kABytes, 16, 1024);
+    const uint64_t bdesc0 = Tr::kBmn ? ptx::smem_desc_sw128(s0 + Tr::kAStage, 8192, 1024)
+                                     : ptx::smem_desc_sw128(s0 + Tr::kAStage, 16, 1024);
     constexpr uint32_t kAstep = Tr::kAmn ? 2048 / 16 : 32 / 16;
     constexpr uint32_t kBstep = Tr::kBmn ? 2048 / 16 : 32 / 16;
     for (int kb = 0; kb < ti.kblocks; ++kb) {
@@ -420,7 +439,7 @@ __device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, 
                 if (!ptx::mbar_wait(&full_bar[rp.stage], rp.phase, abort_flag, lim, p.err_flag)) return false;
                 ptx::tc_fence_after();
                 const uint32_t sA = ptx::smem_u32(smem + rp.stage * stb);
-                const uint32_t sB = sA + kABytes;
+                const uint32_t sB = sA + Tr::kAStage;
                 for (int ks = 0; ks < R / 16; ++ks) {
                     const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024)
                                                     : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
@@ -434,14 +453,151 @@ __device__ __forceinline__ bool mma_item(const TcParams& p, const TileInfo& ti, 
     return true;
 }
 
+// MMA issuer of a 256-row base tile.  Rows 0-127 (half 0) accumulate into TMEM columns b0 * 256..,
+// rows 128-255 (half 1) into b1 * 256.., and both halves multiply each stage's B tile; a stage is
+// released once both have read it.  The fold's k-blocks follow the base ones, as the producer staged
+// them (both halves fold every adapter of the 256-row record: rows outside an adapter's tokens read
+// the zero padding of its H' / G block).  Each half's products run in the order of the 128-row tile,
+// so its sums are bit-identical to it.
+//
+// The halves go k-block by k-block, except over the first and the last `nst` k-blocks (what the ring
+// holds at once), where the half-0 products of all of them go first.  At the end of a tile half 0 then
+// completes early and its accumulator drains while half 1's last k-blocks run; at the start of the next
+// tile half 0 has work queued while half 1 of the previous tile is still draining.  With both
+// accumulators in one tile, this is what keeps the epilogue off the tensor pipe's critical path.
+// aph: the parity of each accumulator's uses so far (bit b for accumulator b).
+template <Op OP>
+__device__ __forceinline__ bool mma_wide(const TcParams& p, const TileInfo& ti, const MTileRec& lr, uint8_t* smem,
+                                         int stb, int nst, uint64_t* full_bar, uint64_t* empty_bar,
+                                         uint64_t* accf_bar, uint64_t* acce_bar, int b0, uint32_t aph,
+                                         uint32_t tmem_base, RingPos& rp, volatile int* abort_flag, uint64_t lim) {
+    using Tr = OpTraits<OP>;
+    static_assert(Tr::kWide, "256-row base tiles only");
+    const uint32_t idesc = ptx::idesc_bf16_f32(kTileM, kTileN, false, Tr::kBmn);
+    const uint32_t s0 = ptx::smem_u32(smem);
+    const uint64_t adesc0 = ptx::smem_desc_sw128(s0, 16, 1024);
+    const uint64_t bdesc0 = Tr::kBmn ? ptx::smem_desc_sw128(s0 + Tr::kAStage, 8192, 1024)
+                                     : ptx::smem_desc_sw128(s0 + Tr::kAStage, 16, 1024);
+    constexpr uint32_t kBstep = Tr::kBmn ? 2048 / 16 : 32 / 16;
+    const int b1 = b0 ^ 1;
+    const uint32_t d_acc[2] = {tmem_base + (uint32_t)(b0 * kTileN), tmem_base + (uint32_t)(b1 * kTileN)};
+
+    // k-block cursor: base k-block kb < kblocks, then k-block f of fold segment q
+    struct Cur { int kb, q, f; };
+    auto kext_of = [&](int q) {
+        const LoraSeg sg = mtile_seg(p, lr, q);
+        return Tr::kBmn ? sg.rp16 : sg.rblk;
+    };
+    int nk = ti.kblocks;
+    for (int q = lr.q0; q < lr.q1; ++q) nk += (kext_of(q) + kBlockK - 1) / kBlockK;
+    auto next = [&](Cur& c) {
+        if (c.kb < ti.kblocks) {
+            if (++c.kb == ti.kblocks) { c.q = lr.q0; c.f = 0; }
+        } else if (++c.f * kBlockK >= kext_of(c.q)) {
+            ++c.q;
+            c.f = 0;
+        }
+    };
+    // the MMAs of half h over the k-block at cursor c, staged in ring stage `stage`
+    auto issue = [&](const Cur& c, int h, int stage) {
+        const uint32_t sA = s0 + (uint32_t)(stage * stb);
+        if (c.kb < ti.kblocks) {
+            const uint64_t so = (uint64_t)(((uint32_t)(stage * stb)) >> 4);
+            const uint64_t ah = (uint64_t)((uint32_t)(h * kABytes) >> 4);
+            const int steps = (c.kb == ti.kblocks - 1) ? ti.last_ksteps : 4;
+            for (int ks = 0; ks < steps; ++ks)
+                ptx::tc_mma_f16(d_acc[h], adesc0 + so + ah + (uint64_t)(ks * 2), bdesc0 + so + ks * kBstep, idesc,
+                                (c.kb | ks) ? 1u : 0u);
+        } else {
+            const int R = min(kBlockK, kext_of(c.q) - c.f * kBlockK);
+            const uint32_t sB = sA + Tr::kAStage;
+            for (int ks = 0; ks < R / 16; ++ks) {
+                const uint64_t bdesc = Tr::kBmn ? ptx::smem_desc_sw128(sB + ks * 2048, (uint32_t)R * 128u, 1024)
+                                                : ptx::smem_desc_sw128(sB + ks * 32, 16, 1024);
+                ptx::tc_mma_f16(d_acc[h], ptx::smem_desc_sw128(sA + h * kABytes + ks * 32, 16, 1024), bdesc, idesc,
+                                1u);
+            }
+        }
+    };
+    auto wait_full = [&]() {
+        if (!ptx::mbar_wait(&full_bar[rp.stage], rp.phase, abort_flag, lim, p.err_flag)) return false;
+        ptx::tc_fence_after();
+        return true;
+    };
+    auto wait_drained = [&](int b) {   // accumulator b drained by the epilogue (its previous use)
+        if (!ptx::mbar_wait(&acce_bar[b], ((aph >> b) & 1u) ^ 1u, abort_flag, lim, p.err_flag)) return false;
+        ptx::tc_fence_after();
+        return true;
+    };
+    const int head = min(nst, nk);
+    const int tail = min(nst, nk - head);
+    Cur c{0, lr.q0, 0};
+    // head: half 0 of the first `head` k-blocks, then half 1 of them
+    if (!wait_drained(b0)) return false;
+    RingPos r0 = rp;
+    Cur c0 = c;
+    for (int i = 0; i < head; ++i) {
+        if (!wait_full()) return false;
+        issue(c, 0, rp.stage);
+        next(c);
+        rp.advance(nst);
+    }
+    if (tail == 0) ptx::tc_commit(&accf_bar[b0]);
+    if (!wait_drained(b1)) return false;
+    rp = r0;
+    c = c0;
+    for (int i = 0; i < head; ++i) {
+        issue(c, 1, rp.stage);
+        ptx::tc_commit(&empty_bar[rp.stage]);
+        next(c);
+        rp.advance(nst);
+    }
+    if (tail == 0) {
+        ptx::tc_commit(&accf_bar[b1]);
+        return true;
+    }
+    // middle: both halves per k-block
+    for (int i = head; i < nk - tail; ++i) {
+        if (!wait_full()) return false;
+        issue(c, 0, rp.stage);
+        issue(c, 1, rp.stage);
+        ptx::tc_commit(&empty_bar[rp.stage]);
+        next(c);
+        rp.advance(nst);
+    }
+    // tail: half 0 of the last `tail` k-blocks (then half 0 is complete), then half 1 of them
+    r0 = rp;
+    c0 = c;
+    for (int i = 0; i < tail; ++i) {
+        if (!wait_full()) return false;
+        issue(c, 0, rp.stage);
+        next(c);
+        rp.advance(nst);
+    }
+    ptx::tc_commit(&accf_bar[b0]);
+    rp = r0;
+    c = c0;
+    for (int i = 0; i < tail; ++i) {
+        issue(c, 1, rp.stage);
+        ptx::tc_commit(&empty_bar[rp.stage]);
+        next(c);
+        rp.advance(nst);
+    }
+    ptx::tc_commit(&accf_bar[b1]);
+    return true;
+}
+
 // Base-GEMM epilogue of one epilogue warp: its 32 accumulator rows (TMEM lanes from t_row) x 256
 // columns, rounded to bf16 (nearest even) and written to rows row0.. and columns n0.. of the output
 // through its two staging buffers: per 64 columns, the lanes write their rows into a 128-byte-swizzled
 // 32 x 64 box (16-byte stores, conflict-free) and one lane issues a TMA tensor store, so whole lines
 // reach L2 and the conversion of a chunk overlaps the store of the one before.  The store clips rows
-// and columns outside the output tensor.
+// and columns outside the output tensor.  seq counts the warp's chunks over the whole launch and picks
+// the buffer, so the alternation carries across calls: a call may store an odd number of chunks (a
+// narrow last n-tile), and the next call's first chunk must not take the buffer whose store may still
+// be reading it.
 __device__ __forceinline__ void epilogue_store_tma(const CUtensorMap* tmC, uint32_t t_row, uint8_t* wbuf, int lane,
-                                                   int row0, int n0, int M_total, int N_total) {
+                                                   int row0, int n0, int M_total, int N_total, uint32_t& seq) {
     if (row0 >= M_total) return;
     const uint32_t sw = (uint32_t)(lane & 7);
     for (int ch = 0; ch < kTileN / 64; ++ch) {
@@ -451,7 +607,7 @@ __device__ __forceinline__ void epilogue_store_tma(const CUtensorMap* tmC, uint3
         ptx::tmem_ld32(t_row + ch * 64, ra);
         ptx::tmem_ld32(t_row + ch * 64 + 32, rb);
         ptx::tmem_ld_wait();
-        uint8_t* buf = wbuf + (ch & 1) * kEpiBufBytes;
+        uint8_t* buf = wbuf + (seq++ & 1u) * kEpiBufBytes;
         if (lane == 0) ptx::bulk_wait_read<1>();   // the store that last read this buffer is done
         __syncwarp();
         const uint32_t rowaddr = ptx::smem_u32(buf) + (uint32_t)lane * 128u;
@@ -478,13 +634,13 @@ __device__ __forceinline__ void epilogue_store_tma(const CUtensorMap* tmC, uint3
 // rows from TMEM at t_row and runs the op's output step.
 template <Op OP>
 __device__ __forceinline__ void epilogue_item(const TcParams& p, const TileInfo& ti, uint32_t t_row, int q, int lane,
-                                              uint8_t* wbuf, const CUtensorMap* tmC, int* red_flag) {
+                                              uint8_t* wbuf, const CUtensorMap* tmC, int* red_flag, uint32_t& epi_seq) {
     using Tr = OpTraits<OP>;
     const int row = q * 32 + lane;          // accumulator row handled by this thread
     const bool row_ok = row < ti.rows_valid;
     float* epi_stage = reinterpret_cast<float*>(wbuf);
     if constexpr (Tr::kBase) {
-        epilogue_store_tma(tmC, t_row, wbuf, lane, ti.out_row + q * 32, ti.n0, p.M_total, p.N_total);
+        epilogue_store_tma(tmC, t_row, wbuf, lane, ti.out_row + q * 32, ti.n0, p.M_total, p.N_total, epi_seq);
     } else if constexpr (Tr::kShrink) {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (int64_t)(ti.out_row + row) * p.out_ld;
         // (the TMEM loads below are warp-collective: a failed check skips this thread's stores only)
@@ -813,16 +969,25 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
         if (lane == 0) {
             RingPos rp{0, 0u};
             int abuf = 0;
-            uint32_t aphase = 0;
+            uint32_t aph = 0;    // bit b: parity of accumulator b's uses so far
             MTileRec lr_next = rec_of(blockIdx.x);
             for (int t = blockIdx.x; t < total; t += gridDim.x) {
                 const MTileRec lr = lr_next;
                 lr_next = rec_of(t + gridDim.x);
-                if (!ptx::mbar_wait(&acce_bar[abuf], aphase ^ 1u, abort_flag, lim, p0.err_flag)) break;
-                ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
                 const int j = seg_of(t);
                 const TcParams& pj = g.p[j];
+                if constexpr (Tr::kWide) {
+                    if (j < g.n_op1) {   // a 256-row base tile: both accumulators, in the order abuf, abuf ^ 1
+                        if (!mma_wide<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar,
+                                          empty_bar, accf_bar, acce_bar, abuf, aph, tmem_base, rp, abort_flag, lim))
+                            break;
+                        aph ^= 3u;
+                        continue;
+                    }
+                }
+                if (!ptx::mbar_wait(&acce_bar[abuf], ((aph >> abuf) & 1u) ^ 1u, abort_flag, lim, p0.err_flag)) break;
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
                 const bool ok = (j >= g.n_op1)
                     ? mma_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar,
                                     empty_bar, d_tmem, rp, abort_flag, lim)
@@ -830,7 +995,8 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
                                    d_tmem, rp, abort_flag, lim);
                 if (!ok) break;
                 ptx::tc_commit(&accf_bar[abuf]);
-                if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+                aph ^= 1u << abuf;
+                abuf ^= 1;
             }
             // Drain: all issued MMAs complete before TMEM is released.
             ptx::tc_commit(drain_bar);
@@ -842,23 +1008,47 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         uint8_t* wbuf = smem + kEpiOffset + q * kEpiWarpBytes;
         int abuf = 0;
-        uint32_t aphase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            if (!ptx::mbar_wait(&accf_bar[abuf], aphase, abort_flag, lim, p0.err_flag)) break;
-            ptx::tc_fence_after();
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
+        uint32_t aph = 0;        // bit b: parity of accumulator b's uses so far
+        uint32_t epi_seq = 0;    // this warp's output chunks so far (staging buffer = epi_seq & 1)
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const int j = seg_of(t);
             const TcParams& pj = g.p[j];
+            if constexpr (Tr::kWide) {
+                if (j < g.n_op1) {   // a 256-row base tile: half 0 from accumulator abuf, half 1 from abuf ^ 1
+                    const TileInfo ti = decode_tile<OP>(pj, t - g.begin[j]);
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        const int b = abuf ^ h;
+                        if (!ptx::mbar_wait(&accf_bar[b], (aph >> b) & 1u, abort_flag, lim, p0.err_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kTileN);
+                        epilogue_store_tma(&maps.m[j][4], t_row, wbuf, lane, ti.out_row + h * kTileM + q * 32, ti.n0,
+                                           pj.M_total, pj.N_total, epi_seq);
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&acce_bar[b]);
+                    }
+                    aph ^= 3u;
+                    continue;
+                }
+            }
+            if (!ptx::mbar_wait(&accf_bar[abuf], (aph >> abuf) & 1u, abort_flag, lim, p0.err_flag)) break;
+            ptx::tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
             if (j >= g.n_op1)
                 epilogue_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), t_row, q, lane, wbuf, &maps.m[j][4],
-                                   red_flag);
+                                   red_flag, epi_seq);
             else
                 epilogue_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), t_row, q, lane, wbuf, &maps.m[j][4],
-                                  red_flag);
+                                  red_flag, epi_seq);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
-            if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+            aph ^= 1u << abuf;
+            abuf ^= 1;
         }
         // Every output store has been performed before the CTA (and its staging) goes away.
         if (Tr::kBase && lane == 0) ptx::bulk_wait<0>();

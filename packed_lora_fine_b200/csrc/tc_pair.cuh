@@ -235,6 +235,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         uint8_t* wbuf = smem + kEpiOffset + q * kEpiWarpBytes;
         int abuf = 0;
         uint32_t aphase = 0;
+        uint32_t epi_seq = 0;    // this warp's output chunks so far (staging buffer = epi_seq & 1)
         for (int t = pair; t < p.num_tiles; t += npairs) {
             int mb, nb;
             tile_mn(t, mb, nb);
@@ -242,7 +243,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
             const int out_row = mb * kPairTileM + (int)crank * kTileM;
-            epilogue_store_tma(&tmC, t_row, wbuf, lane, out_row + q * 32, nb * kTileN, p.M_total, p.N_total);
+            epilogue_store_tma(&tmC, t_row, wbuf, lane, out_row + q * 32, nb * kTileN, p.M_total, p.N_total, epi_seq);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive_cluster(&acce_bar[abuf], 0);
