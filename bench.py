@@ -415,7 +415,8 @@ def main(argv=None):
                         max_tokens=T, unfused=args.unfused, base_pair=args.base_pair)
     dev_info = pl.plora_device_info(eng.h)
     base_gemm = ("SM-pair 256x256 tiles, %d co-resident pairs of %d SMs" % (dev_info["pairs_fwd"], dev_info["sms"])
-                 if args.base_pair else "1-SM 128x256 tiles on %d SMs" % dev_info["sms"])
+                 if args.base_pair else "1-SM %dx256 tiles on %d SMs, %d-row windows" %
+                 (dev_info["base_rows"], dev_info["sms"], dev_info["window_rows"]))
     tab_f = eng.table(p.scales, A, B)
     tab_b = eng.table(p.scales, A, B, dA, dB)
     saved = torch.empty(eng.saved_bytes(p.off, tab_f), dtype=torch.uint8, device=dev)

@@ -308,10 +308,11 @@ PLORA_API plora_status plora_capture_reserve(plora_handle h, int32_t n);
 PLORA_API plora_status plora_capture_release(plora_handle h);
 
 /*
- * Launch geometry of the handle's device (a diagnostic; the method itself has no such
- * call): out[0] = SMs, out[1] / out[2] = the 2-SM clusters that can be resident at once
- * for the SM-pair Y / dX base GEMMs (PLORA_FLAG_BASE_PAIR), each <= SMs / 2.  At most
- * `capacity` values are written; *count receives 3.
+ * Launch geometry of the handle's device and of this build (a diagnostic; the method itself
+ * has no such call): out[0] = SMs, out[1] / out[2] = the 2-SM clusters that can be resident at
+ * once for the SM-pair Y / dX base GEMMs (PLORA_FLAG_BASE_PAIR), each <= SMs / 2; out[3] = rows
+ * of a single-SM base-GEMM tile (256 or 128), out[4] / out[5] = the rasterisation windows of the
+ * Y / dX base GEMMs in rows.  At most `capacity` values are written; *count receives 6.
  */
 PLORA_API plora_status plora_device_info(plora_handle h, int32_t* out, int32_t capacity, int32_t* count);
 

@@ -290,11 +290,13 @@ def plora_capture_release(h: int) -> None:
 
 
 def plora_device_info(h: int) -> dict:
-    """SMs of the handle's device and the co-resident 2-SM clusters of the pair base GEMMs."""
-    out = (ctypes.c_int32 * 3)()
+    """SMs of the handle's device, the co-resident 2-SM clusters of the pair base GEMMs, and this
+    build's single-SM base-GEMM tile rows and rasterisation windows."""
+    out = (ctypes.c_int32 * 6)()
     cnt = ctypes.c_int32(0)
-    _raise(h, load().plora_device_info(h, ctypes.cast(out, ctypes.c_void_p), 3, ctypes.byref(cnt)))
-    return {"sms": int(out[0]), "pairs_fwd": int(out[1]), "pairs_dx": int(out[2])}
+    _raise(h, load().plora_device_info(h, ctypes.cast(out, ctypes.c_void_p), 6, ctypes.byref(cnt)))
+    return {"sms": int(out[0]), "pairs_fwd": int(out[1]), "pairs_dx": int(out[2]), "base_rows": int(out[3]),
+            "window_rows": int(out[4]), "dx_window_rows": int(out[5])}
 
 
 # Nominal B200 peaks for the partition cost model (dense bf16 tensor FLOP/s, HBM bytes/s); only their

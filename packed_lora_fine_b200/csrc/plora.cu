@@ -30,13 +30,15 @@ using namespace plora;
 namespace {
 
 constexpr int kSlots = 4;                   // host staging / device schedule ring depth
-// Rasterisation windows of the base GEMMs (rows of A whose tiles walk every n-tile together):
-// 4096 rows keeps X's window (32 MB for d_in = 4096) in L2 while W streams past it.
+// Rasterisation windows of the base GEMMs (rows of A whose tiles walk every n-tile together): 2048
+// rows, eight 256-row m-tiles, so that a wave of 148 tiles spans about 18 n-tiles and A's window (16 MB
+// of X for d_in = 4096) stays in L2 while W streams past it.  Measured on whole benchmark steps against
+// 1024, 4096 and 8192 rows (and mixed forward / dX windows): 2048 was the fastest.
 #ifndef PLORA_WINDOW_ROWS
-#define PLORA_WINDOW_ROWS 4096
+#define PLORA_WINDOW_ROWS 2048
 #endif
 #ifndef PLORA_DX_WINDOW_ROWS
-#define PLORA_DX_WINDOW_ROWS 4096
+#define PLORA_DX_WINDOW_ROWS 2048
 #endif
 constexpr int kWindowRows = PLORA_WINDOW_ROWS;
 constexpr int kDxWindowRows = PLORA_DX_WINDOW_ROWS;
@@ -1512,9 +1514,9 @@ plora_status plora_backward(plora_handle h, const void* X, const void* W, const 
 
 plora_status plora_device_info(plora_handle h, int32_t* out, int32_t capacity, int32_t* count) {
     if (!h || !count || capacity < 0 || (capacity > 0 && !out)) return PLORA_ERR_INVALID_ARG;
-    const int32_t v[3] = {h->num_sms, h->pairs_fwd, h->pairs_dx};
-    for (int32_t i = 0; i < 3 && i < capacity; ++i) out[i] = v[i];
-    *count = 3;
+    const int32_t v[6] = {h->num_sms, h->pairs_fwd, h->pairs_dx, kBaseRows, kWindowRows, kDxWindowRows};
+    for (int32_t i = 0; i < 6 && i < capacity; ++i) out[i] = v[i];
+    *count = 6;
     return PLORA_OK;
 }
 
