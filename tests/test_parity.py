@@ -90,6 +90,19 @@ def test_weight_grad_split_path():
     assert not bad, (bad, errs)
 
 
+def test_narrow_last_n_tile_over_many_tiles():
+    """Outputs whose last n-tile is narrower than 256 columns (d_out = 392: a 136-column last tile; dX:
+    136 columns) store an odd number of 64-column chunks per 128-row half, and 100 000 rows give every
+    SM several 256-row tiles in a row: the epilogue's staging buffers must alternate across calls, not
+    restart per call.  Full comparison with the oracle, and two runs bit-identical."""
+    p = mix(330, "bf16", 136, 392, [8, 16, 32, 4, 64], [40000, 1, 30000, 129, 29870])
+    g = run(p)
+    errs, bad = compare(p, g, full_oracle(p), BF16_TOL)
+    assert not bad, (bad, errs)
+    h = run(p)
+    assert np.array_equal(g["Y"], h["Y"]) and np.array_equal(g["dX"], h["dX"])
+
+
 def test_no_dX_gives_same_weight_grads():
     p = mix(310, "bf16", 520, 328, [1, 3, 17, 64, 100], [1, 127, 129, 0, 300])
     a, b = run(p), run(p, want_dX=False)
