@@ -103,6 +103,21 @@ def test_narrow_last_n_tile_over_many_tiles():
     assert np.array_equal(g["Y"], h["Y"]) and np.array_equal(g["dX"], h["dX"])
 
 
+@pytest.mark.parametrize("counts", [[1], [0, 129], [128, 127], [256], [200, 57], [1, 384]])
+@pytest.mark.parametrize("path", ["tc", "tc_unfused"])
+def test_row_counts_at_the_256_row_tile_edges(counts, path):
+    """Packed row counts at and around a base-GEMM tile (256 rows) and its 128-row halves: a half with no
+    rows, a single row, a full tile, one row past it.  d_in = 64 gives Y's tiles a single base k-block
+    (the whole tile fits the ring at once), d_out = 448 gives dX's seven (first, middle and last
+    k-blocks), and dX's 64 columns are one output chunk.  Full oracle comparison, with W as drawn and
+    with W = 0 (Y and dX then hold only the low-rank terms)."""
+    ranks = [16, 40][:len(counts)]
+    p = mix(340 + sum(counts), "bf16", 64, 448, ranks, counts)
+    for q in (p, wl.with_zero_W(p)):
+        errs, bad = compare(q, run(q, unfused=(path == "tc_unfused")), full_oracle(q), BF16_TOL)
+        assert not bad, (bad, errs)
+
+
 def test_no_dX_gives_same_weight_grads():
     p = mix(310, "bf16", 520, 328, [1, 3, 17, 64, 100], [1, 127, 129, 0, 300])
     a, b = run(p), run(p, want_dX=False)
