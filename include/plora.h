@@ -390,11 +390,14 @@ PLORA_API plora_status plora_grad_B_static(const plora_config* cfg, const void* 
  * job adapts several linear modules of each layer (query, key, value, output, and the MLP's gate, up
  * and down projections; "LoRA加速集成方案", cloud.baidu.com, 七 › 2. 层的选择), and PLoRA packs each
  * adapter's tokens through all of them.  Projections that read one input (q|k|v, gate|up) go in as
- * one projection with output blocks.  Each projection is a segment of every launch, with its own
- * parameters and tensor maps: a forward launches one schedule copy, one pack, one shrink and one
- * base GEMM; a backward one schedule copy, one launch of G's shrink with dB, and one of the dX GEMMs
- * with dA filling their last wave.  Results are bit for bit those of separate plora_forward /
- * plora_backward calls on the projections' handles.
+ * one projection with output blocks.  Each projection is a segment of the memory-bound launches, with its
+ * own parameters and tensor maps: a forward launches one schedule copy, one pack and one shrink for
+ * all projections, and one base GEMM per projection; a backward one schedule copy and one launch of
+ * G's shrink with dB for all projections, and per projection one dX GEMM with its dA filling the last
+ * wave (projections whose dX is skipped run their dA together).  The base GEMMs get a launch each
+ * because their tiles differ in length between projections, and one persistent launch over them would
+ * let the SMs drift apart in the tile order, at a cost in L2 reuse.  Results are bit for bit those of
+ * separate plora_forward / plora_backward calls on the projections' handles.
  *
  * The projections must not depend on each other within a call (the launch set runs them
  * concurrently): in a model, a layer call groups projections whose inputs are all ready, for example

@@ -959,7 +959,7 @@ std::vector<int> by_k(const C* calls, int nc, F k_of) {
 }
 
 // The forward of every prepared call: one schedule copy, one pack, one shrink launch, one base-GEMM
-// launch (the SM-pair and unfused variants, single calls only, keep their own launches).
+// launch per call (the SM-pair and unfused variants, single calls only, keep their own launches).
 plora_status fwd_launch(FwdCall* calls, int nc, cudaStream_t st, StageCopies& cs) {
     plora_ctx* h0 = calls[0].h;
     cudaError_t e = stage_copy_run(h0, cs, st);
@@ -1007,12 +1007,17 @@ plora_status fwd_launch(FwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
             launch_tc<Op::ExpandY>(h, c.mHk, c.mPBk, c.mHk, c.mPBk, c.mHk, r, st);
         }
     } else {
-        S = Segments{};
+        // One base-GEMM launch per call.  A persistent launch over several projections deals every
+        // SM the same number of tiles of each, except that some get one more of the first: with tiles
+        // of different lengths (K = 14336 and 4096 in a LLaMA layer), those that got one fewer start
+        // the next projection a tile early and stay ahead through it, so the tiles in flight spread
+        // over several waves and W's slices leave L2 before the window's m-tiles have all read them.
         for (int k : order) {
             FwdCall& c = calls[k];
+            S = Segments{};
             seg_add(S, c.p, SegMaps{&c.mXb, &c.mW, &c.mHkb, &c.mPBk, &c.mY}, false);
+            tracked(h0, kBaseFwd, st, [&] { launch_segments<Op::BaseFwd>(S, h0->num_sms, st); });
         }
-        tracked(h0, kBaseFwd, st, [&] { launch_segments<Op::BaseFwd>(S, h0->num_sms, st); });
     }
     for (int k = 0; k < nc; ++k) {
         const plora_status s = finish(calls[k].h, calls[k].D, st);
@@ -1099,8 +1104,8 @@ plora_status bwd_prepare(BwdCall& c, cudaStream_t st, StageCopies& cs) {
 }
 
 // The backward of every prepared call: one schedule copy, one launch of the shrink of G with dB's
-// items, one launch of the dX GEMM with dA's items filling its last wave (the SM-pair variant, single
-// calls only, keeps dA in a launch of its own; the unfused one adds its expand pass).
+// items, and per call one launch of the dX GEMM with its dA items filling its last wave (the SM-pair
+// variant, single calls only, keeps dA in a launch of its own; the unfused one adds its expand pass).
 plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs) {
     plora_ctx* h0 = calls[0].h;
     cudaError_t e = stage_copy_run(h0, cs, st);
@@ -1130,32 +1135,29 @@ plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
         narrow_ring(c.wa, c.P.RP);
         launch_tc<Op::WgradA>(h, c.mX_mn, c.mG_mn, c.mX_mn, c.mG_mn, c.mX_mn, c.wa, st);
     } else {
-        // K8 needs neither dX nor K6, so its items follow the dX tiles in the same persistent launch and
-        // fill its last, partial wave (on the dX GEMM's ring, whose stages hold them).  Without dX, K8's
-        // items run on their own narrow ring.
-        bool any_dx = false;
-        for (int k = 0; k < nc; ++k) any_dx = any_dx || calls[k].dX != nullptr;
-        S = Segments{};
-        if (any_dx) {
-            for (int k : order) {
-                BwdCall& c = calls[k];
-                seg_add(S, c.p, SegMaps{&c.mdY_kb, &c.mW_mn, &c.mG_kb, &c.mPA16, &c.mdX}, false);
-            }
-            for (int k : order) {
-                BwdCall& c = calls[k];
-                c.wa.stages = c.p.stages;
-                c.wa.stage_bytes = c.p.stage_bytes;
-                seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, true);
-            }
+        // K8 needs neither dX nor K6, so a call's dA items follow its dX tiles in the same persistent
+        // launch and fill its last, partial wave (on the dX GEMM's ring, whose stages hold them): one
+        // launch per call with dX, for the reason the forward gives.  The calls without dX run their
+        // dA items together, on a narrow ring.
+        for (int k : order) {
+            BwdCall& c = calls[k];
+            if (!c.dX) continue;
+            S = Segments{};
+            seg_add(S, c.p, SegMaps{&c.mdY_kb, &c.mW_mn, &c.mG_kb, &c.mPA16, &c.mdX}, false);
+            c.wa.stages = c.p.stages;
+            c.wa.stage_bytes = c.p.stage_bytes;
+            seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, true);
             tracked(h0, kBaseDxWgradA, st, [&] { launch_segments<Op::BaseDx, Op::WgradA>(S, h0->num_sms, st); });
-        } else {
-            for (int k = 0; k < nc; ++k) {
-                BwdCall& c = calls[k];
-                narrow_ring(c.wa, RPmax);
-                seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, false);
-            }
-            tracked(h0, kWgradA, st, [&] { launch_segments<Op::WgradA>(S, h0->num_sms, st); });
         }
+        S = Segments{};
+        for (int k : order) {
+            BwdCall& c = calls[k];
+            if (c.dX) continue;
+            narrow_ring(c.wa, RPmax);
+            seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, false);
+        }
+        if (S.g.n_op1 > 0)
+            tracked(h0, kWgradA, st, [&] { launch_segments<Op::WgradA>(S, h0->num_sms, st); });
         if (nc == 1 && (flags & PLORA_FLAG_UNFUSED) && calls[0].dX) {
             // K6 as its own pass: dX_i += G_i A_i^T (read-modify-write of dX).
             BwdCall& c = calls[0];
