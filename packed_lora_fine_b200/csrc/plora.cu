@@ -899,7 +899,7 @@ struct FwdCall {
     void* saved = nullptr;
     HostPlan P;
     DevPlan D;
-    CUtensorMap mX, mXb, mW, mW128, mPA16, mHk, mHkb, mPBk, mPBk128, mY;
+    CUtensorMap mX, mXb, mW, mW128, mPA16, mPA32, mPA64, mPA128, mHk, mHkb, mPBk, mPBk128, mY;
     TcParams q{}, p{};
 };
 
@@ -911,7 +911,8 @@ plora_status fwd_prepare(FwdCall& c, cudaStream_t st, StageCopies& cs) {
     plora_status s = upload(h, P, {}, st, c.D, &cs);
     if (s != PLORA_OK) return s;
     const int64_t d_in = h->cfg.d_in, d_out = h->cfg.d_out;
-    // mPA16: the A pack in 16-row boxes (the shrink's K-major B); mPBk / mPBk128: the B pack, K-major,
+    // mPA16 .. mPA128: the A pack in boxes of 16 to 128 rows (the shrink's K-major B, an adapter's rows
+    // in at most four copies per k-block); mPBk / mPBk128: the B pack, K-major,
     // 256 rows for the 1-SM tile and the expand, 128 per CTA of an SM pair; mXb / mHkb: X and H' in
     // boxes of a 1-SM base tile's rows.
     const SavedLayout L = saved_layout(h, P);
@@ -921,6 +922,9 @@ plora_status fwd_prepare(FwdCall& c, cudaStream_t st, StageCopies& cs) {
               make_map(&c.mW, c.W, d_in, d_out, d_in, 64, kTileN) &&
               make_map(&c.mW128, c.W, d_in, d_out, d_in, 64, kTileM) &&
               make_map(&c.mPA16, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 16) &&
+              make_map(&c.mPA32, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 32) &&
+              make_map(&c.mPA64, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 64) &&
+              make_map(&c.mPA128, sv + L.o_packA, d_in, (uint64_t)P.n * P.RP, d_in, 64, 128) &&
               make_map(&c.mHk, c.saved, P.RP, P.h_rows, P.RP, 64, kTileM) &&
               make_map(&c.mXb, c.X, d_in, P.T, d_in, 64, kBaseRows) &&
               make_map(&c.mHkb, c.saved, P.RP, P.h_rows, P.RP, 64, kBaseRows) &&
@@ -981,7 +985,7 @@ plora_status fwd_launch(FwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
     for (int k : order) {   // one narrow ring that holds every call's widest B tile
         FwdCall& c = calls[k];
         narrow_ring(c.q, RPmax);
-        seg_add(S, c.q, SegMaps{&c.mX, &c.mPA16, nullptr, nullptr, nullptr}, false);
+        seg_add(S, c.q, SegMaps{&c.mX, &c.mPA16, &c.mPA32, &c.mPA64, &c.mPA128}, false);
     }
     tracked(h0, kShrinkX, st, [&] { launch_segments<Op::ShrinkX>(S, h0->num_sms, st); });
     const uint32_t flags = h0->cfg.flags;

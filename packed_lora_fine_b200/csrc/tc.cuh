@@ -321,15 +321,20 @@ struct RingPos {
 };
 
 // Producer (one thread): TMA loads of every k-block of work item ti into the ring.  Returns
-// false when a wait ran out of time (the error flag is then set).
+// false when a wait ran out of time (the error flag is then set).  m: the segment's five tensor maps
+// (A, B, a base GEMM's fold A2 and B2, and the output C; for the shrink of H, B, A2, B2 and C are the A
+// pack in boxes of 16, 32, 64 and 128 rows).
 template <Op OP>
 __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& ti, const MTileRec& lr,
-                                             const CUtensorMap* tmA, const CUtensorMap* tmB,
-                                             const CUtensorMap* tmA2, const CUtensorMap* tmB2, uint8_t* smem,
+                                             const CUtensorMap* m, uint8_t* smem,
                                              int stb, int nst, uint64_t* full_bar, uint64_t* empty_bar,
                                              RingPos& rp, uint32_t& armed, uint32_t& armed_par,
                                              volatile int* abort_flag, uint64_t lim) {
     using Tr = OpTraits<OP>;
+    const CUtensorMap* tmA = &m[0];
+    const CUtensorMap* tmB = &m[1];
+    const CUtensorMap* tmA2 = &m[2];
+    const CUtensorMap* tmB2 = &m[3];
     uint32_t b_bytes;
     if constexpr (OP == Op::ShrinkX) b_bytes = (uint32_t)ti.mma_n * 128u;        // rp16 rows of 64
     else if constexpr (OP == Op::ExpandY) b_bytes = (uint32_t)kTileN * 128u;     // 256 rows of 64
@@ -349,8 +354,17 @@ __device__ __forceinline__ bool produce_item(const TcParams& p, const TileInfo& 
             ptx::tma_load_2d(sA, tmA, &full_bar[rp.stage], ti.a_x + kb * kBlockK, ti.a_y);
         }
         if constexpr (OP == Op::ShrinkX) {
-            for (int h = 0; h < ti.nb_boxes; ++h)
-                ptx::tma_load_2d(sB + h * 2048, tmB, &full_bar[rp.stage], kb * kBlockK, ti.b_y + 16 * h);
+            // the adapter's rp16 rows as boxes of 128, 64, 32 and 16 rows (m[4], m[3], m[2], m[1]):
+            // at most four copies of exactly its rows (16-row boxes alone took up to eight, and the
+            // copies, more than their bytes, set this launch's rate)
+            int r0 = 0;
+            for (int lg = 3; lg >= 0; --lg) {
+                const int box = 16 << lg;
+                while (ti.mma_n - r0 >= box) {
+                    ptx::tma_load_2d(sB + r0 * 128, &m[1 + lg], &full_bar[rp.stage], kb * kBlockK, ti.b_y + r0);
+                    r0 += box;
+                }
+            }
         } else if constexpr (OP == Op::ShrinkDy) {
             for (int h = 0; h < ti.nb_boxes; ++h)
                 ptx::tma_load_3d(sB + h * 8192, tmB, &full_bar[rp.stage], 64 * h, kb * kBlockK, ti.b_z);
@@ -951,11 +965,11 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
                 const CUtensorMap* m = maps.m[j];
                 const TcParams& pj = g.p[j];
                 if (j >= g.n_op1)
-                    ok = produce_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), lr, &m[0], &m[1], &m[2], &m[3],
-                                           smem, stb, nst, full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
+                    ok = produce_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), lr, m, smem, stb, nst, full_bar,
+                                           empty_bar, rp, armed, armed_par, abort_flag, lim);
                 else
-                    ok = produce_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, &m[0], &m[1], &m[2], &m[3],
-                                          smem, stb, nst, full_bar, empty_bar, rp, armed, armed_par, abort_flag, lim);
+                    ok = produce_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, m, smem, stb, nst, full_bar,
+                                          empty_bar, rp, armed, armed_par, abort_flag, lim);
             }
             // Drain: every load this thread issued must have landed before the CTA exits.
             for (int s = 0; s < nst; ++s)

@@ -2,8 +2,8 @@
 schedule against the extent of the buffer it addresses, records PLORA_ERR_BOUNDS on a failure and
 skips the access, so a wrong schedule shows up as an error status, not as a fault.  This test runs the
 small-mix parity tests (every path: 1-SM and SM-pair tensor cores, unfused, SIMT bf16, fp32), the
-weight-gradient split path, many adapters in one tile, narrow last n-tiles over many tiles, output
-blocks and the allocation-free dB
+weight-gradient split path, many adapters in one tile, narrow last n-tiles over many tiles, row counts
+at the base tile's edges, output blocks, layer calls and the allocation-free dB
 entry point once more, in a child process that loads the debug build: on valid inputs no check
 fires (each run's plora_check returns PLORA_OK) and every result still matches the oracle."""
 import os
@@ -30,9 +30,11 @@ def test_parity_suite_under_the_debug_build():
                            text=True, timeout=300)
     assert which.returncode == 0 and which.stdout.strip() == "1", which.stderr
     sel = ("small_mixes or weight_grad_split or many_adapters_in_one_tile or lora_delta_with_zero_base or "
-           "narrow_last_n_tile or output_blocks_match_each_projection_alone or static_grad_B")
+           "narrow_last_n_tile or tile_edges or output_blocks_match_each_projection_alone or static_grad_B or "
+           "layer_call")
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider", "-k", sel,
-                        "tests/test_parity.py", "tests/test_out_blocks.py", "tests/test_zz_no_alloc.py"],
+                        "tests/test_parity.py", "tests/test_out_blocks.py", "tests/test_layer.py",
+                        "tests/test_zz_no_alloc.py"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)
     tail = "\n".join(r.stdout.splitlines()[-15:])
     assert r.returncode == 0, tail
