@@ -681,14 +681,20 @@ def run_base_gemm_reference(args):
 
 
 def source_sha() -> str:
-    """Hash of the kernel sources, to tell whether committed ncu counters still describe them."""
+    """Hash of the kernel sources' code (comments and blank lines left out), to tell whether committed
+    ncu counters still describe them."""
     import hashlib
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "packed_lora_fine_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode())
-            h.update(fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(f.encode())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

@@ -13,7 +13,7 @@ constexpr int kBlockK = 64;     // K elements per pipeline stage (128 bytes of b
 constexpr int kRankAlign = 64;  // the padded rank width RP of the saved/G buffers is a multiple of this
 constexpr int kSplitTokens = 16384; // weight-gradient split size along the tokens (fixed: deterministic)
 constexpr int kLoraPad = 256;       // zero rows before and after each adapter's H' / G block
-constexpr int kLoraTileM = 256;     // base-GEMM rows per overlap record (one CTA-pair tile)
+constexpr int kLoraTileM = 256;     // base-GEMM rows per overlap record (one 256-row tile, 1-SM or SM pair)
 
 constexpr int kMaxOutBlocks = 8;    // output blocks (shared-input projections stacked along d_out)
 
@@ -85,16 +85,16 @@ struct RedEntry {
 };
 static_assert(sizeof(RedEntry) == 32, "RedEntry layout");
 
-// One adapter overlapping one global 128-row tile of a base GEMM (low-rank branch folded in).
+// One adapter overlapping one 256-row record (kLoraTileM rows) of a base GEMM (low-rank branch folded in).
 struct LoraSeg {
     int32_t adapter;
-    int32_t h_y;       // H' / G row holding the tile's first token, inside the adapter's zero-padded block
+    int32_t h_y;       // H' / G row holding the record's first token, inside the adapter's zero-padded block
     int32_t rp16;      // K extent of the folded dX product (the adapter's P rblk)
     int32_t rblk;      // K extent of the folded Y product (one output block's rank, rounded up to 16)
 };
 static_assert(sizeof(LoraSeg) == 16, "LoraSeg layout");
 
-// Per global 128-row tile of a base GEMM: the range of its LoraSeg entries, with the first two
+// Per 256-row record of a base GEMM's rows: the range of its LoraSeg entries, with the first two
 // inlined so that one 48-byte load gives everything in the common case.
 struct MTileRec {
     int32_t q0, q1;    // entries mt_seg[q0 .. q1)
