@@ -417,6 +417,12 @@ plora_status check_extents(plora_ctx* h, const HostPlan& P, const plora_adapter*
 }
 
 // Copy the plan blob to the device through the staging ring. Returns device pointers.
+// Item counters of the launches that claim their second op's items (GroupParams::dyn): the
+// backward's shrink of G with dB, and its dX GEMM with dA.
+constexpr int kDynCounters = 4;
+constexpr int kDynShrinkDyWgradB = 0;
+constexpr int kDynBaseDxWgradA = 1;
+
 struct DevPlan {
     AdapterDev* ad = nullptr;
     TokTile* tok = nullptr;
@@ -424,6 +430,7 @@ struct DevPlan {
     SimtOp* ops = nullptr;
     MTileRec* mt_rec = nullptr;
     LoraSeg* mt_seg = nullptr;
+    int32_t* dyn = nullptr;   // kDynCounters item counters, zero when the call's launches start
     int slot = 0;
 };
 
@@ -536,6 +543,8 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     const size_t o_ops = put(ops.data(), ops.size() * sizeof(SimtOp));
     const size_t o_mto = put(P.mt_rec.data(), P.mt_rec.size() * sizeof(MTileRec));
     const size_t o_mtl = put(P.mt_seg.data(), P.mt_seg.size() * sizeof(LoraSeg));
+    const int32_t zeros[kDynCounters] = {};
+    const size_t o_dyn = put(zeros, sizeof(zeros));   // the schedule copy clears the item counters
     if (o > h->blob_bytes) return fail(h, PLORA_ERR_INVALID_ARG, "schedule exceeds the handle's staging size");
     uint8_t* d = sl.dev;
     if (defer) {
@@ -550,6 +559,7 @@ plora_status upload(plora_ctx* h, const HostPlan& P, const std::vector<SimtOp>& 
     D.ops = reinterpret_cast<SimtOp*>(d + o_ops);
     D.mt_rec = reinterpret_cast<MTileRec*>(d + o_mto);
     D.mt_seg = reinterpret_cast<LoraSeg*>(d + o_mtl);
+    D.dyn = reinterpret_cast<int32_t*>(d + o_dyn);
     D.slot = sl.index;
     return PLORA_OK;
 }
@@ -1127,6 +1137,7 @@ plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
         seg_add(S, c.q, SegMaps{&c.mdY_k, &c.mPB_mn, nullptr, nullptr, nullptr}, false);
         seg_add(S, c.wb, SegMaps{&c.mdY_mn, &c.mH_mn, nullptr, nullptr, nullptr}, true);
     }
+    S.g.dyn = calls[0].D.dyn + kDynShrinkDyWgradB;   // dB's items are claimed: they fill G's last wave
     tracked(h0, kShrinkDyWgradB, st, [&] { launch_segments<Op::ShrinkDy, Op::WgradB>(S, h0->num_sms, st); });
     const uint32_t flags = h0->cfg.flags;
     if (nc == 1 && (flags & PLORA_FLAG_BASE_PAIR)) {
@@ -1151,6 +1162,7 @@ plora_status bwd_launch(BwdCall* calls, int nc, cudaStream_t st, StageCopies& cs
             c.wa.stages = c.p.stages;
             c.wa.stage_bytes = c.p.stage_bytes;
             seg_add(S, c.wa, SegMaps{&c.mX_mn, &c.mG_mn, nullptr, nullptr, nullptr}, true);
+            S.g.dyn = c.D.dyn + kDynBaseDxWgradA;   // dA's items are claimed: they fill the GEMM's last wave
             tracked(h0, kBaseDxWgradA, st, [&] { launch_segments<Op::BaseDx, Op::WgradA>(S, h0->num_sms, st); });
         }
         S = Segments{};
@@ -1277,7 +1289,8 @@ plora_status plora_create(plora_handle* out, const plora_config* cfg) {
                     (size_t)round_up(red_max * (int64_t)sizeof(RedEntry), 256) +
                     (size_t)round_up(ops_max * (int64_t)sizeof(SimtOp), 256) +
                     (size_t)round_up((tok_max + 1) * (int64_t)sizeof(MTileRec), 256) +
-                    (size_t)round_up((tok_max + na) * (int64_t)sizeof(LoraSeg), 256) + 1024;
+                    (size_t)round_up((tok_max + na) * (int64_t)sizeof(LoraSeg), 256) +
+                    (size_t)round_up(kDynCounters * (int64_t)sizeof(int32_t), 256) + 1024;
     // The AdamW step's tables (segments and chunks) travel through the same staging ring.
     const int64_t adamw_chunks =
         2 * na + na * (int64_t)cfg->max_rank * (nblk * cfg->d_in + cfg->d_out) / kAdamwChunk;

@@ -97,7 +97,7 @@ static_assert(kEpiStageFloats * 4 <= kEpiWarpBytes, "dB staging fits a warp's ep
 // Layout: [operand ring][4 warps' epilogue staging][barriers], from a 1024-byte-aligned base.
 constexpr int kEpiOffset = kRingBytes;
 constexpr int kBarOffset = kRingBytes + 4 * kEpiWarpBytes;
-constexpr int kTcSmemBytes = kBarOffset + 256 /* barriers */ + 1024 /* align */;
+constexpr int kTcSmemBytes = kBarOffset + 512 /* barriers, flags, item queue */ + 1024 /* align */;
 static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
 
 struct TcParams {
@@ -877,8 +877,12 @@ constexpr int kMaxSeg = 16;
 struct GroupParams {
     int32_t n_seg, n_op1;
     int32_t begin[kMaxSeg + 1];
+    // With a second op, a counter that starts at zero (the call's schedule copy clears it): its items
+    // are then claimed one at a time (nullptr: every item dealt round-robin).
+    int32_t* dyn;
     TcParams p[kMaxSeg];
 };
+constexpr int kItemQ = 4;   // item queue slots (producer -> MMA and epilogue roles) for claimed items
 struct GroupMaps {
     CUtensorMap m[kMaxSeg][5];
 };
@@ -898,11 +902,21 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
     uint64_t* accf_bar = bars + 2 * kMaxStages;      // [2]
     uint64_t* acce_bar = bars + 2 * kMaxStages + 2;  // [2]
     uint64_t* drain_bar = bars + 2 * kMaxStages + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 5);
+    uint64_t* itemf_bar = bars + 2 * kMaxStages + 5;             // [kItemQ] a claimed item is published
+    uint64_t* iteme_bar = bars + 2 * kMaxStages + 5 + kItemQ;    // [kItemQ] its slot has been read
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kMaxStages + 5 + 2 * kItemQ);
     const int nst = p0.stages;                       // ring depth of this launch
     const int stb = p0.stage_bytes;                  // bytes per stage (multiple of 1024)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* red_flag = reinterpret_cast<int*>(tmem_slot + 2);
+    volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(tmem_slot + 4);   // [kItemQ]
+    // Items [0, n_static) are dealt round-robin over the CTAs.  With g.dyn, the second op's items
+    // [n_static, total) are claimed one at a time once a CTA's share of the first op is done, so the
+    // CTAs that hold no item of the first op's last, partial wave take more of them.  The producer
+    // claims and publishes each item; the MMA and epilogue roles read the same sequence.  Which CTA
+    // runs an item changes no result: every item is computed on its own.
+    const bool dyn = OP2 != OP && g.dyn != nullptr && g.n_seg > g.n_op1;
+    const int n_static = dyn ? g.begin[g.n_op1] : total;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -932,6 +946,10 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
             ptx::mbar_init(&acce_bar[b], 4);
         }
         ptx::mbar_init(drain_bar, 1);
+        for (int s = 0; s < kItemQ; ++s) {
+            ptx::mbar_init(&itemf_bar[s], 1);
+            ptx::mbar_init(&iteme_bar[s], 5);   // the MMA lane and the four epilogue warps
+        }
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -958,7 +976,7 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
             bool ok = true;
             // The folded low-rank record of a base tile is fetched one tile ahead.
             MTileRec lr_next = rec_of(blockIdx.x);
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = blockIdx.x; t < n_static && ok; t += gridDim.x) {
                 const MTileRec lr = lr_next;
                 lr_next = rec_of(t + gridDim.x);
                 const int j = seg_of(t);
@@ -970,6 +988,24 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
                 else
                     ok = produce_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, m, smem, stb, nst, full_bar,
                                           empty_bar, rp, armed, armed_par, abort_flag, lim);
+            }
+            if (dyn && ok) {
+                int qs = 0;
+                uint32_t qph = 0;
+                for (;;) {
+                    const int idx = atomicAdd(g.dyn, 1);
+                    const int t = idx < total - n_static ? n_static + idx : -1;   // -1: no items left
+                    if (!ptx::mbar_wait(&iteme_bar[qs], qph ^ 1u, abort_flag, lim, p0.err_flag)) break;
+                    item_q[qs] = t;
+                    ptx::mbar_arrive(&itemf_bar[qs]);
+                    if (++qs == kItemQ) { qs = 0; qph ^= 1u; }
+                    if (t < 0) break;
+                    const int j = seg_of(t);
+                    if (!produce_item<OP2>(g.p[j], decode_tile<OP2>(g.p[j], t - g.begin[j]), MTileRec{}, maps.m[j],
+                                           smem, stb, nst, full_bar, empty_bar, rp, armed, armed_par, abort_flag,
+                                           lim))
+                        break;
+                }
             }
             // Drain: every load this thread issued must have landed before the CTA exits.
             for (int s = 0; s < nst; ++s)
@@ -984,8 +1020,9 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
             RingPos rp{0, 0u};
             int abuf = 0;
             uint32_t aph = 0;    // bit b: parity of accumulator b's uses so far
+            bool ok = true;
             MTileRec lr_next = rec_of(blockIdx.x);
-            for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            for (int t = blockIdx.x; t < n_static; t += gridDim.x) {
                 const MTileRec lr = lr_next;
                 lr_next = rec_of(t + gridDim.x);
                 const int j = seg_of(t);
@@ -993,16 +1030,21 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
                 if constexpr (Tr::kWide) {
                     if (j < g.n_op1) {   // a 256-row base tile: both accumulators, in the order abuf, abuf ^ 1
                         if (!mma_wide<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar,
-                                          empty_bar, accf_bar, acce_bar, abuf, aph, tmem_base, rp, abort_flag, lim))
+                                          empty_bar, accf_bar, acce_bar, abuf, aph, tmem_base, rp, abort_flag, lim)) {
+                            ok = false;
                             break;
+                        }
                         aph ^= 3u;
                         continue;
                     }
                 }
-                if (!ptx::mbar_wait(&acce_bar[abuf], ((aph >> abuf) & 1u) ^ 1u, abort_flag, lim, p0.err_flag)) break;
+                if (!ptx::mbar_wait(&acce_bar[abuf], ((aph >> abuf) & 1u) ^ 1u, abort_flag, lim, p0.err_flag)) {
+                    ok = false;
+                    break;
+                }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(abuf * kTileN);
-                const bool ok = (j >= g.n_op1)
+                ok = (j >= g.n_op1)
                     ? mma_item<OP2>(pj, decode_tile<OP2>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar,
                                     empty_bar, d_tmem, rp, abort_flag, lim)
                     : mma_item<OP>(pj, decode_tile<OP>(pj, t - g.begin[j]), lr, smem, stb, nst, full_bar, empty_bar,
@@ -1011,6 +1053,26 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
                 ptx::tc_commit(&accf_bar[abuf]);
                 aph ^= 1u << abuf;
                 abuf ^= 1;
+            }
+            if (dyn && ok) {
+                int qs = 0;
+                uint32_t qph = 0;
+                for (;;) {
+                    if (!ptx::mbar_wait(&itemf_bar[qs], qph, abort_flag, lim, p0.err_flag)) break;
+                    const int t = item_q[qs];
+                    ptx::mbar_arrive(&iteme_bar[qs]);
+                    if (++qs == kItemQ) { qs = 0; qph ^= 1u; }
+                    if (t < 0) break;
+                    if (!ptx::mbar_wait(&acce_bar[abuf], ((aph >> abuf) & 1u) ^ 1u, abort_flag, lim, p0.err_flag)) break;
+                    ptx::tc_fence_after();
+                    const int j = seg_of(t);
+                    if (!mma_item<OP2>(g.p[j], decode_tile<OP2>(g.p[j], t - g.begin[j]), MTileRec{}, smem, stb, nst,
+                                       full_bar, empty_bar, tmem_base + (uint32_t)(abuf * kTileN), rp, abort_flag, lim))
+                        break;
+                    ptx::tc_commit(&accf_bar[abuf]);
+                    aph ^= 1u << abuf;
+                    abuf ^= 1;
+                }
             }
             // Drain: all issued MMAs complete before TMEM is released.
             ptx::tc_commit(drain_bar);
@@ -1025,7 +1087,7 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
         uint32_t aph = 0;        // bit b: parity of accumulator b's uses so far
         uint32_t epi_seq = 0;    // this warp's output chunks so far (staging buffer = epi_seq & 1)
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = blockIdx.x; t < n_static && ok; t += gridDim.x) {
             const int j = seg_of(t);
             const TcParams& pj = g.p[j];
             if constexpr (Tr::kWide) {
@@ -1049,7 +1111,10 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
                     continue;
                 }
             }
-            if (!ptx::mbar_wait(&accf_bar[abuf], (aph >> abuf) & 1u, abort_flag, lim, p0.err_flag)) break;
+            if (!ptx::mbar_wait(&accf_bar[abuf], (aph >> abuf) & 1u, abort_flag, lim, p0.err_flag)) {
+                ok = false;
+                break;
+            }
             ptx::tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
             if (j >= g.n_op1)
@@ -1063,6 +1128,29 @@ tc_kernel(const __grid_constant__ GroupMaps maps, const __grid_constant__ GroupP
             if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
             aph ^= 1u << abuf;
             abuf ^= 1;
+        }
+        if (dyn && ok) {
+            int qs = 0;
+            uint32_t qph = 0;
+            for (;;) {
+                if (!ptx::mbar_wait(&itemf_bar[qs], qph, abort_flag, lim, p0.err_flag)) break;
+                const int t = item_q[qs];
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&iteme_bar[qs]);
+                if (++qs == kItemQ) { qs = 0; qph ^= 1u; }
+                if (t < 0) break;
+                if (!ptx::mbar_wait(&accf_bar[abuf], (aph >> abuf) & 1u, abort_flag, lim, p0.err_flag)) break;
+                ptx::tc_fence_after();
+                const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(abuf * kTileN);
+                const int j = seg_of(t);
+                epilogue_item<OP2>(g.p[j], decode_tile<OP2>(g.p[j], t - g.begin[j]), t_row, q, lane, wbuf, &maps.m[j][4],
+                                   red_flag, epi_seq);
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&acce_bar[abuf]);
+                aph ^= 1u << abuf;
+                abuf ^= 1;
+            }
         }
         // Every output store has been performed before the CTA (and its staging) goes away.
         if (Tr::kBase && lane == 0) ptx::bulk_wait<0>();
