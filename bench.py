@@ -512,17 +512,26 @@ def main(argv=None):
             ach = by / (avg_ms / 1e3) / 1e9
             kernels[kind] = {"launches": cnt, "avg_ms": avg_ms, "bound": "hbm", "achieved": ach, "unit": "GB/s",
                              "frac": ach / peaks["hbm_gbs"]}
-    dom = max(kernels, key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
-    kd = kernels[dom]
-    traffic = None
+    # DRAM bytes per launch from the committed ncu captures (the 16384-token case of the LLaMA up_proj
+    # mix), scaled by this rank's tokens: X, Y and the passes over W all grow in proportion.  Only for
+    # that projection's workloads, and only while the kernel sources still hash to the captures'.
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             tr = json.load(f)
-        e = tr.get(dom)
-        if e and e.get("source_sha") == source_sha():
-            traffic = e["bytes_per_launch"]
     except Exception:
-        pass
+        tr = {}
+    sha = source_sha()
+
+    def traffic_of(kind):
+        e = tr.get(kind)
+        if not e or e.get("source_sha") != sha or args.workload not in ("llama_up32", "small"):
+            return None
+        return int(round(e["captured_bytes"] * T / 16384))
+    for kind in kernels:
+        kernels[kind]["traffic"] = traffic_of(kind)
+    dom = max(kernels, key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
+    kd = kernels[dom]
+    traffic = traffic_of(dom)
     peak_key = "bf16_tflops_sustained" if kd["bound"] == "tensor" else "hbm_gbs"
     roofline = {"bound": kd["bound"], "achieved": kd["achieved"], "peak": peaks[peak_key], "unit": kd["unit"],
                 "frac": kd["frac"], "traffic": traffic, "kernel": dom,
